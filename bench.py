@@ -1,0 +1,352 @@
+#!/usr/bin/env python
+"""Throughput of the SO(2) edge convolution, forward + backward, on B200.
+
+One step = so2conv_forward + so2conv_backward (all five gradients) over the
+eSEN-like synthetic graph (2,000 atoms, periodic, 0.1 atoms/A^3, 30 nearest
+neighbours within 6 A -> E = 60,000 edges; lmax 4, mmax 2, C 128, 16 RBFs,
+f32).  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own copy of
+the workload: independent graphs, no collective on the data path ("weak"
+scaling); the barrier and the max-over-ranks of the timed region are the only
+cross-rank steps.  ``--impl reference`` times the float64 CPU oracle on a
+bounded sample of the same workload on the host cores (rank 0 only).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from so_edge_convolution_b200 import synth  # noqa: E402
+
+METRIC = "SO(2)-conv edges/sec (fwd+bwd, lmax=4, C=128) and % of roofline"
+WORKLOAD = ("eSEN-like: N=2000 atoms periodic at 0.1/A^3, 30 nearest within 6 A (E=60000), "
+            "lmax=4, mmax=2, C=128, 16 RBFs, f32 features and weights, forward+backward")
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def mixing_flops_per_edge(L, M, ci, co):
+    f = 2 * ((L + 1) * co) * ((L + 1) * ci)
+    for m in range(1, M + 1):
+        k = L + 1 - m
+        f += 8 * (k * co) * (k * ci)
+    return f
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.ident = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.ident:
+            cmd += ["-i", self.ident]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [s.strip() for s in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world, device):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline object)
+# ---------------------------------------------------------------------------
+def oracle_sample_time(p, n_edges_sample, reps=1):
+    import oracle as O
+    torch.set_num_threads(os.cpu_count() or 1)
+    sel = np.arange(min(n_edges_sample, p.n_edges))
+    src = torch.from_numpy(p.edge_index[0, sel].copy())
+    dst = torch.from_numpy(p.edge_index[1, sel].copy())
+    vec = torch.from_numpy(p.edge_vec[sel].copy())
+    desc = O.Desc(p.lmax, p.mmax, p.c_in, p.c_out, p.n_rbf, p.rbf_cutoff)
+    args = (torch.from_numpy(p.x), src, dst, vec, torch.from_numpy(p.w),
+            torch.from_numpy(p.w_rad), torch.from_numpy(p.b_rad), desc)
+    G = torch.from_numpy(p.grad_out)
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        O.forward(*args)
+        O.backward(*args, G)
+        times.append(time.perf_counter() - t0)
+    return len(sel), times, torch.get_num_threads()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    p = synth.make_problem("esen", seed=0)
+    n = 512
+    oracle_sample_time(p, n, reps=1)  # warm caches
+    ts = []
+    for _ in range(max(args.warmup, 0)):
+        oracle_sample_time(p, n, reps=1)
+    for _ in range(args.steps):
+        _, t, cores = oracle_sample_time(p, n, reps=1)
+        ts += t
+    per_step = statistics.mean(ts)
+    value = n / per_step
+    sample = (f"first {n} edges (destination-major) of the eSEN-like graph per step, "
+              "float64 oracle forward+backward on the host cores")
+    line = {"metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample_edges_per_step": n},
+            "cpu_baseline": {"value": value, "unit": "edges/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "edges/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# The CUDA path
+# ---------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    from so_edge_convolution_b200 import binding as B
+    from so_edge_convolution_b200 import build
+    build.build()
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    p = synth.make_problem("esen", seed=rank)
+    E = p.n_edges
+    desc = B.make_desc(p.lmax, p.mmax, p.c_in, p.c_out, p.n_rbf, p.rbf_cutoff, B.SO2_F32)
+    host = {
+        "x": torch.from_numpy(p.x.astype(np.float32)).pin_memory(),
+        "edge_index": torch.from_numpy(p.edge_index).pin_memory(),
+        "edge_vec": torch.from_numpy(p.edge_vec.astype(np.float32)).pin_memory(),
+        "w": torch.from_numpy(p.w.astype(np.float32)).pin_memory(),
+        "w_rad": torch.from_numpy(p.w_rad.astype(np.float32)).pin_memory(),
+        "b_rad": torch.from_numpy(p.b_rad.astype(np.float32)).pin_memory(),
+        "grad_out": torch.from_numpy(p.grad_out.astype(np.float32)).pin_memory(),
+    }
+    d = {k: v.to(dev) for k, v in host.items()}
+    ws = B.Workspace(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(t):
+        out = B.forward(desc, t["x"], t["edge_index"], t["edge_vec"], t["w"], t["w_rad"],
+                        t["b_rad"], ws=ws)
+        g = B.backward(desc, t["x"], t["edge_index"], t["edge_vec"], t["w"], t["w_rad"],
+                       t["b_rad"], t["grad_out"], ws=ws)
+        return out, g
+
+    for _ in range(max(args.warmup, 3)):
+        step(d)
+    torch.cuda.synchronize()
+    st = B.check(dev, ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    # ---- device-resident timed region ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(dev) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    B.profile_enable(True)
+    launches0 = B.launch_count()
+    for k in range(args.steps):
+        flush.zero_()  # evict L2 between steps (outside the timed events)
+        starts[k].record()
+        step(d)
+        ends[k].record()
+    torch.cuda.synchronize()
+    launches = (B.launch_count() - launches0) // max(args.steps, 1)
+    B.profile_enable(False)
+    prof = B.profile_read()
+    clk = clocks.stop() if clocks else None
+    barrier(world)
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    total_ms = max_over_ranks(total_ms, world, dev)
+    ms_per_step = total_ms / args.steps
+    value = world * E * args.steps / (total_ms * 1e-3)
+
+    # ---- roofline of the dominant kernel (the tcgen05 mixing GEMM) ----
+    pk, src = peaks()
+    fpe = mixing_flops_per_edge(p.lmax, p.mmax, p.c_in, p.c_out)
+    n_gemm = sum(v[0] for v in prof.values())
+    gemm_ms = sum(v[1] for v in prof.values())
+    alg_flops = 4.0 * fpe * E * args.steps  # fwd: 1 product; bwd: 3 (recompute, transpose, weights)
+    achieved = alg_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    tf32_ratio = 1.1 / 2.25  # nominal dense TF32 / BF16 on B200
+    peak_tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * tf32_ratio
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "gemm_tc_esen_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            with open(tpath) as f:
+                traffic = json.load(f).get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": (achieved / peak_tf) if achieved else None, "traffic": traffic,
+                "kernel": "k_gemm_tc (split-bf16 x3, f32 accumulate)",
+                "peak_basis": f"{src} bf16 sustained x nominal TF32/BF16 ratio 1.1/2.25",
+                "gemm_launches_per_step": n_gemm / args.steps,
+                "gemm_ms_per_step": gemm_ms / args.steps,
+                "step_roofline_frac": (alg_flops / (total_ms * 1e-3) / 1e12) / peak_tf}
+
+    # ---- end to end through the C ABI from pinned host buffers ----
+    outs_host = None
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    e2e_s = torch.cuda.Event(enable_timing=True)
+    e2e_e = torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, args.steps // 2)
+    barrier(world)
+    torch.cuda.synchronize()
+    e2e_s.record()
+    d2h = 0
+    for _ in range(n_e2e):
+        dd = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+        out, g = step(dd)
+        res = [out] + [g[k] for k in sorted(g)]
+        if outs_host is None:
+            outs_host = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in res]
+        for hbuf, r in zip(outs_host, res):
+            hbuf.copy_(r, non_blocking=True)
+        d2h = sum(r.numel() * r.element_size() for r in res)
+    e2e_e.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e2e_s.elapsed_time(e2e_e), world, dev) / n_e2e
+    e2e = {"value": world * E / (e2e_ms * 1e-3), "unit": "edges/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    # ---- CPU oracle on a bounded sample (rank 0, one GPU only) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, ts, cores = oracle_sample_time(p, 2048, reps=1)
+        cpu = {"value": n / ts[-1], "unit": "edges/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {n} edges (destination-major) of the same graph, float64 "
+                         "oracle forward+backward, one timed run"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "edges": E, "nodes": p.n_nodes,
+                           "l2": "flushed between timed steps (256 MB write)",
+                           "parallelism": f"replicas x{world}" if world > 1 else "single"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clk}
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,250 @@
+"""Thin ctypes binding of libso2conv (include/so2conv.h) for torch tensors.
+
+Argument marshalling only: every step of the convolution runs in the
+library's CUDA kernels.  Torch supplies device memory (inputs, outputs and
+the workspace) and the current stream.  If the shared library is missing or
+does not load, every call raises -- there is no fallback path.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libso2conv.so")
+
+SO2_F32, SO2_BF16 = 0, 1
+WS_FORWARD, WS_BACKWARD, WS_DOUBLE_BACKWARD = 0, 1, 2
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace",
+          4: "cuda", 5: "index", 6: "timeout", 7: "degenerate edge"}
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [("lmax", ctypes.c_int32), ("mmax", ctypes.c_int32),
+                ("c_in", ctypes.c_int32), ("c_out", ctypes.c_int32),
+                ("n_rbf", ctypes.c_int32), ("rbf_cutoff", ctypes.c_float),
+                ("dtype", ctypes.c_int32)]
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("w", ctypes.c_void_p), ("w_rad", ctypes.c_void_p),
+                ("b_rad", ctypes.c_void_p)]
+
+
+class So2Error(RuntimeError):
+    def __init__(self, code, where):
+        super().__init__(f"{where}: {STATUS.get(code, code)} (status {code})")
+        self.code = code
+
+
+_lib = None
+
+
+def load():
+    """Load libso2conv.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing; build it with "
+            "`python -m so_edge_convolution_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+    pd = ctypes.POINTER(Desc)
+    lib.so2conv_workspace_size.argtypes = [pd, i64, i64, ctypes.c_int]
+    lib.so2conv_workspace_size.restype = sz
+    lib.so2conv_num_weights.argtypes = [pd]
+    lib.so2conv_num_weights.restype = i64
+    lib.so2conv_forward.argtypes = [pd, i64, i64, vp, vp, vp, Params, vp, vp, sz, vp]
+    lib.so2conv_forward.restype = ctypes.c_int
+    lib.so2conv_backward.argtypes = [pd, i64, i64, vp, vp, vp, Params, vp, vp, vp, vp,
+                                     vp, vp, vp, sz, vp]
+    lib.so2conv_backward.restype = ctypes.c_int
+    lib.so2conv_double_backward.argtypes = [pd, i64, i64, vp, vp, vp, Params, vp, vp, vp,
+                                            vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.so2conv_double_backward.restype = ctypes.c_int
+    lib.so2conv_check.argtypes = [vp, vp]
+    lib.so2conv_check.restype = ctypes.c_int
+    lib.so2conv_status_string.argtypes = [ctypes.c_int]
+    lib.so2conv_status_string.restype = ctypes.c_char_p
+    lib.so2conv_edge_frames.argtypes = [ctypes.c_int32, i64, vp, vp, vp, vp]
+    lib.so2conv_edge_frames.restype = ctypes.c_int
+    lib.so2conv_launch_count.argtypes = []
+    lib.so2conv_launch_count.restype = ctypes.c_longlong
+    lib.so2conv_profile_enable.argtypes = [ctypes.c_int]
+    lib.so2conv_profile_enable.restype = None
+    lib.so2conv_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                         ctypes.POINTER(ctypes.c_double)]
+    lib.so2conv_profile_read.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def make_desc(lmax, mmax, c_in, c_out, n_rbf, rbf_cutoff, dtype=SO2_F32):
+    return Desc(lmax, mmax, c_in, c_out, n_rbf, float(rbf_cutoff), dtype)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check_call(code, where):
+    if code != 0:
+        raise So2Error(code, where)
+
+
+class Workspace:
+    """A reusable device workspace (grown on demand, 256-byte aligned)."""
+
+    def __init__(self, device):
+        self.device = torch.device(device)
+        self.buf = None
+
+    def get(self, nbytes):
+        if self.buf is None or self.buf.numel() < nbytes + 256:
+            self.buf = torch.empty(nbytes + 256, dtype=torch.uint8,
+                                   device=self.device)
+        base = self.buf.data_ptr()
+        off = (-base) % 256
+        return ctypes.c_void_p(base + off), nbytes
+
+
+_WS = {}
+
+
+def workspace(device):
+    key = torch.device(device)
+    if key not in _WS:
+        _WS[key] = Workspace(key)
+    return _WS[key]
+
+
+def num_weights(desc):
+    return int(load().so2conv_num_weights(ctypes.byref(desc)))
+
+
+def workspace_size(desc, n_nodes, n_edges, which):
+    return int(load().so2conv_workspace_size(ctypes.byref(desc), n_nodes, n_edges, which))
+
+
+def _wsarg(desc, n_nodes, n_edges, which, device, ws):
+    need = workspace_size(desc, n_nodes, n_edges, which)
+    if need == 0:
+        raise So2Error(2, "workspace_size")
+    w = ws or workspace(device)
+    return w.get(need)
+
+
+def forward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, out=None, ws=None):
+    lib = load()
+    N, E = x.shape[0], edge_index.shape[1]
+    if out is None:
+        out = torch.empty((N, (desc.lmax + 1) ** 2, desc.c_out), dtype=torch.float32,
+                          device=x.device)
+    p, nb = _wsarg(desc, N, E, WS_FORWARD, x.device, ws)
+    code = lib.so2conv_forward(ctypes.byref(desc), N, E, _ptr(x), _ptr(edge_index),
+                               _ptr(edge_vec), Params(w.data_ptr(), w_rad.data_ptr(),
+                                                      b_rad.data_ptr()),
+                               _ptr(out), p, nb, _stream(x.device))
+    _check_call(code, "so2conv_forward")
+    return out
+
+
+def backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, need=None,
+             ws=None):
+    """Returns a dict of gradients; `need` limits which ones are computed."""
+    lib = load()
+    N, E = x.shape[0], edge_index.shape[1]
+    names = ["grad_x", "grad_w", "grad_w_rad", "grad_b_rad", "grad_edge_vec"]
+    need = set(names if need is None else need)
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    S = (desc.lmax + 1) ** 2
+    shapes = {"grad_x": (N, S, desc.c_in), "grad_w": (num_weights(desc),),
+              "grad_w_rad": (desc.n_rbf, desc.c_out), "grad_b_rad": (desc.c_out,),
+              "grad_edge_vec": (E, 3)}
+    outs = {n: (torch.empty(shapes[n], **f32) if n in need else None) for n in names}
+    p, nb = _wsarg(desc, N, E, WS_BACKWARD, dev, ws)
+    code = lib.so2conv_backward(ctypes.byref(desc), N, E, _ptr(x), _ptr(edge_index),
+                                _ptr(edge_vec), Params(w.data_ptr(), w_rad.data_ptr(),
+                                                       b_rad.data_ptr()),
+                                _ptr(grad_out), *[_ptr(outs[n]) for n in names], p, nb,
+                                _stream(dev))
+    _check_call(code, "so2conv_backward")
+    return {n: t for n, t in outs.items() if t is not None}
+
+
+def double_backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg_x=None,
+                    gg_edge_vec=None, need=None, ws=None):
+    lib = load()
+    N, E = x.shape[0], edge_index.shape[1]
+    names = ["d_x", "d_w", "d_w_rad", "d_b_rad", "d_grad_out"]
+    need = set(names if need is None else need)
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    S = (desc.lmax + 1) ** 2
+    shapes = {"d_x": (N, S, desc.c_in), "d_w": (num_weights(desc),),
+              "d_w_rad": (desc.n_rbf, desc.c_out), "d_b_rad": (desc.c_out,),
+              "d_grad_out": (N, S, desc.c_out)}
+    outs = {n: (torch.empty(shapes[n], **f32) if n in need else None) for n in names}
+    p, nb = _wsarg(desc, N, E, WS_DOUBLE_BACKWARD, dev, ws)
+    code = lib.so2conv_double_backward(
+        ctypes.byref(desc), N, E, _ptr(x), _ptr(edge_index), _ptr(edge_vec),
+        Params(w.data_ptr(), w_rad.data_ptr(), b_rad.data_ptr()), _ptr(grad_out),
+        _ptr(gg_x), _ptr(gg_edge_vec), *[_ptr(outs[n]) for n in names], None, p, nb,
+        _stream(dev))
+    _check_call(code, "so2conv_double_backward")
+    return {n: t for n, t in outs.items() if t is not None}
+
+
+def check(device, ws=None):
+    """Synchronise and return the device status of the last call (0 = ok)."""
+    w = ws or workspace(device)
+    if w.buf is None:
+        return 0
+    base = w.buf.data_ptr()
+    return int(load().so2conv_check(ctypes.c_void_p(base + (-base) % 256),
+                                    _stream(device)))
+
+
+def edge_frames(lmax, edge_vec):
+    """Frames R [E, 3, 3] and full Wigner-D blocks [E, Dsz] as the library
+    computes them."""
+    E = edge_vec.shape[0]
+    dsz = sum((2 * l + 1) ** 2 for l in range(lmax + 1))
+    R = torch.empty((E, 9), dtype=torch.float32, device=edge_vec.device)
+    D = torch.empty((E, dsz), dtype=torch.float32, device=edge_vec.device)
+    code = load().so2conv_edge_frames(lmax, E, _ptr(edge_vec), _ptr(R), _ptr(D),
+                                      _stream(edge_vec.device))
+    _check_call(code, "so2conv_edge_frames")
+    return R.view(E, 3, 3), D
+
+
+def launch_count():
+    """Kernels launched by the library so far in this process."""
+    return int(load().so2conv_launch_count())
+
+
+def profile_enable(on=True):
+    load().so2conv_profile_enable(1 if on else 0)
+
+
+PROFILE_KINDS = {0: "mixing (x W^T)", 1: "mixing transposed (g W)", 2: "weight gradient"}
+
+
+def profile_read():
+    """{kind: (launches, total_ms)} of the recorded tensor-core launches."""
+    lib = load()
+    res = {}
+    for k in PROFILE_KINDS:
+        n, ms = ctypes.c_int(0), ctypes.c_double(0.0)
+        _check_call(lib.so2conv_profile_read(k, ctypes.byref(n), ctypes.byref(ms)),
+                    "so2conv_profile_read")
+        res[k] = (n.value, ms.value)
+    return res

@@ -1,0 +1,633 @@
+// so2conv_api.cu -- host side of libso2conv: argument checks, workspace plan,
+// tensor maps and the launch sequence of forward / backward / double
+// backward.  Every step runs in this library's own kernels; the host only
+// orchestrates on the caller's stream.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "edge_kernels.cuh"
+#include "gemm_tc.cuh"
+
+using namespace so2;
+
+namespace {
+
+constexpr int CHUNK_MAX = 8192;  // edges per chunk of per-edge intermediates
+
+// --------------------------------------------------------------------------
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda, so the library also loads on machines without a GPU).
+// --------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 matrix [rows x cols] with row stride ld (elements); box 64 x box_rows,
+// 128-byte swizzle, zero fill outside.
+bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld,
+              int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------------------------
+// Workspace plan
+// --------------------------------------------------------------------------
+struct Plan {
+  Layout y;
+  int64_t N = 0, E = 0;
+  int chunk = 0, chunkp = 0;
+  bool split = true, xbf16 = false;
+  size_t total = 0;
+  // byte offsets
+  size_t status, counts, cursor, offsets, perm, rec, geo, D, gate, wst_hi, wst_lo, wtr_hi, wtr_lo,
+      a_hi, a_lo, V, gv_hi, gv_lo, aT_hi, aT_lo, gvT_hi, gvT_lo, Ga, Gg, h, dws;
+};
+
+size_t take(size_t &cur, size_t bytes) {
+  cur = (cur + 1023) & ~static_cast<size_t>(1023);
+  const size_t at = cur;
+  cur += bytes;
+  return at;
+}
+
+bool desc_ok(const so2conv_desc *d) {
+  if (!d) return false;
+  if (d->lmax < 0 || d->lmax > LMAX_SUPPORTED) return false;
+  if (d->mmax < 0 || d->mmax > d->lmax) return false;
+  if (d->c_in < 16 || d->c_in > 512 || d->c_in % 16) return false;
+  if (d->c_out < 16 || d->c_out > 512 || d->c_out % 16) return false;
+  if (d->n_rbf < 2 || d->n_rbf > 64) return false;
+  if (!(d->rbf_cutoff > 0.f)) return false;
+  if (d->dtype != SO2_F32 && d->dtype != SO2_BF16) return false;
+  return true;
+}
+
+Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
+  Plan p;
+  p.y = make_layout(d->lmax, d->mmax, d->c_in, d->c_out, d->n_rbf);
+  p.N = N;
+  p.E = E;
+  p.split = d->dtype == SO2_F32;
+  p.xbf16 = d->dtype == SO2_BF16;
+  const int64_t ch = E < CHUNK_MAX ? E : CHUNK_MAX;
+  p.chunk = static_cast<int>(round_up(static_cast<int>(ch > 0 ? ch : 1), 128));
+  p.chunkp = p.chunk;  // multiple of 64 already
+  const Layout &y = p.y;
+  const bool bwd = which >= SO2_WS_BACKWARD;
+  const int lo = p.split ? 1 : 0;
+  size_t c = 0;
+  p.status = take(c, 256);
+  p.counts = take(c, sizeof(int) * (N + 1));
+  p.cursor = take(c, sizeof(int) * (N + 1));
+  p.offsets = take(c, sizeof(int) * (N + 1));
+  p.perm = take(c, sizeof(int) * (E > 0 ? E : 1));
+  p.rec = take(c, sizeof(EdgeRec) * p.chunk);
+  p.geo = take(c, sizeof(float) * GEO * p.chunk);
+  p.D = take(c, sizeof(float) * (size_t)y.dsz * p.chunk);
+  p.gate = take(c, sizeof(float) * (size_t)y.co * p.chunk);
+  p.wst_hi = take(c, 2ull * y.WR * y.WK);
+  p.wst_lo = take(c, 2ull * y.WR * y.WK * lo);
+  p.wtr_hi = take(c, 2ull * y.WTR * y.WTK);
+  p.wtr_lo = take(c, 2ull * y.WTR * y.WTK * lo);
+  p.a_hi = take(c, 2ull * p.chunk * y.KA);
+  p.a_lo = take(c, 2ull * p.chunk * y.KA * lo);
+  p.V = take(c, 4ull * p.chunk * y.KG);
+  if (bwd) {
+    p.gv_hi = take(c, 2ull * p.chunk * y.KG);
+    p.gv_lo = take(c, 2ull * p.chunk * y.KG * lo);
+    p.aT_hi = take(c, 2ull * y.KA * p.chunkp);
+    p.aT_lo = take(c, 2ull * y.KA * p.chunkp * lo);
+    p.gvT_hi = take(c, 2ull * y.KG * p.chunkp);
+    p.gvT_lo = take(c, 2ull * y.KG * p.chunkp * lo);
+    p.Ga = take(c, 4ull * p.chunk * y.KA);
+    p.Gg = take(c, 4ull * p.chunk * y.co);
+    p.h = take(c, 8ull * p.chunk);
+    p.dws = take(c, 4ull * y.WR * y.WK);
+  }
+  p.total = (c + 1023) & ~static_cast<size_t>(1023);
+  return p;
+}
+
+template <typename T>
+T *at(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+BlockOffsets block_offsets(const Layout &y) {
+  BlockOffsets b{};
+  long long off = 0;
+  b.off[0] = 0;
+  off += static_cast<long long>(y.Kout[0]) * y.Kin[0];
+  for (int g = 1; g < y.ng; ++g) {
+    const long long sz = static_cast<long long>((y.L + 1 - g) * y.co) * ((y.L + 1 - g) * y.ci);
+    b.off[2 * g - 1] = off;
+    off += sz;
+    b.off[2 * g] = off;
+    off += sz;
+  }
+  return b;
+}
+
+int64_t num_weights(const Layout &y) {
+  BlockOffsets b = block_offsets(y);
+  if (y.ng == 1) return static_cast<int64_t>(y.Kout[0]) * y.Kin[0];
+  const int g = y.ng - 1;
+  return b.off[2 * g] + static_cast<long long>((y.L + 1 - g) * y.co) * ((y.L + 1 - g) * y.ci);
+}
+
+#define CK(call)                                  \
+  do {                                            \
+    if ((call) != cudaSuccess) return SO2_ERR_CUDA; \
+  } while (0)
+
+// Every kernel launch of the library is counted (so2conv_launch_count).
+long long g_launches = 0;
+
+#define CKL()                                                      \
+  do {                                                             \
+    ++g_launches;                                                  \
+    if (cudaPeekAtLastError() != cudaSuccess) return SO2_ERR_CUDA; \
+  } while (0)
+
+// Optional CUDA-event timing of the tensor-core launches, by kind.
+constexpr int PROF_KINDS = 3;  // 0: products with W, 1: with W^T, 2: weight gradients
+struct Prof {
+  bool on = false;
+  std::vector<cudaEvent_t> ev[PROF_KINDS];  // start/stop pairs
+  int used[PROF_KINDS] = {0, 0, 0};
+};
+Prof g_prof;
+
+cudaEvent_t prof_event(int kind) {
+  Prof &P = g_prof;
+  if (P.used[kind] >= static_cast<int>(P.ev[kind].size())) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    P.ev[kind].push_back(e);
+  }
+  return P.ev[kind][P.used[kind]++];
+}
+
+int grid_for(int64_t n, int block) {
+  int64_t g = (n + block - 1) / block;
+  if (g < 1) g = 1;
+  if (g > 148 * 16) g = 148 * 16;
+  return static_cast<int>(g);
+}
+
+// --------------------------------------------------------------------------
+// GEMM launcher
+// --------------------------------------------------------------------------
+struct GemmLauncher {
+  GemmParams p{};
+  void add(int M, int N, int K, int a_row, int a_col, int b_row, int b_col, long long c_off,
+           int ldc) {
+    if (M <= 0 || N <= 0) return;
+    GemmGroup &g = p.g[p.n_groups++];
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.a_row = a_row;
+    g.a_col = a_col;
+    g.b_row = b_row;
+    g.b_col = b_col;
+    g.c_off = c_off;
+    g.ldc = ldc;
+    g.tiles_n = (N + GEMM_BN - 1) / GEMM_BN;
+    g.tile_begin = p.total_tiles;
+    p.total_tiles += ((M + GEMM_BM - 1) / GEMM_BM) * g.tiles_n;
+  }
+};
+
+template <int STAGES, bool SPLIT>
+cudaError_t launch_gemm_t(const CUtensorMap &a_hi, const CUtensorMap &a_lo, const CUtensorMap &b_hi,
+                          const CUtensorMap &b_lo, const GemmParams &p, cudaStream_t s) {
+  using L = GemmSmem<STAGES, SPLIT>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<STAGES, SPLIT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  k_gemm_tc<STAGES, SPLIT><<<p.total_tiles, GEMM_THREADS, L::TOTAL, s>>>(a_hi, a_lo, b_hi, b_lo, p);
+  return cudaPeekAtLastError();
+}
+
+cudaError_t launch_gemm(int kind, bool split, const CUtensorMap &a_hi, const CUtensorMap &a_lo,
+                        const CUtensorMap &b_hi, const CUtensorMap &b_lo, GemmParams p,
+                        float *C, int beta, DevStatus *st, cudaStream_t s) {
+  if (p.total_tiles == 0) return cudaSuccess;
+  p.C = C;
+  p.beta = beta;
+  p.split = split ? 1 : 0;
+  p.status = st;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (g_prof.on) {
+    e0 = prof_event(kind);
+    e1 = prof_event(kind);
+    if (e0) cudaEventRecord(e0, s);
+  }
+  ++g_launches;
+  cudaError_t r = split ? launch_gemm_t<3, true>(a_hi, a_lo, b_hi, b_lo, p, s)
+                        : launch_gemm_t<6, false>(a_hi, a_lo, b_hi, b_lo, p, s);
+  if (e1) cudaEventRecord(e1, s);
+  return r;
+}
+
+// --------------------------------------------------------------------------
+// Shared pieces of the three entry points
+// --------------------------------------------------------------------------
+struct Ctx {
+  const so2conv_desc *d;
+  Plan P;
+  void *ws;
+  cudaStream_t s;
+  DevStatus *st;
+  CUtensorMap m_a_hi, m_a_lo, m_v_hi, m_v_lo, m_wst_hi, m_wst_lo, m_wtr_hi, m_wtr_lo, m_aT_hi,
+      m_aT_lo, m_gvT_hi, m_gvT_lo;
+};
+
+so2_status common_checks(const so2conv_desc *d, int64_t N, int64_t E, const void *x,
+                         const int64_t *ei, const float *ev, so2conv_params prm, void *ws,
+                         size_t ws_bytes, int which, Plan &P) {
+  if (!desc_ok(d)) return d ? SO2_ERR_UNSUPPORTED : SO2_ERR_INVALID_ARG;
+  if (N < 0 || E < 0 || N > (1ll << 30) || E > (1ll << 30)) return SO2_ERR_INVALID_ARG;
+  if (N == 0 && E > 0) return SO2_ERR_INVALID_ARG;
+  if ((N > 0 && !x) || (E > 0 && (!ei || !ev)) || !prm.w || !prm.w_rad || !prm.b_rad)
+    return SO2_ERR_INVALID_ARG;
+  if (!ws) return SO2_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return SO2_ERR_WORKSPACE;
+  P = make_plan(d, N, E, which);
+  if (ws_bytes < P.total) return SO2_ERR_WORKSPACE;
+  return SO2_OK;
+}
+
+so2_status build_maps(Ctx &c, bool bwd) {
+  const Plan &P = c.P;
+  const Layout &y = P.y;
+  void *ws = c.ws;
+  bool ok = true;
+  ok &= make_map(&c.m_a_hi, at<void>(ws, P.a_hi), P.chunk, y.KA, y.KA, GEMM_BM);
+  ok &= make_map(&c.m_a_lo, at<void>(ws, P.split ? P.a_lo : P.a_hi), P.chunk, y.KA, y.KA, GEMM_BM);
+  ok &= make_map(&c.m_wst_hi, at<void>(ws, P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN);
+  ok &= make_map(&c.m_wst_lo, at<void>(ws, P.split ? P.wst_lo : P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN);
+  if (bwd) {
+    ok &= make_map(&c.m_v_hi, at<void>(ws, P.gv_hi), P.chunk, y.KG, y.KG, GEMM_BM);
+    ok &= make_map(&c.m_v_lo, at<void>(ws, P.split ? P.gv_lo : P.gv_hi), P.chunk, y.KG, y.KG, GEMM_BM);
+    ok &= make_map(&c.m_wtr_hi, at<void>(ws, P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN);
+    ok &= make_map(&c.m_wtr_lo, at<void>(ws, P.split ? P.wtr_lo : P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN);
+    ok &= make_map(&c.m_aT_hi, at<void>(ws, P.aT_hi), y.KA, P.chunkp, P.chunkp, GEMM_BN);
+    ok &= make_map(&c.m_aT_lo, at<void>(ws, P.split ? P.aT_lo : P.aT_hi), y.KA, P.chunkp, P.chunkp, GEMM_BN);
+    ok &= make_map(&c.m_gvT_hi, at<void>(ws, P.gvT_hi), y.KG, P.chunkp, P.chunkp, GEMM_BM);
+    ok &= make_map(&c.m_gvT_lo, at<void>(ws, P.split ? P.gvT_lo : P.gvT_hi), y.KG, P.chunkp, P.chunkp, GEMM_BM);
+  }
+  return ok ? SO2_OK : SO2_ERR_CUDA;
+}
+
+// Stable sort of edges by edge_index[key_row]; fills offsets [N+1] and perm [E].
+so2_status sort_edges(Ctx &c, const int64_t *ei, int key_row) {
+  const Plan &P = c.P;
+  int *counts = at<int>(c.ws, P.counts), *cursor = at<int>(c.ws, P.cursor);
+  int *offsets = at<int>(c.ws, P.offsets), *perm = at<int>(c.ws, P.perm);
+  CK(cudaMemsetAsync(counts, 0, sizeof(int) * (P.N + 1), c.s));
+  CK(cudaMemsetAsync(cursor, 0, sizeof(int) * (P.N + 1), c.s));
+  const int64_t *keys = ei + key_row * P.E;
+  k_count_keys<<<grid_for(P.E, 256), 256, 0, c.s>>>(keys, P.E, P.N, counts, c.st);
+  CKL();
+  k_scan_offsets<<<1, 1024, 0, c.s>>>(counts, P.N, offsets);
+  CKL();
+  k_place<<<grid_for(P.E, 256), 256, 0, c.s>>>(keys, P.E, P.N, offsets, cursor, perm);
+  CKL();
+  k_sort_segments<<<grid_for(P.N, 128), 128, 0, c.s>>>(offsets, P.N, perm);
+  CKL();
+  return SO2_OK;
+}
+
+so2_status pack_weights(Ctx &c, const void *w) {
+  const Plan &P = c.P;
+  const Layout &y = P.y;
+  __nv_bfloat16 *wh = at<__nv_bfloat16>(c.ws, P.wst_hi), *wl = P.split ? at<__nv_bfloat16>(c.ws, P.wst_lo) : nullptr;
+  __nv_bfloat16 *th = at<__nv_bfloat16>(c.ws, P.wtr_hi), *tl = P.split ? at<__nv_bfloat16>(c.ws, P.wtr_lo) : nullptr;
+  // zero padding first
+  CK(cudaMemsetAsync(wh, 0, 2ull * y.WR * y.WK, c.s));
+  CK(cudaMemsetAsync(th, 0, 2ull * y.WTR * y.WTK, c.s));
+  if (wl) CK(cudaMemsetAsync(wl, 0, 2ull * y.WR * y.WK, c.s));
+  if (tl) CK(cudaMemsetAsync(tl, 0, 2ull * y.WTR * y.WTK, c.s));
+  dim3 grid(64, y.ng);
+  BlockOffsets bo = block_offsets(y);
+  if (P.xbf16)
+    k_pack_weights<__nv_bfloat16><<<grid, 256, 0, c.s>>>(y, bo, static_cast<const __nv_bfloat16 *>(w), wh, wl, th, tl);
+  else
+    k_pack_weights<float><<<grid, 256, 0, c.s>>>(y, bo, static_cast<const float *>(w), wh, wl, th, tl);
+  CKL();
+  return SO2_OK;
+}
+
+// Per chunk: records, frames, Wigner-D, gate.
+so2_status chunk_prep(Ctx &c, int64_t e0, int M, const int64_t *ei, const float *ev, int key_row,
+                      so2conv_params prm) {
+  const Plan &P = c.P;
+  k_edge_prep<<<(M + 127) / 128, 128, 0, c.s>>>(P.y, at<int>(c.ws, P.perm), e0, M, ei, P.E, P.N,
+                                                 key_row, ev, at<EdgeRec>(c.ws, P.rec),
+                                                 at<float>(c.ws, P.geo), at<float>(c.ws, P.D), c.st);
+  CKL();
+  k_edge_gate<<<M, 128, 0, c.s>>>(P.y, c.d->rbf_cutoff, M, at<float>(c.ws, P.geo), prm.w_rad,
+                                  prm.b_rad, at<float>(c.ws, P.gate));
+  CKL();
+  return SO2_OK;
+}
+
+so2_status rotate_x(Ctx &c, int M, const void *x) {
+  const Plan &P = c.P;
+  __nv_bfloat16 *hi = at<__nv_bfloat16>(c.ws, P.a_hi), *lo = P.split ? at<__nv_bfloat16>(c.ws, P.a_lo) : nullptr;
+  if (P.xbf16)
+    k_rotate_gather<__nv_bfloat16><<<M, 128, 0, c.s>>>(P.y, M, at<EdgeRec>(c.ws, P.rec), at<float>(c.ws, P.D),
+                                                     static_cast<const __nv_bfloat16 *>(x), 0, 1, nullptr, hi, lo, P.y.KA);
+  else
+    k_rotate_gather<float><<<M, 128, 0, c.s>>>(P.y, M, at<EdgeRec>(c.ws, P.rec), at<float>(c.ws, P.D),
+                                             static_cast<const float *>(x), 0, 1, nullptr, hi, lo, P.y.KA);
+  CKL();
+  return SO2_OK;
+}
+
+// V = rotated features times stacked weights (one group per m).
+so2_status gemm_v(Ctx &c, int M) {
+  const Plan &P = c.P;
+  const Layout &y = P.y;
+  GemmLauncher L;
+  for (int g = 0; g < y.ng; ++g)
+    L.add(M, y.Kout[g], y.Kin_pad[g], 0, y.kin_off[g], y.wr_off[g], 0, y.kout_off[g], y.KG);
+  CK(launch_gemm(0, P.split, c.m_a_hi, c.m_a_lo, c.m_wst_hi, c.m_wst_lo, L.p, at<float>(c.ws, P.V), 0,
+                 c.st, c.s));
+  return SO2_OK;
+}
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+size_t so2conv_workspace_size(const so2conv_desc *desc, int64_t n_nodes, int64_t n_edges,
+                              int which) {
+  if (!desc_ok(desc) || n_nodes < 0 || n_edges < 0) return 0;
+  return make_plan(desc, n_nodes, n_edges, which).total;
+}
+
+int64_t so2conv_num_weights(const so2conv_desc *desc) {
+  if (!desc_ok(desc)) return 0;
+  return num_weights(make_layout(desc->lmax, desc->mmax, desc->c_in, desc->c_out, desc->n_rbf));
+}
+
+so2_status so2conv_forward(const so2conv_desc *desc, int64_t N, int64_t E, const void *x,
+                           const int64_t *edge_index, const float *edge_vec,
+                           so2conv_params prm, float *out, void *ws, size_t ws_bytes,
+                           so2_stream_t stream) {
+  Plan P;
+  so2_status r = common_checks(desc, N, E, x, edge_index, edge_vec, prm, ws, ws_bytes,
+                               SO2_WS_FORWARD, P);
+  if (r != SO2_OK) return r;
+  if (N > 0 && !out) return SO2_ERR_INVALID_ARG;
+  Ctx c;
+  c.d = desc;
+  c.P = P;
+  c.ws = ws;
+  c.s = reinterpret_cast<cudaStream_t>(stream);
+  c.st = at<DevStatus>(ws, P.status);
+  CK(cudaMemsetAsync(c.st, 0, sizeof(DevStatus), c.s));
+  const Layout &y = P.y;
+  if (N > 0) CK(cudaMemsetAsync(out, 0, sizeof(float) * N * y.S * y.co, c.s));
+  if (E == 0) return SO2_OK;
+  if ((r = build_maps(c, false)) != SO2_OK) return r;
+  if ((r = sort_edges(c, edge_index, 1)) != SO2_OK) return r;
+  if ((r = pack_weights(c, prm.w)) != SO2_OK) return r;
+  for (int64_t e0 = 0; e0 < E; e0 += P.chunk) {
+    const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
+    if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 1, prm)) != SO2_OK) return r;
+    if ((r = rotate_x(c, M, x)) != SO2_OK) return r;
+    if ((r = gemm_v(c, M)) != SO2_OK) return r;
+    k_scatter_nodes<<<grid_for(M, 1), y.co < 1024 ? y.co : 1024, 0, c.s>>>(
+        y, e0, M, at<EdgeRec>(ws, P.rec), at<int>(ws, P.offsets), at<float>(ws, P.D),
+        at<float>(ws, P.V), y.KG, 1, at<float>(ws, P.gate), out);
+    CKL();
+  }
+  return SO2_OK;
+}
+
+so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, const void *x,
+                            const int64_t *edge_index, const float *edge_vec,
+                            so2conv_params prm, const float *grad_out, float *grad_x,
+                            float *grad_w, float *grad_w_rad, float *grad_b_rad,
+                            float *grad_edge_vec, void *ws, size_t ws_bytes,
+                            so2_stream_t stream) {
+  Plan P;
+  so2_status r = common_checks(desc, N, E, x, edge_index, edge_vec, prm, ws, ws_bytes,
+                               SO2_WS_BACKWARD, P);
+  if (r != SO2_OK) return r;
+  if (N > 0 && !grad_out) return SO2_ERR_INVALID_ARG;
+  Ctx c;
+  c.d = desc;
+  c.P = P;
+  c.ws = ws;
+  c.s = reinterpret_cast<cudaStream_t>(stream);
+  c.st = at<DevStatus>(ws, P.status);
+  CK(cudaMemsetAsync(c.st, 0, sizeof(DevStatus), c.s));
+  const Layout &y = P.y;
+  const int64_t nw = num_weights(y);
+  if (grad_x && N > 0) CK(cudaMemsetAsync(grad_x, 0, sizeof(float) * N * y.S * y.ci, c.s));
+  if (grad_w) CK(cudaMemsetAsync(grad_w, 0, sizeof(float) * nw, c.s));
+  if (grad_w_rad) CK(cudaMemsetAsync(grad_w_rad, 0, sizeof(float) * y.nr * y.co, c.s));
+  if (grad_b_rad) CK(cudaMemsetAsync(grad_b_rad, 0, sizeof(float) * y.co, c.s));
+  if (E == 0) return SO2_OK;
+  const bool need_v = grad_edge_vec || grad_w_rad || grad_b_rad;
+  const bool need_ga = grad_x || grad_edge_vec;
+  const bool need_terms = grad_edge_vec || grad_w_rad || grad_b_rad;
+  if ((r = build_maps(c, true)) != SO2_OK) return r;
+  if ((r = sort_edges(c, edge_index, 0)) != SO2_OK) return r;
+  if ((r = pack_weights(c, prm.w)) != SO2_OK) return r;
+  float *dws = at<float>(ws, P.dws);
+  if (grad_w) CK(cudaMemsetAsync(dws, 0, 4ull * y.WR * y.WK, c.s));
+  __nv_bfloat16 *gv_hi = at<__nv_bfloat16>(ws, P.gv_hi);
+  __nv_bfloat16 *gv_lo = P.split ? at<__nv_bfloat16>(ws, P.gv_lo) : nullptr;
+  for (int64_t e0 = 0; e0 < E; e0 += P.chunk) {
+    const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
+    if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 0, prm)) != SO2_OK) return r;
+    if ((r = rotate_x(c, M, x)) != SO2_OK) return r;
+    // Gv = g * (D G[dst]) on the kept rows
+    k_rotate_gather<float><<<M, 128, 0, c.s>>>(y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
+                                             grad_out, 1, 0, at<float>(ws, P.gate), gv_hi, gv_lo, y.KG);
+    CKL();
+    if (need_v && (r = gemm_v(c, M)) != SO2_OK) return r;
+    if (need_ga) {
+      GemmLauncher L;
+      for (int g = 0; g < y.ng; ++g)
+        L.add(M, y.Kin[g], y.Kout_pad[g], 0, y.kout_off[g], y.wt_off[g], 0, y.kin_off[g], y.KA);
+      CK(launch_gemm(1, P.split, c.m_v_hi, c.m_v_lo, c.m_wtr_hi, c.m_wtr_lo, L.p, at<float>(ws, P.Ga),
+                     0, c.st, c.s));
+    }
+    if (grad_w) {
+      const int Kp = round_up(M, 64);
+      dim3 tb(32, 8);
+      k_transpose_bf16<<<dim3((y.KA + 31) / 32, (P.chunkp + 31) / 32), tb, 0, c.s>>>(
+          at<__nv_bfloat16>(ws, P.a_hi), M, y.KA, y.KA, at<__nv_bfloat16>(ws, P.aT_hi), P.chunkp);
+      CKL();
+      k_transpose_bf16<<<dim3((y.KG + 31) / 32, (P.chunkp + 31) / 32), tb, 0, c.s>>>(
+          gv_hi, M, y.KG, y.KG, at<__nv_bfloat16>(ws, P.gvT_hi), P.chunkp);
+      CKL();
+      if (P.split) {
+        k_transpose_bf16<<<dim3((y.KA + 31) / 32, (P.chunkp + 31) / 32), tb, 0, c.s>>>(
+            at<__nv_bfloat16>(ws, P.a_lo), M, y.KA, y.KA, at<__nv_bfloat16>(ws, P.aT_lo), P.chunkp);
+        CKL();
+        k_transpose_bf16<<<dim3((y.KG + 31) / 32, (P.chunkp + 31) / 32), tb, 0, c.s>>>(
+            gv_lo, M, y.KG, y.KG, at<__nv_bfloat16>(ws, P.gvT_lo), P.chunkp);
+        CKL();
+      }
+      GemmLauncher L;
+      for (int g = 0; g < y.ng; ++g)
+        L.add(y.Kout[g], y.Kin[g], Kp, y.kout_off[g], 0, y.kin_off[g], 0,
+              static_cast<long long>(y.wr_off[g]) * y.WK, y.WK);
+      CK(launch_gemm(2, P.split, c.m_gvT_hi, c.m_gvT_lo, c.m_aT_hi, c.m_aT_lo, L.p, dws, 1, c.st,
+                     c.s));
+    }
+    if (grad_x) {
+      k_scatter_nodes<<<grid_for(M, 1), y.ci < 1024 ? y.ci : 1024, 0, c.s>>>(
+          y, e0, M, at<EdgeRec>(ws, P.rec), at<int>(ws, P.offsets), at<float>(ws, P.D),
+          at<float>(ws, P.Ga), y.KA, 0, nullptr, grad_x);
+      CKL();
+    }
+    if (need_terms) {
+      if (P.xbf16)
+        k_edge_terms<__nv_bfloat16><<<M, 128, 0, c.s>>>(
+            y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), at<float>(ws, P.gate), grad_out,
+            static_cast<const __nv_bfloat16 *>(x), at<float>(ws, P.V), at<float>(ws, P.Ga),
+            at<float>(ws, P.Gg), at<float>(ws, P.h));
+      else
+        k_edge_terms<float><<<M, 128, 0, c.s>>>(
+            y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), at<float>(ws, P.gate), grad_out,
+            static_cast<const float *>(x), at<float>(ws, P.V), at<float>(ws, P.Ga),
+            at<float>(ws, P.Gg), at<float>(ws, P.h));
+      CKL();
+      if (grad_edge_vec) {
+        k_edge_final<<<(M + 3) / 4, 128, 0, c.s>>>(y, desc->rbf_cutoff, M, at<EdgeRec>(ws, P.rec),
+                                                   at<float>(ws, P.geo), at<float>(ws, P.Gg),
+                                                   at<float>(ws, P.h), prm.w_rad, grad_edge_vec);
+        CKL();
+      }
+      if (grad_w_rad || grad_b_rad) {
+        k_rad_grad<<<dim3((y.co + 31) / 32, y.nr + 1), dim3(32, 8), 0, c.s>>>(
+            y, desc->rbf_cutoff, M, at<float>(ws, P.geo), at<float>(ws, P.Gg), grad_w_rad,
+            grad_b_rad);
+        CKL();
+      }
+    }
+  }
+  if (grad_w) {
+    k_unstack_grad<<<dim3(64, y.ng), 256, 0, c.s>>>(y, block_offsets(y), dws, grad_w);
+    CKL();
+  }
+  return SO2_OK;
+}
+
+so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t E, const void *x,
+                                   const int64_t *edge_index, const float *edge_vec,
+                                   so2conv_params prm, const float *grad_out, const float *gg_x,
+                                   const float *gg_edge_vec, float *d_x, float *d_w,
+                                   float *d_w_rad, float *d_b_rad, float *d_grad_out,
+                                   float *d_edge_vec, void *ws, size_t ws_bytes,
+                                   so2_stream_t stream) {
+  (void)desc; (void)N; (void)E; (void)x; (void)edge_index; (void)edge_vec; (void)prm;
+  (void)grad_out; (void)gg_x; (void)gg_edge_vec; (void)d_x; (void)d_w; (void)d_w_rad;
+  (void)d_b_rad; (void)d_grad_out; (void)d_edge_vec; (void)ws; (void)ws_bytes; (void)stream;
+  return SO2_ERR_UNSUPPORTED;
+}
+
+so2_status so2conv_check(void *ws, so2_stream_t stream) {
+  if (!ws) return SO2_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SO2_ERR_CUDA;
+  DevStatus h{};
+  // the status word is the first thing in every workspace plan
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return SO2_ERR_CUDA;
+  if (h.code != 0) {
+    DevStatus z{};
+    if (cudaMemcpy(ws, &z, sizeof(z), cudaMemcpyHostToDevice) != cudaSuccess) return SO2_ERR_CUDA;
+  }
+  return static_cast<so2_status>(h.code);
+}
+
+long long so2conv_launch_count(void) { return g_launches; }
+
+void so2conv_profile_enable(int on) {
+  g_prof.on = on != 0;
+  for (int k = 0; k < PROF_KINDS; ++k) g_prof.used[k] = 0;
+}
+
+so2_status so2conv_profile_read(int kind, int *n_launches, double *total_ms) {
+  if (kind < 0 || kind >= PROF_KINDS || !n_launches || !total_ms) return SO2_ERR_INVALID_ARG;
+  double ms = 0.0;
+  const int n = g_prof.used[kind] / 2;
+  for (int i = 0; i < n; ++i) {
+    float t = 0.f;
+    if (cudaEventSynchronize(g_prof.ev[kind][2 * i + 1]) != cudaSuccess) return SO2_ERR_CUDA;
+    if (cudaEventElapsedTime(&t, g_prof.ev[kind][2 * i], g_prof.ev[kind][2 * i + 1]) != cudaSuccess)
+      return SO2_ERR_CUDA;
+    ms += t;
+  }
+  *n_launches = n;
+  *total_ms = ms;
+  return SO2_OK;
+}
+
+const char *so2conv_status_string(so2_status s) {
+  switch (s) {
+    case SO2_OK: return "ok";
+    case SO2_ERR_INVALID_ARG: return "invalid argument";
+    case SO2_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case SO2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SO2_ERR_CUDA: return "CUDA runtime error";
+    case SO2_ERR_INDEX: return "edge index outside [0, n_nodes)";
+    case SO2_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case SO2_ERR_DEGENERATE: return "zero-length edge vector";
+  }
+  return "unknown status";
+}
+
+so2_status so2conv_edge_frames(int32_t lmax, int64_t E, const float *edge_vec, float *R_out,
+                               float *D_out, so2_stream_t stream) {
+  if (lmax < 0 || lmax > LMAX_SUPPORTED || E < 0) return SO2_ERR_UNSUPPORTED;
+  if (E == 0) return SO2_OK;
+  if (!edge_vec) return SO2_ERR_INVALID_ARG;
+  k_frames<<<(E + 127) / 128, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(lmax, E, edge_vec,
+                                                                             R_out, D_out);
+  return cudaPeekAtLastError() == cudaSuccess ? SO2_OK : SO2_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,165 @@
+// wigner.cuh -- per-edge frame, real Wigner-D and rotation generators.
+//
+// Frame: R = R_y(-theta) R_z(-phi) for the edge direction (polar angle
+// theta, azimuth phi), so R r_hat = z_hat.  Any roll about z would do: the
+// convolution's output does not depend on it.
+//
+// Wigner-D: D^1 = P R P^T (P maps (x, y, z) to the l = 1 order (y, z, x)),
+// then D^l for l >= 2 by the Ivanic-Ruedenberg recursion (J. Phys. Chem.
+// 1996, 100, 6342; corrections 1998, 102, 9099), which builds each D^l from
+// D^1 and D^{l-1}.  This is the rotation of real spherical harmonics without
+// the Condon-Shortley phase, with Y(R n) = D(R) Y(n).
+//
+// Generators: J_x, J_y are d/dtheta D(R_{x,y}(theta)) at theta = 0 in the
+// same real basis; they couple |m| to |m| +- 1 with weights
+// s_k = sqrt((l-k)(l+k+1)) / 2 (sqrt(2) s_0 where m = 0 is involved).  With
+// them, a small turn (I + [w]x) R of the frame changes D by
+// (w_x J_x + w_y J_y + w_z J_z) D.
+#pragma once
+
+#include "common.cuh"
+
+namespace so2 {
+
+constexpr int LMAX_SUPPORTED = 6;
+
+__host__ __device__ constexpr int dblock_off(int l) { return l * (4 * l * l - 1) / 3; }
+__host__ __device__ constexpr int dsize(int lmax) { return dblock_off(lmax + 1); }
+
+struct Frame {
+  float d;
+  float rh[3];
+  float R[9];  // row-major
+};
+
+// Returns false for a zero-length vector (the frame is then the identity).
+__device__ __forceinline__ bool make_frame(float rx, float ry, float rz, Frame &f) {
+  const float d = sqrtf(rx * rx + ry * ry + rz * rz);
+  f.d = d;
+  if (!(d > 0.f)) {
+    f.rh[0] = 0.f;
+    f.rh[1] = 0.f;
+    f.rh[2] = 1.f;
+    for (int i = 0; i < 9; ++i) f.R[i] = (i % 4 == 0) ? 1.f : 0.f;
+    return false;
+  }
+  const float inv = 1.f / d;
+  const float x = rx * inv, y = ry * inv, z = rz * inv;
+  f.rh[0] = x;
+  f.rh[1] = y;
+  f.rh[2] = z;
+  const float rho = sqrtf(x * x + y * y);
+  float cp = 1.f, sp = 0.f;
+  if (rho > 0.f) {
+    cp = x / rho;
+    sp = y / rho;
+  }
+  const float ct = z, st = rho;
+  f.R[0] = ct * cp;
+  f.R[1] = ct * sp;
+  f.R[2] = -st;
+  f.R[3] = -sp;
+  f.R[4] = cp;
+  f.R[5] = 0.f;
+  f.R[6] = st * cp;
+  f.R[7] = st * sp;
+  f.R[8] = ct;
+  return true;
+}
+
+// Full blocks D^0..D^lmax, each (2l+1)^2 row-major, concatenated into D.
+__device__ inline void wigner_blocks(const float *R, int lmax, float *D) {
+  D[0] = 1.f;
+  if (lmax < 1) return;
+  // (y, z, x) ordering: sh index 0 <- y(1), 1 <- z(2), 2 <- x(0)
+  const int pm[3] = {1, 2, 0};
+  float *D1 = D + dblock_off(1);
+  for (int a = 0; a < 3; ++a)
+    for (int b = 0; b < 3; ++b) D1[a * 3 + b] = R[pm[a] * 3 + pm[b]];
+  for (int l = 2; l <= lmax; ++l) {
+    const float *Dp = D + dblock_off(l - 1);
+    float *Dl = D + dblock_off(l);
+    const int wp = 2 * l - 1;  // width of D^{l-1}
+    const int w = 2 * l + 1;
+    auto r1 = [&](int i, int j) { return D1[(i + 1) * 3 + (j + 1)]; };
+    auto rp = [&](int a, int b) { return Dp[(a + l - 1) * wp + (b + l - 1)]; };
+    auto P = [&](int i, int a, int b) -> float {
+      if (b == -l) return r1(i, 1) * rp(a, -l + 1) + r1(i, -1) * rp(a, l - 1);
+      if (b == l) return r1(i, 1) * rp(a, l - 1) - r1(i, -1) * rp(a, -l + 1);
+      return r1(i, 0) * rp(a, b);
+    };
+    for (int m = -l; m <= l; ++m) {
+      const int am = m < 0 ? -m : m;
+      const int dm0 = (m == 0);
+      for (int n = -l; n <= l; ++n) {
+        const int an = n < 0 ? -n : n;
+        const float den = (an == l) ? static_cast<float>((2 * l) * (2 * l - 1))
+                                    : static_cast<float>((l + n) * (l - n));
+        const float u = sqrtf(static_cast<float>((l + m) * (l - m)) / den);
+        const float v = 0.5f * sqrtf(static_cast<float>((1 + dm0) * (l + am - 1) * (l + am)) / den) *
+                        static_cast<float>(1 - 2 * dm0);
+        const float wc = -0.5f * sqrtf(static_cast<float>((l - am - 1) * (l - am)) / den) *
+                         static_cast<float>(1 - dm0);
+        float val = 0.f;
+        if (u != 0.f) val += u * P(0, m, n);
+        if (v != 0.f) {
+          float V;
+          if (m == 0) {
+            V = P(1, 1, n) + P(-1, -1, n);
+          } else if (m > 0) {
+            V = P(1, m - 1, n) * (m == 1 ? 1.41421356237f : 1.f) -
+                (m == 1 ? 0.f : P(-1, -m + 1, n));
+          } else {
+            V = (m == -1 ? 0.f : P(1, m + 1, n)) +
+                P(-1, -m - 1, n) * (m == -1 ? 1.41421356237f : 1.f);
+          }
+          val += v * V;
+        }
+        if (wc != 0.f) {
+          float W;
+          if (m > 0)
+            W = P(1, m + 1, n) + P(-1, -m - 1, n);
+          else
+            W = P(1, m - 1, n) - P(-1, -m + 1, n);
+          val += wc * W;
+        }
+        Dl[(m + l) * w + (n + l)] = val;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ float gen_s(int l, int k) {
+  return 0.5f * sqrtf(static_cast<float>((l - k) * (l + k + 1)));
+}
+
+// (J_x a)[m] and (J_y a)[m] for one l; `a(q)` returns the coefficient of
+// order q (only |q| <= |m| + 1 is touched).
+template <typename F>
+__device__ __forceinline__ void gen_xy(int l, int m, F a, float &jx, float &jy) {
+  const float r2 = 1.41421356237f;
+  if (l == 0) {
+    jx = 0.f;
+    jy = 0.f;
+    return;
+  }
+  if (m == 0) {
+    const float s0 = r2 * gen_s(l, 0);
+    jx = s0 * a(-1);
+    jy = -s0 * a(1);
+    return;
+  }
+  if (m > 0) {
+    const int k = m;
+    jx = (k < l ? gen_s(l, k) * a(-(k + 1)) : 0.f) + (k >= 2 ? gen_s(l, k - 1) * a(-(k - 1)) : 0.f);
+    jy = (k == 1 ? r2 * gen_s(l, 0) * a(0) : gen_s(l, k - 1) * a(k - 1)) -
+         (k < l ? gen_s(l, k) * a(k + 1) : 0.f);
+    return;
+  }
+  const int k = -m;
+  jx = (k == 1 ? -r2 * gen_s(l, 0) * a(0) : -gen_s(l, k - 1) * a(k - 1)) -
+       (k < l ? gen_s(l, k) * a(k + 1) : 0.f);
+  jy = (k >= 2 ? gen_s(l, k - 1) * a(-(k - 1)) : 0.f) - (k < l ? gen_s(l, k) * a(-(k + 1)) : 0.f);
+}
+
+}  // namespace so2

@@ -1,0 +1,94 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, sizes workspaces and rejects bad arguments before touching a device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle as O
+from so_edge_convolution_b200 import binding as B
+from so_edge_convolution_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return B.load()
+
+
+def _declared():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"^[a-z_0-9 *]+?\b(so2conv_\w+)\s*\(", txt, re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "so2conv_forward" in names and "so2conv_double_backward" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+@pytest.mark.parametrize("L,M,ci,co", [(2, 2, 16, 16), (4, 2, 128, 128), (6, 2, 128, 128),
+                                       (3, 0, 32, 48), (5, 5, 16, 32)])
+def test_num_weights_matches_layout(lib, L, M, ci, co):
+    d = B.make_desc(L, M, ci, co, 8, 5.0)
+    assert B.num_weights(d) == O.n_weights(O.Desc(L, M, ci, co, 8, 5.0))
+
+
+def test_workspace_sizes(lib):
+    d = B.make_desc(4, 2, 128, 128, 16, 6.0)
+    f = B.workspace_size(d, 2000, 60000, B.WS_FORWARD)
+    b = B.workspace_size(d, 2000, 60000, B.WS_BACKWARD)
+    assert 0 < f < b
+    assert B.workspace_size(d, 0, 0, B.WS_FORWARD) > 0
+    bad = B.make_desc(7, 2, 128, 128, 16, 6.0)
+    assert B.workspace_size(bad, 10, 10, B.WS_FORWARD) == 0
+
+
+def _fwd(lib, desc, N=4, E=3, x=1, ei=1, ev=1, w=1, ws=1, nbytes=None):
+    P = lambda f: ctypes.c_void_p(0x1000 if f else 0)  # noqa: E731 (never dereferenced)
+    prm = B.Params(0x1000 if w else 0, 0x1000, 0x1000)
+    nb = nbytes if nbytes is not None else (1 << 40)
+    return lib.so2conv_forward(ctypes.byref(desc), N, E, P(x), P(ei), P(ev), prm,
+                               ctypes.c_void_p(0x2000), ctypes.c_void_p(0x100000 if ws else 0),
+                               nb, None)
+
+
+def test_argument_errors_are_reported_before_any_launch(lib):
+    good = B.make_desc(2, 2, 16, 16, 8, 5.0)
+    assert _fwd(lib, B.make_desc(7, 2, 16, 16, 8, 5.0)) == 2       # lmax > 6
+    assert _fwd(lib, B.make_desc(2, 3, 16, 16, 8, 5.0)) == 2       # mmax > lmax
+    assert _fwd(lib, B.make_desc(2, 2, 24, 16, 8, 5.0)) == 2       # c_in % 16
+    assert _fwd(lib, B.make_desc(2, 2, 16, 16, 1, 5.0)) == 2       # n_rbf < 2
+    assert _fwd(lib, good, x=0) == 1
+    assert _fwd(lib, good, ei=0) == 1
+    assert _fwd(lib, good, w=0) == 1
+    assert _fwd(lib, good, ws=0) == 3
+    assert _fwd(lib, good, nbytes=16) == 3
+    assert _fwd(lib, good, N=-1) == 1
+    assert lib.so2conv_forward(None, 1, 1, None, None, None, B.Params(0, 0, 0), None, None, 0,
+                               None) == 1
+
+
+def test_double_backward_rejects_second_order_edge_output(lib):
+    d = B.make_desc(2, 2, 16, 16, 8, 5.0)
+    P = ctypes.c_void_p(0x1000)
+    code = lib.so2conv_double_backward(ctypes.byref(d), 4, 3, P, P, P,
+                                       B.Params(0x1000, 0x1000, 0x1000), P, None, P,
+                                       None, None, None, None, None, P,
+                                       ctypes.c_void_p(0x100000), 1 << 40, None)
+    assert code == 2
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        s = lib.so2conv_status_string(code)
+        assert s and len(s) > 1
