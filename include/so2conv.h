@@ -151,7 +151,8 @@ long long so2conv_launch_count(void);
 
 /* Live timing of the tensor-core launches.  so2conv_profile_enable(1) clears
  * the record and starts recording a pair of CUDA events around every
- * tensor-core launch, on the stream it is launched on; (0) stops recording.
+ * tensor-core launch, on the stream it is launched on; (0) stops recording
+ * and keeps the record for so2conv_profile_read.
  * so2conv_profile_read waits for the recorded events and returns, for one
  * kind (0: products with the stacked weights, 1: with their transposes,
  * 2: weight-gradient products), the number of launches and their summed

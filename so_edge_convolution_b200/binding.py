@@ -87,7 +87,15 @@ def make_desc(lmax, mmax, c_in, c_out, n_rbf, rbf_cutoff, dtype=SO2_F32):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("so2conv tensors must be contiguous (row-major)")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _c(t):
+    return None if t is None else t.contiguous()
 
 
 def _stream(device):
@@ -143,14 +151,14 @@ def _wsarg(desc, n_nodes, n_edges, which, device, ws):
 
 def forward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, out=None, ws=None):
     lib = load()
+    x, edge_index, edge_vec, w, w_rad, b_rad = map(_c, (x, edge_index, edge_vec, w, w_rad, b_rad))
     N, E = x.shape[0], edge_index.shape[1]
     if out is None:
         out = torch.empty((N, (desc.lmax + 1) ** 2, desc.c_out), dtype=torch.float32,
                           device=x.device)
     p, nb = _wsarg(desc, N, E, WS_FORWARD, x.device, ws)
     code = lib.so2conv_forward(ctypes.byref(desc), N, E, _ptr(x), _ptr(edge_index),
-                               _ptr(edge_vec), Params(w.data_ptr(), w_rad.data_ptr(),
-                                                      b_rad.data_ptr()),
+                               _ptr(edge_vec), Params(_ptr(w).value, _ptr(w_rad).value, _ptr(b_rad).value),
                                _ptr(out), p, nb, _stream(x.device))
     _check_call(code, "so2conv_forward")
     return out
@@ -160,6 +168,8 @@ def backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, need=None
              ws=None):
     """Returns a dict of gradients; `need` limits which ones are computed."""
     lib = load()
+    x, edge_index, edge_vec, w, w_rad, b_rad, grad_out = map(
+        _c, (x, edge_index, edge_vec, w, w_rad, b_rad, grad_out))
     N, E = x.shape[0], edge_index.shape[1]
     names = ["grad_x", "grad_w", "grad_w_rad", "grad_b_rad", "grad_edge_vec"]
     need = set(names if need is None else need)
@@ -183,6 +193,8 @@ def backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, need=None
 def double_backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg_x=None,
                     gg_edge_vec=None, need=None, ws=None):
     lib = load()
+    x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg_x, gg_edge_vec = map(
+        _c, (x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg_x, gg_edge_vec))
     N, E = x.shape[0], edge_index.shape[1]
     names = ["d_x", "d_w", "d_w_rad", "d_b_rad", "d_grad_out"]
     need = set(names if need is None else need)

@@ -96,36 +96,45 @@ struct EdgeRec {
 // Geometry record: d, r_hat[3], R[9] (row-major), 3 spare.
 constexpr int GEO = 16;
 
+// One thread per edge; the Wigner-D recursion runs in this thread's slice of
+// dynamic shared memory (blockDim.x * dsz floats) and is then copied out
+// with coalesced stores.
 __global__ void k_edge_prep(Layout y, const int *__restrict__ perm, int64_t e0, int M,
                             const int64_t *__restrict__ ei, int64_t E, int64_t N, int key_row,
                             const float *__restrict__ edge_vec, EdgeRec *__restrict__ rec,
                             float *__restrict__ geo, float *__restrict__ D, DevStatus *st) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= M) return;
-  const int e = perm[e0 + i];
-  int64_t s = ei[e], d = ei[E + e];
-  if (s < 0 || s >= N) s = 0;  // already reported by the sort
-  if (d < 0 || d >= N) d = 0;
-  EdgeRec r;
-  r.eid = e;
-  r.src = static_cast<int>(s);
-  r.dst = static_cast<int>(d);
-  r.key = key_row == 0 ? r.src : r.dst;
-  rec[i] = r;
-  Frame f;
-  if (!make_frame(edge_vec[3 * (int64_t)e], edge_vec[3 * (int64_t)e + 1],
-                  edge_vec[3 * (int64_t)e + 2], f))
-    raise_error(st, SO2_ERR_DEGENERATE, e);
-  float *gr = geo + (int64_t)i * GEO;
-  gr[0] = f.d;
-  gr[1] = f.rh[0];
-  gr[2] = f.rh[1];
-  gr[3] = f.rh[2];
-  for (int k = 0; k < 9; ++k) gr[4 + k] = f.R[k];
-  float Dl[dsize(LMAX_SUPPORTED)];
-  wigner_blocks(f.R, y.L, Dl);
-  float *Dg = D + (int64_t)i * y.dsz;
-  for (int k = 0; k < y.dsz; ++k) Dg[k] = Dl[k];
+  extern __shared__ float sD[];
+  const int i0 = blockIdx.x * blockDim.x;
+  const int i = i0 + threadIdx.x;
+  float *mine = sD + threadIdx.x * y.dsz;
+  if (i < M) {
+    const int e = perm[e0 + i];
+    int64_t s = ei[e], d = ei[E + e];
+    if (s < 0 || s >= N) s = 0;  // already reported by the sort
+    if (d < 0 || d >= N) d = 0;
+    EdgeRec r;
+    r.eid = e;
+    r.src = static_cast<int>(s);
+    r.dst = static_cast<int>(d);
+    r.key = key_row == 0 ? r.src : r.dst;
+    rec[i] = r;
+    Frame f;
+    if (!make_frame(edge_vec[3 * (int64_t)e], edge_vec[3 * (int64_t)e + 1],
+                    edge_vec[3 * (int64_t)e + 2], f))
+      raise_error(st, SO2_ERR_DEGENERATE, e);
+    float *gr = geo + (int64_t)i * GEO;
+    gr[0] = f.d;
+    gr[1] = f.rh[0];
+    gr[2] = f.rh[1];
+    gr[3] = f.rh[2];
+    for (int k = 0; k < 9; ++k) gr[4 + k] = f.R[k];
+    wigner_blocks(f.R, y.L, mine);
+  }
+  __syncthreads();
+  const int n_here = (M - i0) < (int)blockDim.x ? (M - i0) : (int)blockDim.x;
+  const int total = n_here * y.dsz;
+  float *dst = D + (int64_t)i0 * y.dsz;
+  for (int k = threadIdx.x; k < total; k += blockDim.x) dst[k] = sD[k];
 }
 
 __device__ __forceinline__ float rbf_val(float d, int k, const Layout &y, float cutoff) {
@@ -152,108 +161,165 @@ __global__ void k_edge_gate(Layout y, float cutoff, int M, const float *__restri
 // ---------------------------------------------------------------------------
 // Rotation on gather: row (l, m) of the edge frame = sum_m' D^l[m][m'] X[node][l, m'],
 // optionally times the gate, written in the grouped layout as bf16 (hi, lo).
-// One block per edge, threads over channels.
+// One warp per edge, lanes over channel pairs; |m| <= MM is unrolled at
+// compile time so the per-row accumulators stay in registers.
 // ---------------------------------------------------------------------------
-template <typename TX>
+__device__ __forceinline__ float2 load2(const float *p) { return *reinterpret_cast<const float2 *>(p); }
+__device__ __forceinline__ float2 load2(const __nv_bfloat16 *p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+}
+__device__ __forceinline__ void store_split2(__nv_bfloat16 *hi, __nv_bfloat16 *lo, float a, float b) {
+  __nv_bfloat16 h0, l0, h1, l1;
+  split_bf16(a, h0, l0);
+  split_bf16(b, h1, l1);
+  *reinterpret_cast<__nv_bfloat162 *>(hi) = __halves2bfloat162(h0, h1);
+  if (lo) *reinterpret_cast<__nv_bfloat162 *>(lo) = __halves2bfloat162(l0, l1);
+}
+
+template <typename TX, int MM>
 __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec,
                                 const float *__restrict__ D, const TX *__restrict__ X, int side,
                                 int use_src, const float *__restrict__ gate,
                                 __nv_bfloat16 *__restrict__ out_hi, __nv_bfloat16 *__restrict__ out_lo,
                                 int ld) {
-  const int i = blockIdx.x;
-  if (i >= M) return;
   const int C = side ? y.co : y.ci;
   const int *col_off = side ? y.kout_off : y.kin_off;
   const int *col_pad = side ? y.Kout_pad : y.Kin_pad;
-  const EdgeRec r = rec[i];
-  const int node = use_src ? r.src : r.dst;
-  const float *De = D + (int64_t)i * y.dsz;
-  const TX *Xn = X + (int64_t)node * y.S * C;
-  __nv_bfloat16 *oh = out_hi + (int64_t)i * ld;
-  __nv_bfloat16 *ol = out_lo ? out_lo + (int64_t)i * ld : nullptr;
-  for (int g = 0; g < y.ng; ++g) {
-    const int base = col_off[g];
-    const int width = y.rows[g] * C;
-    for (int j = 0; j < y.rows[g]; ++j) {
-      int l, m;
-      group_row_lm(y, g, j, l, m);
-      const float *Drow = De + dblock_off(l) + (m + l) * (2 * l + 1);
-      for (int c = threadIdx.x; c < C; c += blockDim.x) {
-        float acc = 0.f;
-        for (int mp = -l; mp <= l; ++mp)
-          acc += Drow[mp + l] * to_f32(Xn[(l * l + l + mp) * C + c]);
-        if (gate) acc *= gate[(int64_t)i * C + c];
-        __nv_bfloat16 h, lo;
-        split_bf16(acc, h, lo);
-        oh[base + j * C + c] = h;
-        if (ol) ol[base + j * C + c] = lo;
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
+    const EdgeRec r = rec[i];
+    const int node = use_src ? r.src : r.dst;
+    const float *De = D + (int64_t)i * y.dsz;
+    const TX *Xn = X + (int64_t)node * y.S * C;
+    __nv_bfloat16 *oh = out_hi + (int64_t)i * ld;
+    __nv_bfloat16 *ol = out_lo ? out_lo + (int64_t)i * ld : nullptr;
+    for (int c = 2 * lane; c < C; c += 64) {
+      float2 gv = make_float2(1.f, 1.f);
+      if (gate) gv = load2(gate + (int64_t)i * C + c);
+      for (int l = 0; l <= y.L; ++l) {
+        float a0[2 * MM + 1], a1[2 * MM + 1];
+#pragma unroll
+        for (int k = 0; k < 2 * MM + 1; ++k) a0[k] = a1[k] = 0.f;
+        const float *Dl = De + dblock_off(l);
+        const int w = 2 * l + 1;
+        for (int mp = -l; mp <= l; ++mp) {
+          const float2 xv = load2(Xn + (l * l + l + mp) * C + c);
+#pragma unroll
+          for (int m = -MM; m <= MM; ++m) {
+            if (m < -l || m > l) continue;
+            const float dv = Dl[(m + l) * w + mp + l];
+            a0[m + MM] += dv * xv.x;
+            a1[m + MM] += dv * xv.y;
+          }
+        }
+#pragma unroll
+        for (int m = -MM; m <= MM; ++m) {
+          if (m < -l || m > l) continue;
+          int g, j;
+          lm_group_row(y, l, m, g, j);
+          const int col = col_off[g] + j * C + c;
+          store_split2(oh + col, ol ? ol + col : nullptr, a0[m + MM] * gv.x, a1[m + MM] * gv.y);
+        }
       }
     }
-    for (int k = width + threadIdx.x; k < col_pad[g]; k += blockDim.x) {
-      oh[base + k] = __float2bfloat16_rn(0.f);
-      if (ol) ol[base + k] = __float2bfloat16_rn(0.f);
+    for (int g = 0; g < y.ng; ++g) {
+      const int width = y.rows[g] * C;
+      for (int k = width + 2 * lane; k < col_pad[g]; k += 64)
+        store_split2(oh + col_off[g] + k, ol ? ol + col_off[g] + k : nullptr, 0.f, 0.f);
     }
   }
 }
 
 // [M x K] bf16 row-major -> [K x Mp] (Mp = ld of the output), columns >= M zero.
+// 64 x 64 tiles through shared memory, 32-bit accesses.
 __global__ void k_transpose_bf16(const __nv_bfloat16 *__restrict__ in, int M, int K, int ld_in,
                                  __nv_bfloat16 *__restrict__ out, int Mp) {
-  __shared__ __nv_bfloat16 tile[32][33];
-  const int k0 = blockIdx.x * 32, m0 = blockIdx.y * 32;
-  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-    const int m = m0 + r, k = k0 + threadIdx.x;
-    tile[r][threadIdx.x] = (m < M && k < K) ? in[(int64_t)m * ld_in + k] : __float2bfloat16_rn(0.f);
+  __shared__ __nv_bfloat16 tile[64][66];
+  const int k0 = blockIdx.x * 64, m0 = blockIdx.y * 64;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+  for (int r = ty; r < 64; r += 8) {
+    const int m = m0 + r, k = k0 + 2 * tx;
+    __nv_bfloat162 v = __floats2bfloat162_rn(0.f, 0.f);
+    if (m < M && k < K) v = *reinterpret_cast<const __nv_bfloat162 *>(in + (int64_t)m * ld_in + k);
+    tile[r][2 * tx] = v.x;
+    tile[r][2 * tx + 1] = v.y;
   }
   __syncthreads();
-  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-    const int k = k0 + r, m = m0 + threadIdx.x;
-    if (k < K && m < Mp) out[(int64_t)k * Mp + m] = tile[threadIdx.x][r];
+  for (int r = ty; r < 64; r += 8) {
+    const int k = k0 + r, m = m0 + 2 * tx;
+    if (k < K && m < Mp) {
+      __nv_bfloat162 v;
+      v.x = tile[2 * tx][r];
+      v.y = tile[2 * tx + 1][r];
+      *reinterpret_cast<__nv_bfloat162 *>(out + (int64_t)k * Mp + m) = v;
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
 // Inverse rotation on reduction, node-centric.  For every node whose sorted
 // segment meets this chunk, out[n][(l,m')][c] += sum over its chunk edges of
-// sum_m D^l[m][m'] * F[i][row(l,m)][c] (* gate).  One block per node, threads
-// over channels; the chunks run in stream order, so every output element is
-// updated by one thread at a time and the sum order is fixed.
+// sum_m D^l[m][m'] * F[i][row(l,m)][c] (* gate).  One block per node,
+// threads over channel pairs, the node's sums in shared memory; the chunks
+// run in stream order, so every output element is updated by one thread at
+// a time and the sum order is fixed.
 // ---------------------------------------------------------------------------
+template <int MM>
 __global__ void k_scatter_nodes(Layout y, int64_t e0, int M, const EdgeRec *__restrict__ rec,
                                 const int *__restrict__ offsets, const float *__restrict__ D,
                                 const float *__restrict__ F, int ldf, int side,
                                 const float *__restrict__ gate, float *__restrict__ out) {
+  extern __shared__ float acc[];  // [S][C]
   if (M <= 0) return;
   const int C = side ? y.co : y.ci;
   const int *col_off = side ? y.kout_off : y.kin_off;
   const int n_first = rec[0].key, n_last = rec[M - 1].key;
-  float acc[(LMAX_SUPPORTED + 1) * (LMAX_SUPPORTED + 1)];
   for (int n = n_first + blockIdx.x; n <= n_last; n += gridDim.x) {
     int b = offsets[n] - static_cast<int>(e0), e = offsets[n + 1] - static_cast<int>(e0);
     b = b < 0 ? 0 : b;
     e = e > M ? M : e;
     if (b >= e) continue;
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
-      for (int s = 0; s < y.S; ++s) acc[s] = 0.f;
+    for (int k = threadIdx.x; k < y.S * C; k += blockDim.x) acc[k] = 0.f;
+    __syncthreads();
+    for (int c = 2 * threadIdx.x; c < C; c += 2 * blockDim.x) {
       for (int i = b; i < e; ++i) {
         const float *De = D + (int64_t)i * y.dsz;
         const float *Fi = F + (int64_t)i * ldf;
-        const float gv = gate ? gate[(int64_t)i * C + c] : 1.f;
+        float2 gv = make_float2(1.f, 1.f);
+        if (gate) gv = load2(gate + (int64_t)i * C + c);
         for (int l = 0; l <= y.L; ++l) {
-          const int mm = l < y.mmax ? l : y.mmax;
-          const float *Dl = De + dblock_off(l);
-          for (int m = -mm; m <= mm; ++m) {
+          float2 v[2 * MM + 1];
+#pragma unroll
+          for (int m = -MM; m <= MM; ++m) {
+            v[m + MM] = make_float2(0.f, 0.f);
+            if (m < -l || m > l) continue;
             int g, j;
             lm_group_row(y, l, m, g, j);
-            const float v = gv * Fi[col_off[g] + j * C + c];
-            const float *Drow = Dl + (m + l) * (2 * l + 1);
-            for (int mp = -l; mp <= l; ++mp) acc[l * l + l + mp] += Drow[mp + l] * v;
+            const float2 f = load2(Fi + col_off[g] + j * C + c);
+            v[m + MM] = make_float2(f.x * gv.x, f.y * gv.y);
+          }
+          const float *Dl = De + dblock_off(l);
+          const int w = 2 * l + 1;
+          for (int mp = -l; mp <= l; ++mp) {
+            float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+            for (int m = -MM; m <= MM; ++m) {
+              if (m < -l || m > l) continue;
+              const float dv = Dl[(m + l) * w + mp + l];
+              t0 += dv * v[m + MM].x;
+              t1 += dv * v[m + MM].y;
+            }
+            float *a = acc + (l * l + l + mp) * C + c;
+            a[0] += t0;
+            a[1] += t1;
           }
         }
       }
-      float *o = out + (int64_t)n * y.S * C + c;
-      for (int s = 0; s < y.S; ++s) o[s * C] += acc[s];
     }
+    __syncthreads();
+    float *o = out + (int64_t)n * y.S * C;
+    for (int k = threadIdx.x; k < y.S * C; k += blockDim.x) o[k] += acc[k];
+    __syncthreads();
   }
 }
 
@@ -332,161 +398,188 @@ __global__ void k_unstack_grad(Layout y, BlockOffsets bo, const float *__restric
 }
 
 // ---------------------------------------------------------------------------
-// Backward per-edge terms.  For one edge (block) and all channels:
+// Backward per-edge terms.  For one edge (warp) and all channels:
 //   Gy~ = D G[dst] on rows |m| <= mmax+1,   a = D x[src] on the same rows,
 //   Gg[c'] = sum_{kept rows} Gy~ * v,
 //   h_k   = sum_{kept rows, c'} (g v) (J_k Gy~) + sum_{kept rows, c} Ga (J_k a),
 // where v (mixing output) and Ga (gradient of the rotated input) come from
 // the two products.  h_x, h_y give the frame part of dL/dr.
 // ---------------------------------------------------------------------------
-template <typename TX>
+template <typename TX, int MM>
 __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
                              const float *__restrict__ D, const float *__restrict__ gate,
                              const float *__restrict__ G, const TX *__restrict__ X,
                              const float *__restrict__ V, const float *__restrict__ Ga,
                              float *__restrict__ Gg, float *__restrict__ h) {
-  const int i = blockIdx.x;
-  if (i >= M) return;
-  const int *kout_off = y.kout_off;
-  const int *kin_off = y.kin_off;
-  const EdgeRec r = rec[i];
-  const float *De = D + (int64_t)i * y.dsz;
-  float hx = 0.f, hy = 0.f;
-  const int wide = y.mmax + 1;
-  float buf[2 * LMAX_SUPPORTED + 1];
-  // output side
-  for (int c = threadIdx.x; c < y.co; c += blockDim.x) {
-    const float gv = gate[(int64_t)i * y.co + c];
+  constexpr int W = MM + 1;  // widest |m| needed by the generators
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
+    const EdgeRec r = rec[i];
+    const float *De = D + (int64_t)i * y.dsz;
+    float hx = 0.f, hy = 0.f;
+    // output side
     const float *Gn = G + (int64_t)r.dst * y.S * y.co;
     const float *Vi = V + (int64_t)i * y.KG;
-    float gg = 0.f;
-    for (int l = 0; l <= y.L; ++l) {
-      const int mw = l < wide ? l : wide;
-      const float *Dl = De + dblock_off(l);
-      for (int m = -mw; m <= mw; ++m) {
-        float acc = 0.f;
-        for (int mp = -l; mp <= l; ++mp) acc += Dl[(m + l) * (2 * l + 1) + mp + l] * Gn[(l * l + l + mp) * y.co + c];
-        buf[m + mw] = acc;
+    for (int c = 2 * lane; c < y.co; c += 64) {
+      const float2 gv = load2(gate + (int64_t)i * y.co + c);
+      float gg0 = 0.f, gg1 = 0.f;
+      for (int l = 0; l <= y.L; ++l) {
+        float b0[2 * W + 1], b1[2 * W + 1];
+#pragma unroll
+        for (int k = 0; k < 2 * W + 1; ++k) b0[k] = b1[k] = 0.f;
+        const float *Dl = De + dblock_off(l);
+        const int w = 2 * l + 1;
+        for (int mp = -l; mp <= l; ++mp) {
+          const float2 gx = load2(Gn + (l * l + l + mp) * y.co + c);
+#pragma unroll
+          for (int m = -W; m <= W; ++m) {
+            if (m < -l || m > l) continue;
+            const float dv = Dl[(m + l) * w + mp + l];
+            b0[m + W] += dv * gx.x;
+            b1[m + W] += dv * gx.y;
+          }
+        }
+#pragma unroll
+        for (int m = -MM; m <= MM; ++m) {
+          if (m < -l || m > l) continue;
+          int g, j;
+          lm_group_row(y, l, m, g, j);
+          const float2 v = load2(Vi + y.kout_off[g] + j * y.co + c);
+          gg0 += b0[m + W] * v.x;
+          gg1 += b1[m + W] * v.y;
+          float jx0, jy0, jx1, jy1;
+          gen_xy(l, m, [&](int q) { return b0[q + W]; }, jx0, jy0);
+          gen_xy(l, m, [&](int q) { return b1[q + W]; }, jx1, jy1);
+          hx += gv.x * v.x * jx0 + gv.y * v.y * jx1;
+          hy += gv.x * v.x * jy0 + gv.y * v.y * jy1;
+        }
       }
-      const int mm = l < y.mmax ? l : y.mmax;
-      for (int m = -mm; m <= mm; ++m) {
-        int g, j;
-        lm_group_row(y, l, m, g, j);
-        const float v = Vi[kout_off[g] + j * y.co + c];
-        gg += buf[m + mw] * v;
-        float jx, jy;
-        gen_xy(l, m, [&](int q) { return buf[q + mw]; }, jx, jy);
-        hx += gv * v * jx;
-        hy += gv * v * jy;
-      }
+      *reinterpret_cast<float2 *>(Gg + (int64_t)i * y.co + c) = make_float2(gg0, gg1);
     }
-    Gg[(int64_t)i * y.co + c] = gg;
-  }
-  // input side
-  for (int c = threadIdx.x; c < y.ci; c += blockDim.x) {
+    // input side
     const TX *Xn = X + (int64_t)r.src * y.S * y.ci;
     const float *Gai = Ga + (int64_t)i * y.KA;
-    for (int l = 0; l <= y.L; ++l) {
-      const int mw = l < wide ? l : wide;
-      const float *Dl = De + dblock_off(l);
-      for (int m = -mw; m <= mw; ++m) {
-        float acc = 0.f;
-        for (int mp = -l; mp <= l; ++mp) acc += Dl[(m + l) * (2 * l + 1) + mp + l] * to_f32(Xn[(l * l + l + mp) * y.ci + c]);
-        buf[m + mw] = acc;
-      }
-      const int mm = l < y.mmax ? l : y.mmax;
-      for (int m = -mm; m <= mm; ++m) {
-        int g, j;
-        lm_group_row(y, l, m, g, j);
-        const float ga = Gai[kin_off[g] + j * y.ci + c];
-        float jx, jy;
-        gen_xy(l, m, [&](int q) { return buf[q + mw]; }, jx, jy);
-        hx += ga * jx;
-        hy += ga * jy;
+    for (int c = 2 * lane; c < y.ci; c += 64) {
+      for (int l = 0; l <= y.L; ++l) {
+        float b0[2 * W + 1], b1[2 * W + 1];
+#pragma unroll
+        for (int k = 0; k < 2 * W + 1; ++k) b0[k] = b1[k] = 0.f;
+        const float *Dl = De + dblock_off(l);
+        const int w = 2 * l + 1;
+        for (int mp = -l; mp <= l; ++mp) {
+          const float2 xv = load2(Xn + (l * l + l + mp) * y.ci + c);
+#pragma unroll
+          for (int m = -W; m <= W; ++m) {
+            if (m < -l || m > l) continue;
+            const float dv = Dl[(m + l) * w + mp + l];
+            b0[m + W] += dv * xv.x;
+            b1[m + W] += dv * xv.y;
+          }
+        }
+#pragma unroll
+        for (int m = -MM; m <= MM; ++m) {
+          if (m < -l || m > l) continue;
+          int g, j;
+          lm_group_row(y, l, m, g, j);
+          const float2 ga = load2(Gai + y.kin_off[g] + j * y.ci + c);
+          float jx0, jy0, jx1, jy1;
+          gen_xy(l, m, [&](int q) { return b0[q + W]; }, jx0, jy0);
+          gen_xy(l, m, [&](int q) { return b1[q + W]; }, jx1, jy1);
+          hx += ga.x * jx0 + ga.y * jx1;
+          hy += ga.x * jy0 + ga.y * jy1;
+        }
       }
     }
-  }
-  // block reduction of (hx, hy) in a fixed order
-  __shared__ float red[2][32];
-  for (int o = 16; o > 0; o >>= 1) {
-    hx += __shfl_xor_sync(0xffffffffu, hx, o);
-    hy += __shfl_xor_sync(0xffffffffu, hy, o);
-  }
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) {
-    red[0][w] = hx;
-    red[1][w] = hy;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float sx = 0.f, sy = 0.f;
-    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) {
-      sx += red[0][k];
-      sy += red[1][k];
+    for (int o = 16; o > 0; o >>= 1) {
+      hx += __shfl_xor_sync(0xffffffffu, hx, o);
+      hy += __shfl_xor_sync(0xffffffffu, hy, o);
     }
-    h[2 * (int64_t)i] = sx;
-    h[2 * (int64_t)i + 1] = sy;
+    if (lane == 0) {
+      h[2 * (int64_t)i] = hx;
+      h[2 * (int64_t)i + 1] = hy;
+    }
   }
 }
 
 // grad_r[eid] = R^T (-h_y, h_x, 0) / d + (sum_c' Gg[c'] sum_k W_rad[k][c'] phi'_k(d)) r_hat.
-// One warp per edge.
+// One warp per edge; phi'_k(d) is computed once per edge (lanes over k).
 __global__ void k_edge_final(Layout y, float cutoff, int M, const EdgeRec *__restrict__ rec,
                              const float *__restrict__ geo, const float *__restrict__ Gg,
                              const float *__restrict__ h, const float *__restrict__ w_rad,
                              float *__restrict__ grad_r) {
-  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (i >= M) return;
-  const float *gr = geo + (int64_t)i * GEO;
-  const float d = gr[0];
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
   const float sig = cutoff / static_cast<float>(y.nr - 1);
-  float dd = 0.f;
-  for (int c = lane; c < y.co; c += 32) {
-    float dg = 0.f;
-    for (int k = 0; k < y.nr; ++k) {
-      const float mu = sig * static_cast<float>(k);
-      const float t = (d - mu) / sig;
-      dg += w_rad[k * y.co + c] * (-t / sig) * __expf(-0.5f * t * t);
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
+    const float *gr = geo + (int64_t)i * GEO;
+    const float d = gr[0];
+    float dphi[2];  // k = lane, lane + 32
+    for (int u = 0; u < 2; ++u) {
+      const int k = lane + 32 * u;
+      const float t = (d - sig * static_cast<float>(k)) / sig;
+      dphi[u] = (k < y.nr) ? (-t / sig) * __expf(-0.5f * t * t) : 0.f;
     }
-    dd += Gg[(int64_t)i * y.co + c] * dg;
-  }
-  for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
-  if (lane == 0) {
-    const float hx = h[2 * (int64_t)i], hy = h[2 * (int64_t)i + 1];
-    const float inv = d > 0.f ? 1.f / d : 0.f;
-    const float *R = gr + 4;
-    const int e = rec[i].eid;
-    for (int a = 0; a < 3; ++a)
-      grad_r[3 * (int64_t)e + a] = (R[0 * 3 + a] * (-hy) + R[1 * 3 + a] * hx) * inv + dd * gr[1 + a];
+    float dd = 0.f;
+    // every lane runs every shuffle: the channel loop is warp-uniform
+    for (int c0 = 0; c0 < y.co; c0 += 32) {
+      const int c = c0 + lane;
+      float dg = 0.f;
+      for (int k = 0; k < y.nr; ++k) {
+        const float dk = __shfl_sync(0xffffffffu, dphi[k >> 5], k & 31);
+        if (c < y.co) dg += w_rad[k * y.co + c] * dk;
+      }
+      if (c < y.co) dd += Gg[(int64_t)i * y.co + c] * dg;
+    }
+    for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
+    if (lane == 0) {
+      const float hx = h[2 * (int64_t)i], hy = h[2 * (int64_t)i + 1];
+      const float inv = d > 0.f ? 1.f / d : 0.f;
+      const float *R = gr + 4;
+      const int e = rec[i].eid;
+      for (int a = 0; a < 3; ++a)
+        grad_r[3 * (int64_t)e + a] = (R[0 * 3 + a] * (-hy) + R[1 * 3 + a] * hx) * inv + dd * gr[1 + a];
+    }
   }
 }
 
-// grad_w_rad[k][c'] += sum_i phi_k(d_i) Gg[i][c'];  grad_b[c'] += sum_i Gg[i][c'].
-// Block (32 channels, 8 edge lanes); fixed-order reduction.
-__global__ void k_rad_grad(Layout y, float cutoff, int M, const float *__restrict__ geo,
-                           const float *__restrict__ Gg, float *__restrict__ grad_w_rad,
-                           float *__restrict__ grad_b) {
-  const int c = blockIdx.x * 32 + threadIdx.x;
-  const int k = blockIdx.y;  // 0..nr-1 for w_rad, nr for the bias
-  __shared__ float red[8][32];
-  float acc = 0.f;
-  if (c < y.co) {
-    for (int i = threadIdx.y; i < M; i += blockDim.y) {
-      const float phi = (k < y.nr) ? rbf_val(geo[(int64_t)i * GEO], k, y, cutoff) : 1.f;
-      acc += phi * Gg[(int64_t)i * y.co + c];
-    }
+// Radial-gate gradients, stage 1: each block sums phi_k(d_i) Gg[i][c'] (and
+// Gg for the bias row k = nr) over a tile of RAD_TILE edges into
+// part[block][k][c'].  Stage 2 adds the blocks in order.  Deterministic.
+constexpr int RAD_TILE = 256;
+__global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__restrict__ geo,
+                              const float *__restrict__ Gg, float *__restrict__ part) {
+  extern __shared__ float phi[];  // [RAD_TILE][nr]
+  const int i0 = blockIdx.x * RAD_TILE;
+  const int n = (M - i0) < RAD_TILE ? (M - i0) : RAD_TILE;
+  for (int t = threadIdx.x; t < n * y.nr; t += blockDim.x) {
+    const int i = t / y.nr, k = t % y.nr;
+    phi[t] = rbf_val(geo[(int64_t)(i0 + i) * GEO], k, y, cutoff);
   }
-  red[threadIdx.y][threadIdx.x] = acc;
   __syncthreads();
-  if (threadIdx.y == 0 && c < y.co) {
+  const int P = (y.nr + 1) * y.co;
+  for (int pidx = threadIdx.x; pidx < P; pidx += blockDim.x) {
+    const int k = pidx / y.co, c = pidx % y.co;
     float s = 0.f;
-    for (int t = 0; t < (int)blockDim.y; ++t) s += red[t][threadIdx.x];
     if (k < y.nr) {
-      if (grad_w_rad) grad_w_rad[k * y.co + c] += s;
-    } else if (grad_b) {
-      grad_b[c] += s;
+      for (int i = 0; i < n; ++i) s += phi[i * y.nr + k] * Gg[(int64_t)(i0 + i) * y.co + c];
+    } else {
+      for (int i = 0; i < n; ++i) s += Gg[(int64_t)(i0 + i) * y.co + c];
     }
+    part[(int64_t)blockIdx.x * P + pidx] = s;
+  }
+}
+
+__global__ void k_rad_reduce(Layout y, int nblk, const float *__restrict__ part,
+                             float *__restrict__ grad_w_rad, float *__restrict__ grad_b) {
+  const int P = (y.nr + 1) * y.co;
+  const int pidx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (pidx >= P) return;
+  float s = 0.f;
+  for (int b = 0; b < nblk; ++b) s += part[(int64_t)b * P + pidx];
+  const int k = pidx / y.co, c = pidx % y.co;
+  if (k < y.nr) {
+    if (grad_w_rad) grad_w_rad[k * y.co + c] += s;
+  } else if (grad_b) {
+    grad_b[c] += s;
   }
 }
 

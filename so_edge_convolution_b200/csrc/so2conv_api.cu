@@ -14,7 +14,7 @@ using namespace so2;
 
 namespace {
 
-constexpr int CHUNK_MAX = 8192;  // edges per chunk of per-edge intermediates
+constexpr int CHUNK_MAX = 32768;  // edges per chunk of per-edge intermediates
 
 // --------------------------------------------------------------------------
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -66,7 +66,7 @@ struct Plan {
   size_t total = 0;
   // byte offsets
   size_t status, counts, cursor, offsets, perm, rec, geo, D, gate, wst_hi, wst_lo, wtr_hi, wtr_lo,
-      a_hi, a_lo, V, gv_hi, gv_lo, aT_hi, aT_lo, gvT_hi, gvT_lo, Ga, Gg, h, dws;
+      a_hi, a_lo, V, gv_hi, gv_lo, aT_hi, aT_lo, gvT_hi, gvT_lo, Ga, Gg, h, dws, radp;
 };
 
 size_t take(size_t &cur, size_t bytes) {
@@ -129,6 +129,7 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
     p.Gg = take(c, 4ull * p.chunk * y.co);
     p.h = take(c, 8ull * p.chunk);
     p.dws = take(c, 4ull * y.WR * y.WK);
+    p.radp = take(c, 4ull * ((p.chunk + RAD_TILE - 1) / RAD_TILE) * (y.nr + 1) * y.co);
   }
   p.total = (c + 1023) & ~static_cast<size_t>(1023);
   return p;
@@ -199,6 +200,32 @@ int grid_for(int64_t n, int block) {
   if (g < 1) g = 1;
   if (g > 148 * 16) g = 148 * 16;
   return static_cast<int>(g);
+}
+
+#define DISPATCH_MM(mm, ...)                  \
+  switch (mm) {                               \
+    case 0: { constexpr int MM = 0; __VA_ARGS__; } break; \
+    case 1: { constexpr int MM = 1; __VA_ARGS__; } break; \
+    case 2: { constexpr int MM = 2; __VA_ARGS__; } break; \
+    case 3: { constexpr int MM = 3; __VA_ARGS__; } break; \
+    case 4: { constexpr int MM = 4; __VA_ARGS__; } break; \
+    case 5: { constexpr int MM = 5; __VA_ARGS__; } break; \
+    default: { constexpr int MM = 6; __VA_ARGS__; } break; \
+  }
+
+// Raise the dynamic shared memory limit of a kernel (once per kernel).
+template <typename K>
+bool allow_smem(K kernel, int bytes) {
+  if (bytes <= 48 * 1024) return true;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+int warp_grid(int M, int warps_per_block) {
+  int g = (M + warps_per_block - 1) / warps_per_block;
+  if (g < 1) g = 1;
+  if (g > 148 * 8) g = 148 * 8;
+  return g;
 }
 
 // --------------------------------------------------------------------------
@@ -354,9 +381,13 @@ so2_status pack_weights(Ctx &c, const void *w) {
 so2_status chunk_prep(Ctx &c, int64_t e0, int M, const int64_t *ei, const float *ev, int key_row,
                       so2conv_params prm) {
   const Plan &P = c.P;
-  k_edge_prep<<<(M + 127) / 128, 128, 0, c.s>>>(P.y, at<int>(c.ws, P.perm), e0, M, ei, P.E, P.N,
-                                                 key_row, ev, at<EdgeRec>(c.ws, P.rec),
-                                                 at<float>(c.ws, P.geo), at<float>(c.ws, P.D), c.st);
+  const int tpb = P.y.dsz <= 200 ? 64 : 32;
+  const int smem = tpb * P.y.dsz * static_cast<int>(sizeof(float));
+  if (!allow_smem(k_edge_prep, smem)) return SO2_ERR_CUDA;
+  k_edge_prep<<<(M + tpb - 1) / tpb, tpb, smem, c.s>>>(P.y, at<int>(c.ws, P.perm), e0, M, ei, P.E,
+                                                       P.N, key_row, ev, at<EdgeRec>(c.ws, P.rec),
+                                                       at<float>(c.ws, P.geo),
+                                                       at<float>(c.ws, P.D), c.st);
   CKL();
   k_edge_gate<<<M, 128, 0, c.s>>>(P.y, c.d->rbf_cutoff, M, at<float>(c.ws, P.geo), prm.w_rad,
                                   prm.b_rad, at<float>(c.ws, P.gate));
@@ -367,12 +398,17 @@ so2_status chunk_prep(Ctx &c, int64_t e0, int M, const int64_t *ei, const float 
 so2_status rotate_x(Ctx &c, int M, const void *x) {
   const Plan &P = c.P;
   __nv_bfloat16 *hi = at<__nv_bfloat16>(c.ws, P.a_hi), *lo = P.split ? at<__nv_bfloat16>(c.ws, P.a_lo) : nullptr;
-  if (P.xbf16)
-    k_rotate_gather<__nv_bfloat16><<<M, 128, 0, c.s>>>(P.y, M, at<EdgeRec>(c.ws, P.rec), at<float>(c.ws, P.D),
-                                                     static_cast<const __nv_bfloat16 *>(x), 0, 1, nullptr, hi, lo, P.y.KA);
-  else
-    k_rotate_gather<float><<<M, 128, 0, c.s>>>(P.y, M, at<EdgeRec>(c.ws, P.rec), at<float>(c.ws, P.D),
-                                             static_cast<const float *>(x), 0, 1, nullptr, hi, lo, P.y.KA);
+  const EdgeRec *rec = at<EdgeRec>(c.ws, P.rec);
+  const float *D = at<float>(c.ws, P.D);
+  if (P.xbf16) {
+    DISPATCH_MM(P.y.mmax, (k_rotate_gather<__nv_bfloat16, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                               P.y, M, rec, D, static_cast<const __nv_bfloat16 *>(x), 0, 1,
+                               nullptr, hi, lo, P.y.KA)));
+  } else {
+    DISPATCH_MM(P.y.mmax, (k_rotate_gather<float, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                               P.y, M, rec, D, static_cast<const float *>(x), 0, 1, nullptr, hi,
+                               lo, P.y.KA)));
+  }
   CKL();
   return SO2_OK;
 }
@@ -386,6 +422,28 @@ so2_status gemm_v(Ctx &c, int M) {
     L.add(M, y.Kout[g], y.Kin_pad[g], 0, y.kin_off[g], y.wr_off[g], 0, y.kout_off[g], y.KG);
   CK(launch_gemm(0, P.split, c.m_a_hi, c.m_a_lo, c.m_wst_hi, c.m_wst_lo, L.p, at<float>(c.ws, P.V), 0,
                  c.st, c.s));
+  return SO2_OK;
+}
+
+// Node-centric inverse rotation on reduction of F (rows of the grouped
+// layout on `side`) into out, for the chunk's nodes.
+so2_status scatter(Ctx &c, int64_t e0, int M, const float *F, int ldf, int side,
+                   const float *gate, float *out) {
+  const Plan &P = c.P;
+  const Layout &y = P.y;
+  const int C = side ? y.co : y.ci;
+  int threads = C / 2;
+  threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
+  const int smem = y.S * C * static_cast<int>(sizeof(float));
+  const EdgeRec *rec = at<EdgeRec>(c.ws, P.rec);
+  const int *off = at<int>(c.ws, P.offsets);
+  const float *D = at<float>(c.ws, P.D);
+  bool ok = true;
+  DISPATCH_MM(y.mmax, ok = allow_smem(k_scatter_nodes<MM>, smem);
+              if (ok) k_scatter_nodes<MM><<<grid_for(M, 1), threads, smem, c.s>>>(
+                  y, e0, M, rec, off, D, F, ldf, side, gate, out));
+  if (!ok) return SO2_ERR_CUDA;
+  CKL();
   return SO2_OK;
 }
 
@@ -434,10 +492,8 @@ so2_status so2conv_forward(const so2conv_desc *desc, int64_t N, int64_t E, const
     if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 1, prm)) != SO2_OK) return r;
     if ((r = rotate_x(c, M, x)) != SO2_OK) return r;
     if ((r = gemm_v(c, M)) != SO2_OK) return r;
-    k_scatter_nodes<<<grid_for(M, 1), y.co < 1024 ? y.co : 1024, 0, c.s>>>(
-        y, e0, M, at<EdgeRec>(ws, P.rec), at<int>(ws, P.offsets), at<float>(ws, P.D),
-        at<float>(ws, P.V), y.KG, 1, at<float>(ws, P.gate), out);
-    CKL();
+    if ((r = scatter(c, e0, M, at<float>(ws, P.V), y.KG, 1, at<float>(ws, P.gate), out)) != SO2_OK)
+      return r;
   }
   return SO2_OK;
 }
@@ -482,8 +538,9 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
     if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 0, prm)) != SO2_OK) return r;
     if ((r = rotate_x(c, M, x)) != SO2_OK) return r;
     // Gv = g * (D G[dst]) on the kept rows
-    k_rotate_gather<float><<<M, 128, 0, c.s>>>(y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
-                                             grad_out, 1, 0, at<float>(ws, P.gate), gv_hi, gv_lo, y.KG);
+    DISPATCH_MM(y.mmax, (k_rotate_gather<float, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                            y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), grad_out, 1, 0,
+                            at<float>(ws, P.gate), gv_hi, gv_lo, y.KG)));
     CKL();
     if (need_v && (r = gemm_v(c, M)) != SO2_OK) return r;
     if (need_ga) {
@@ -495,18 +552,18 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
     }
     if (grad_w) {
       const int Kp = round_up(M, 64);
-      dim3 tb(32, 8);
-      k_transpose_bf16<<<dim3((y.KA + 31) / 32, (P.chunkp + 31) / 32), tb, 0, c.s>>>(
+      const int mt = (Kp + 63) / 64;  // only the columns the product reads
+      k_transpose_bf16<<<dim3((y.KA + 63) / 64, mt), 256, 0, c.s>>>(
           at<__nv_bfloat16>(ws, P.a_hi), M, y.KA, y.KA, at<__nv_bfloat16>(ws, P.aT_hi), P.chunkp);
       CKL();
-      k_transpose_bf16<<<dim3((y.KG + 31) / 32, (P.chunkp + 31) / 32), tb, 0, c.s>>>(
+      k_transpose_bf16<<<dim3((y.KG + 63) / 64, mt), 256, 0, c.s>>>(
           gv_hi, M, y.KG, y.KG, at<__nv_bfloat16>(ws, P.gvT_hi), P.chunkp);
       CKL();
       if (P.split) {
-        k_transpose_bf16<<<dim3((y.KA + 31) / 32, (P.chunkp + 31) / 32), tb, 0, c.s>>>(
+        k_transpose_bf16<<<dim3((y.KA + 63) / 64, mt), 256, 0, c.s>>>(
             at<__nv_bfloat16>(ws, P.a_lo), M, y.KA, y.KA, at<__nv_bfloat16>(ws, P.aT_lo), P.chunkp);
         CKL();
-        k_transpose_bf16<<<dim3((y.KG + 31) / 32, (P.chunkp + 31) / 32), tb, 0, c.s>>>(
+        k_transpose_bf16<<<dim3((y.KG + 63) / 64, mt), 256, 0, c.s>>>(
             gv_lo, M, y.KG, y.KG, at<__nv_bfloat16>(ws, P.gvT_lo), P.chunkp);
         CKL();
       }
@@ -517,34 +574,41 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
       CK(launch_gemm(2, P.split, c.m_gvT_hi, c.m_gvT_lo, c.m_aT_hi, c.m_aT_lo, L.p, dws, 1, c.st,
                      c.s));
     }
-    if (grad_x) {
-      k_scatter_nodes<<<grid_for(M, 1), y.ci < 1024 ? y.ci : 1024, 0, c.s>>>(
-          y, e0, M, at<EdgeRec>(ws, P.rec), at<int>(ws, P.offsets), at<float>(ws, P.D),
-          at<float>(ws, P.Ga), y.KA, 0, nullptr, grad_x);
-      CKL();
-    }
+    if (grad_x &&
+        (r = scatter(c, e0, M, at<float>(ws, P.Ga), y.KA, 0, nullptr, grad_x)) != SO2_OK)
+      return r;
     if (need_terms) {
-      if (P.xbf16)
-        k_edge_terms<__nv_bfloat16><<<M, 128, 0, c.s>>>(
-            y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), at<float>(ws, P.gate), grad_out,
-            static_cast<const __nv_bfloat16 *>(x), at<float>(ws, P.V), at<float>(ws, P.Ga),
-            at<float>(ws, P.Gg), at<float>(ws, P.h));
-      else
-        k_edge_terms<float><<<M, 128, 0, c.s>>>(
-            y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), at<float>(ws, P.gate), grad_out,
-            static_cast<const float *>(x), at<float>(ws, P.V), at<float>(ws, P.Ga),
-            at<float>(ws, P.Gg), at<float>(ws, P.h));
+      if (P.xbf16) {
+        DISPATCH_MM(y.mmax, (k_edge_terms<__nv_bfloat16, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                                y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
+                                at<float>(ws, P.gate), grad_out,
+                                static_cast<const __nv_bfloat16 *>(x), at<float>(ws, P.V),
+                                at<float>(ws, P.Ga), at<float>(ws, P.Gg), at<float>(ws, P.h))));
+      } else {
+        DISPATCH_MM(y.mmax, (k_edge_terms<float, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                                y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
+                                at<float>(ws, P.gate), grad_out, static_cast<const float *>(x),
+                                at<float>(ws, P.V), at<float>(ws, P.Ga), at<float>(ws, P.Gg),
+                                at<float>(ws, P.h))));
+      }
       CKL();
       if (grad_edge_vec) {
-        k_edge_final<<<(M + 3) / 4, 128, 0, c.s>>>(y, desc->rbf_cutoff, M, at<EdgeRec>(ws, P.rec),
-                                                   at<float>(ws, P.geo), at<float>(ws, P.Gg),
-                                                   at<float>(ws, P.h), prm.w_rad, grad_edge_vec);
+        k_edge_final<<<warp_grid(M, 8), 256, 0, c.s>>>(y, desc->rbf_cutoff, M,
+                                                        at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo),
+                                                        at<float>(ws, P.Gg), at<float>(ws, P.h),
+                                                        prm.w_rad, grad_edge_vec);
         CKL();
       }
       if (grad_w_rad || grad_b_rad) {
-        k_rad_grad<<<dim3((y.co + 31) / 32, y.nr + 1), dim3(32, 8), 0, c.s>>>(
-            y, desc->rbf_cutoff, M, at<float>(ws, P.geo), at<float>(ws, P.Gg), grad_w_rad,
-            grad_b_rad);
+        const int nblk = (M + RAD_TILE - 1) / RAD_TILE;
+        const int sm = RAD_TILE * y.nr * static_cast<int>(sizeof(float));
+        if (!allow_smem(k_rad_partial, sm)) return SO2_ERR_CUDA;
+        k_rad_partial<<<nblk, 256, sm, c.s>>>(y, desc->rbf_cutoff, M, at<float>(ws, P.geo),
+                                              at<float>(ws, P.Gg), at<float>(ws, P.radp));
+        CKL();
+        const int Pn = (y.nr + 1) * y.co;
+        k_rad_reduce<<<(Pn + 255) / 256, 256, 0, c.s>>>(y, nblk, at<float>(ws, P.radp), grad_w_rad,
+                                                         grad_b_rad);
         CKL();
       }
     }
@@ -587,7 +651,8 @@ long long so2conv_launch_count(void) { return g_launches; }
 
 void so2conv_profile_enable(int on) {
   g_prof.on = on != 0;
-  for (int k = 0; k < PROF_KINDS; ++k) g_prof.used[k] = 0;
+  if (g_prof.on)
+    for (int k = 0; k < PROF_KINDS; ++k) g_prof.used[k] = 0;
 }
 
 so2_status so2conv_profile_read(int kind, int *n_launches, double *total_ms) {
