@@ -176,16 +176,32 @@ __device__ __forceinline__ void store_split2(__nv_bfloat16 *hi, __nv_bfloat16 *l
   if (lo) *reinterpret_cast<__nv_bfloat162 *>(lo) = __halves2bfloat162(l0, l1);
 }
 
+// Per-channel coefficient: 0 (absent), 1, or an [edge][channel] array.
+struct Coef {
+  const float *p;
+  int mode;  // 0 zero, 1 one, 2 array
+};
+__device__ __forceinline__ float2 coef2(const Coef &k, int64_t i, int C, int c) {
+  if (k.mode == 0) return make_float2(0.f, 0.f);
+  if (k.mode == 1) return make_float2(1.f, 1.f);
+  return load2(k.p + i * C + c);
+}
+
+// out[row (l,m)] = A * b[m] + B * (Omega b)[m],  b = D^l X[node][l, :],
+// Omega = w_x J_x + w_y J_y with (w_x, w_y) = omega[i][0..1].  With B absent
+// this is plain rotation on gather (A = 1) or gated rotation (A = g).
 template <typename TX, int MM>
 __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec,
                                 const float *__restrict__ D, const TX *__restrict__ X, int side,
-                                int use_src, const float *__restrict__ gate,
+                                int use_src, Coef A, Coef B, const float *__restrict__ omega,
                                 __nv_bfloat16 *__restrict__ out_hi, __nv_bfloat16 *__restrict__ out_lo,
                                 int ld) {
+  constexpr int W = MM + 1;
   const int C = side ? y.co : y.ci;
   const int *col_off = side ? y.kout_off : y.kin_off;
   const int *col_pad = side ? y.Kout_pad : y.Kin_pad;
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  const bool wide = B.mode != 0;
   for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
     const EdgeRec r = rec[i];
     const int node = use_src ? r.src : r.dst;
@@ -193,23 +209,28 @@ __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec
     const TX *Xn = X + (int64_t)node * y.S * C;
     __nv_bfloat16 *oh = out_hi + (int64_t)i * ld;
     __nv_bfloat16 *ol = out_lo ? out_lo + (int64_t)i * ld : nullptr;
+    float wx = 0.f, wy = 0.f;
+    if (wide) {
+      wx = omega[4 * (int64_t)i];
+      wy = omega[4 * (int64_t)i + 1];
+    }
     for (int c = 2 * lane; c < C; c += 64) {
-      float2 gv = make_float2(1.f, 1.f);
-      if (gate) gv = load2(gate + (int64_t)i * C + c);
+      const float2 ca = coef2(A, i, C, c), cb = coef2(B, i, C, c);
       for (int l = 0; l <= y.L; ++l) {
-        float a0[2 * MM + 1], a1[2 * MM + 1];
+        float a0[2 * W + 1], a1[2 * W + 1];
 #pragma unroll
-        for (int k = 0; k < 2 * MM + 1; ++k) a0[k] = a1[k] = 0.f;
+        for (int k = 0; k < 2 * W + 1; ++k) a0[k] = a1[k] = 0.f;
         const float *Dl = De + dblock_off(l);
         const int w = 2 * l + 1;
+        const int top = wide ? W : MM;
         for (int mp = -l; mp <= l; ++mp) {
           const float2 xv = load2(Xn + (l * l + l + mp) * C + c);
 #pragma unroll
-          for (int m = -MM; m <= MM; ++m) {
-            if (m < -l || m > l) continue;
+          for (int m = -W; m <= W; ++m) {
+            if (m < -l || m > l || m < -top || m > top) continue;
             const float dv = Dl[(m + l) * w + mp + l];
-            a0[m + MM] += dv * xv.x;
-            a1[m + MM] += dv * xv.y;
+            a0[m + W] += dv * xv.x;
+            a1[m + W] += dv * xv.y;
           }
         }
 #pragma unroll
@@ -218,7 +239,15 @@ __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec
           int g, j;
           lm_group_row(y, l, m, g, j);
           const int col = col_off[g] + j * C + c;
-          store_split2(oh + col, ol ? ol + col : nullptr, a0[m + MM] * gv.x, a1[m + MM] * gv.y);
+          float o0 = ca.x * a0[m + W], o1 = ca.y * a1[m + W];
+          if (wide) {
+            float jx0, jy0, jx1, jy1;
+            gen_xy(l, m, [&](int q) { return a0[q + W]; }, jx0, jy0);
+            gen_xy(l, m, [&](int q) { return a1[q + W]; }, jx1, jy1);
+            o0 += cb.x * (wx * jx0 + wy * jy0);
+            o1 += cb.y * (wx * jx1 + wy * jy1);
+          }
+          store_split2(oh + col, ol ? ol + col : nullptr, o0, o1);
         }
       }
     }
@@ -230,10 +259,10 @@ __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec
   }
 }
 
-// [M x K] bf16 row-major -> [K x Mp] (Mp = ld of the output), columns >= M zero.
+// [M x K] bf16 row-major -> [K x Mp] (row stride ld_out), columns in [M, Mp) zero.
 // 64 x 64 tiles through shared memory, 32-bit accesses.
 __global__ void k_transpose_bf16(const __nv_bfloat16 *__restrict__ in, int M, int K, int ld_in,
-                                 __nv_bfloat16 *__restrict__ out, int Mp) {
+                                 __nv_bfloat16 *__restrict__ out, int Mp, int ld_out) {
   __shared__ __nv_bfloat16 tile[64][66];
   const int k0 = blockIdx.x * 64, m0 = blockIdx.y * 64;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
@@ -251,15 +280,25 @@ __global__ void k_transpose_bf16(const __nv_bfloat16 *__restrict__ in, int M, in
       __nv_bfloat162 v;
       v.x = tile[2 * tx][r];
       v.y = tile[2 * tx + 1][r];
-      *reinterpret_cast<__nv_bfloat162 *>(out + (int64_t)k * Mp + m) = v;
+      *reinterpret_cast<__nv_bfloat162 *>(out + (int64_t)k * ld_out + m) = v;
     }
   }
 }
 
+// Up to three per-edge row sets F_u (grouped layout, row stride ld[u]) and
+// their per-channel coefficients: the reduced rows are
+//   Z = sum_u A_u F_u - Omega (sum_{u<2} B_u F_u)      (|m| up to mmax + 1)
+struct ScatterTerms {
+  const float *F[3];
+  int ld[3];
+  Coef A[3];
+  Coef B[2];
+};
+
 // ---------------------------------------------------------------------------
 // Inverse rotation on reduction, node-centric.  For every node whose sorted
 // segment meets this chunk, out[n][(l,m')][c] += sum over its chunk edges of
-// sum_m D^l[m][m'] * F[i][row(l,m)][c] (* gate).  One block per node,
+// sum_m D^l[m][m'] Z[i][(l,m)][c], Z as described by ScatterTerms.  One block per node,
 // threads over channel pairs, the node's sums in shared memory; the chunks
 // run in stream order, so every output element is updated by one thread at
 // a time and the sum order is fixed.
@@ -267,12 +306,14 @@ __global__ void k_transpose_bf16(const __nv_bfloat16 *__restrict__ in, int M, in
 template <int MM>
 __global__ void k_scatter_nodes(Layout y, int64_t e0, int M, const EdgeRec *__restrict__ rec,
                                 const int *__restrict__ offsets, const float *__restrict__ D,
-                                const float *__restrict__ F, int ldf, int side,
-                                const float *__restrict__ gate, float *__restrict__ out) {
+                                ScatterTerms t, int side, const float *__restrict__ omega,
+                                float *__restrict__ out) {
   extern __shared__ float acc[];  // [S][C]
   if (M <= 0) return;
+  constexpr int W = MM + 1;
   const int C = side ? y.co : y.ci;
   const int *col_off = side ? y.kout_off : y.kin_off;
+  const bool wide = t.B[0].mode != 0 || t.B[1].mode != 0;
   const int n_first = rec[0].key, n_last = rec[M - 1].key;
   for (int n = n_first + blockIdx.x; n <= n_last; n += gridDim.x) {
     int b = offsets[n] - static_cast<int>(e0), e = offsets[n + 1] - static_cast<int>(e0);
@@ -284,30 +325,65 @@ __global__ void k_scatter_nodes(Layout y, int64_t e0, int M, const EdgeRec *__re
     for (int c = 2 * threadIdx.x; c < C; c += 2 * blockDim.x) {
       for (int i = b; i < e; ++i) {
         const float *De = D + (int64_t)i * y.dsz;
-        const float *Fi = F + (int64_t)i * ldf;
-        float2 gv = make_float2(1.f, 1.f);
-        if (gate) gv = load2(gate + (int64_t)i * C + c);
-        for (int l = 0; l <= y.L; ++l) {
-          float2 v[2 * MM + 1];
+        float2 ka[3], kb[2];
 #pragma unroll
-          for (int m = -MM; m <= MM; ++m) {
-            v[m + MM] = make_float2(0.f, 0.f);
-            if (m < -l || m > l) continue;
+        for (int u = 0; u < 3; ++u) ka[u] = t.F[u] ? coef2(t.A[u], i, C, c) : make_float2(0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) kb[u] = t.F[u] ? coef2(t.B[u], i, C, c) : make_float2(0.f, 0.f);
+        float wx = 0.f, wy = 0.f;
+        if (wide) {
+          wx = omega[4 * (int64_t)i];
+          wy = omega[4 * (int64_t)i + 1];
+        }
+        for (int l = 0; l <= y.L; ++l) {
+          float z0[2 * W + 1], z1[2 * W + 1], q0[2 * W + 1], q1[2 * W + 1];
+#pragma unroll
+          for (int m = -W; m <= W; ++m) {
+            z0[m + W] = z1[m + W] = q0[m + W] = q1[m + W] = 0.f;
+            if (m < -l || m > l || m < -MM || m > MM) continue;
             int g, j;
             lm_group_row(y, l, m, g, j);
-            const float2 f = load2(Fi + col_off[g] + j * C + c);
-            v[m + MM] = make_float2(f.x * gv.x, f.y * gv.y);
+#pragma unroll
+            for (int u = 0; u < 3; ++u) {
+              if (!t.F[u]) continue;
+              const float2 f = load2(t.F[u] + (int64_t)i * t.ld[u] + col_off[g] + j * C + c);
+              z0[m + W] += ka[u].x * f.x;
+              z1[m + W] += ka[u].y * f.y;
+              if (u < 2) {
+                q0[m + W] += kb[u].x * f.x;
+                q1[m + W] += kb[u].y * f.y;
+              }
+            }
+          }
+          const int top = wide ? W : MM;
+          if (wide) {
+            float r0[2 * W + 1], r1[2 * W + 1];
+#pragma unroll
+            for (int m = -W; m <= W; ++m) {
+              r0[m + W] = r1[m + W] = 0.f;
+              if (m < -l || m > l) continue;
+              float jx0, jy0, jx1, jy1;
+              gen_xy(l, m, [&](int qq) { return (qq < -MM || qq > MM) ? 0.f : q0[qq + W]; }, jx0, jy0);
+              gen_xy(l, m, [&](int qq) { return (qq < -MM || qq > MM) ? 0.f : q1[qq + W]; }, jx1, jy1);
+              r0[m + W] = wx * jx0 + wy * jy0;
+              r1[m + W] = wx * jx1 + wy * jy1;
+            }
+#pragma unroll
+            for (int m = -W; m <= W; ++m) {
+              z0[m + W] -= r0[m + W];
+              z1[m + W] -= r1[m + W];
+            }
           }
           const float *Dl = De + dblock_off(l);
           const int w = 2 * l + 1;
           for (int mp = -l; mp <= l; ++mp) {
             float t0 = 0.f, t1 = 0.f;
 #pragma unroll
-            for (int m = -MM; m <= MM; ++m) {
-              if (m < -l || m > l) continue;
+            for (int m = -W; m <= W; ++m) {
+              if (m < -l || m > l || m < -top || m > top) continue;
               const float dv = Dl[(m + l) * w + mp + l];
-              t0 += dv * v[m + MM].x;
-              t1 += dv * v[m + MM].y;
+              t0 += dv * z0[m + W];
+              t1 += dv * z1[m + W];
             }
             float *a = acc + (l * l + l + mp) * C + c;
             a[0] += t0;
@@ -541,18 +617,27 @@ __global__ void k_edge_final(Layout y, float cutoff, int M, const EdgeRec *__res
   }
 }
 
-// Radial-gate gradients, stage 1: each block sums phi_k(d_i) Gg[i][c'] (and
-// Gg for the bias row k = nr) over a tile of RAD_TILE edges into
-// part[block][k][c'].  Stage 2 adds the blocks in order.  Deterministic.
+// Radial-gate gradients, stage 1: each block sums, over a tile of RAD_TILE
+// edges, phi_k(d_i) A[i][c'] + phi'_k(d_i) dd_i B[i][c'] (rows k < nr) and
+// A[i][c'] (bias row k = nr) into part[block][k][c'].  B (and dd_i =
+// omega[i][2]) is optional.  Stage 2 adds the blocks in order.
 constexpr int RAD_TILE = 256;
 __global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__restrict__ geo,
-                              const float *__restrict__ Gg, float *__restrict__ part) {
-  extern __shared__ float phi[];  // [RAD_TILE][nr]
+                              const float *__restrict__ Ag, const float *__restrict__ Bg,
+                              const float *__restrict__ omega, float *__restrict__ part) {
+  extern __shared__ float phi[];  // [2][RAD_TILE][nr]
   const int i0 = blockIdx.x * RAD_TILE;
   const int n = (M - i0) < RAD_TILE ? (M - i0) : RAD_TILE;
+  float *dphi = phi + RAD_TILE * y.nr;
+  const float sig = cutoff / static_cast<float>(y.nr - 1);
   for (int t = threadIdx.x; t < n * y.nr; t += blockDim.x) {
     const int i = t / y.nr, k = t % y.nr;
-    phi[t] = rbf_val(geo[(int64_t)(i0 + i) * GEO], k, y, cutoff);
+    const float d = geo[(int64_t)(i0 + i) * GEO];
+    phi[t] = rbf_val(d, k, y, cutoff);
+    if (Bg) {
+      const float u = (d - sig * static_cast<float>(k)) / sig;
+      dphi[t] = (-u / sig) * phi[t] * omega[4 * (int64_t)(i0 + i) + 2];
+    }
   }
   __syncthreads();
   const int P = (y.nr + 1) * y.co;
@@ -560,9 +645,11 @@ __global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__rest
     const int k = pidx / y.co, c = pidx % y.co;
     float s = 0.f;
     if (k < y.nr) {
-      for (int i = 0; i < n; ++i) s += phi[i * y.nr + k] * Gg[(int64_t)(i0 + i) * y.co + c];
+      for (int i = 0; i < n; ++i) s += phi[i * y.nr + k] * Ag[(int64_t)(i0 + i) * y.co + c];
+      if (Bg)
+        for (int i = 0; i < n; ++i) s += dphi[i * y.nr + k] * Bg[(int64_t)(i0 + i) * y.co + c];
     } else {
-      for (int i = 0; i < n; ++i) s += Gg[(int64_t)(i0 + i) * y.co + c];
+      for (int i = 0; i < n; ++i) s += Ag[(int64_t)(i0 + i) * y.co + c];
     }
     part[(int64_t)blockIdx.x * P + pidx] = s;
   }
@@ -580,6 +667,120 @@ __global__ void k_rad_reduce(Layout y, int nblk, const float *__restrict__ part,
     if (grad_w_rad) grad_w_rad[k * y.co + c] += s;
   } else if (grad_b) {
     grad_b[c] += s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Double backward, per edge: the frame turn and gate change that the edge
+// cotangent gg_r induces.  With u = R gg_r / d: omega = (u_y, -u_x) (the
+// z component, a roll of the frame, does not change the output),
+// dd = r_hat . gg_r and dg[c'] = dd * sum_k W_rad[k][c'] phi'_k(d).
+// omega[i] = (w_x, w_y, dd, 0).  One warp per edge.
+// ---------------------------------------------------------------------------
+__global__ void k_edge_omega(Layout y, float cutoff, int M, const EdgeRec *__restrict__ rec,
+                             const float *__restrict__ geo, const float *__restrict__ gg_r,
+                             const float *__restrict__ w_rad, float *__restrict__ omega,
+                             float *__restrict__ dgate) {
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  const float sig = cutoff / static_cast<float>(y.nr - 1);
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
+    const float *gr = geo + (int64_t)i * GEO;
+    const float d = gr[0];
+    const int e = rec[i].eid;
+    const float g0 = gg_r[3 * (int64_t)e], g1 = gg_r[3 * (int64_t)e + 1], g2 = gg_r[3 * (int64_t)e + 2];
+    const float *R = gr + 4;
+    const float inv = d > 0.f ? 1.f / d : 0.f;
+    const float ux = (R[0] * g0 + R[1] * g1 + R[2] * g2) * inv;
+    const float uy = (R[3] * g0 + R[4] * g1 + R[5] * g2) * inv;
+    const float dd = gr[1] * g0 + gr[2] * g1 + gr[3] * g2;
+    if (lane == 0) {
+      omega[4 * (int64_t)i] = uy;
+      omega[4 * (int64_t)i + 1] = -ux;
+      omega[4 * (int64_t)i + 2] = dd;
+      omega[4 * (int64_t)i + 3] = 0.f;
+    }
+    float dphi[2];
+    for (int u = 0; u < 2; ++u) {
+      const int k = lane + 32 * u;
+      const float t = (d - sig * static_cast<float>(k)) / sig;
+      dphi[u] = (k < y.nr) ? (-t / sig) * __expf(-0.5f * t * t) : 0.f;
+    }
+    for (int c0 = 0; c0 < y.co; c0 += 32) {
+      const int c = c0 + lane;
+      float dg = 0.f;
+      for (int k = 0; k < y.nr; ++k) {
+        const float dk = __shfl_sync(0xffffffffu, dphi[k >> 5], k & 31);
+        if (c < y.co) dg += w_rad[k * y.co + c] * dk;
+      }
+      if (c < y.co) dgate[(int64_t)i * y.co + c] = dd * dg;
+    }
+  }
+}
+
+// Double backward, per edge and output channel:
+//   A[c'] = sum_{kept rows} (Omega Gy~)(V) + Gy~ dV + Gy~ V~    (d Q / d g)
+//   B[c'] = sum_{kept rows} Gy~ V                              (d Q / d dg)
+// with Gy~ = D G[dst] (rows up to mmax + 1 for Omega), V = M a, dV = M(Omega a),
+// V~ = M(D gg_x[src]) (optional).  One warp per edge, lanes over channels.
+template <int MM>
+__global__ void k_edge_terms2(Layout y, int M, const EdgeRec *__restrict__ rec,
+                              const float *__restrict__ D, const float *__restrict__ G,
+                              const float *__restrict__ omega, const float *__restrict__ V,
+                              const float *__restrict__ dV, const float *__restrict__ Vt,
+                              float *__restrict__ Aout, float *__restrict__ Bout) {
+  constexpr int W = MM + 1;
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
+    const EdgeRec r = rec[i];
+    const float *De = D + (int64_t)i * y.dsz;
+    const float *Gn = G + (int64_t)r.dst * y.S * y.co;
+    const float wx = omega ? omega[4 * (int64_t)i] : 0.f;
+    const float wy = omega ? omega[4 * (int64_t)i + 1] : 0.f;
+    const int64_t ro = (int64_t)i * y.KG;
+    for (int c = 2 * lane; c < y.co; c += 64) {
+      float A0 = 0.f, A1 = 0.f, B0 = 0.f, B1 = 0.f;
+      for (int l = 0; l <= y.L; ++l) {
+        float b0[2 * W + 1], b1[2 * W + 1];
+#pragma unroll
+        for (int k = 0; k < 2 * W + 1; ++k) b0[k] = b1[k] = 0.f;
+        const float *Dl = De + dblock_off(l);
+        const int w = 2 * l + 1;
+        for (int mp = -l; mp <= l; ++mp) {
+          const float2 gx = load2(Gn + (l * l + l + mp) * y.co + c);
+#pragma unroll
+          for (int m = -W; m <= W; ++m) {
+            if (m < -l || m > l) continue;
+            const float dv = Dl[(m + l) * w + mp + l];
+            b0[m + W] += dv * gx.x;
+            b1[m + W] += dv * gx.y;
+          }
+        }
+#pragma unroll
+        for (int m = -MM; m <= MM; ++m) {
+          if (m < -l || m > l) continue;
+          int g, j;
+          lm_group_row(y, l, m, g, j);
+          const int64_t col = ro + y.kout_off[g] + j * y.co + c;
+          const float2 v = load2(V + col);
+          const float2 dv = dV ? load2(dV + col) : make_float2(0.f, 0.f);
+          float jx0, jy0, jx1, jy1;
+          gen_xy(l, m, [&](int q) { return b0[q + W]; }, jx0, jy0);
+          gen_xy(l, m, [&](int q) { return b1[q + W]; }, jx1, jy1);
+          const float og0 = wx * jx0 + wy * jy0, og1 = wx * jx1 + wy * jy1;
+          A0 += og0 * v.x + b0[m + W] * dv.x;
+          A1 += og1 * v.y + b1[m + W] * dv.y;
+          if (Vt) {
+            const float2 vt = load2(Vt + col);
+            A0 += b0[m + W] * vt.x;
+            A1 += b1[m + W] * vt.y;
+          }
+          B0 += b0[m + W] * v.x;
+          B1 += b1[m + W] * v.y;
+        }
+      }
+      *reinterpret_cast<float2 *>(Aout + (int64_t)i * y.co + c) = make_float2(A0, A1);
+      *reinterpret_cast<float2 *>(Bout + (int64_t)i * y.co + c) = make_float2(B0, B1);
+    }
   }
 }
 

@@ -65,8 +65,10 @@ struct Plan {
   bool split = true, xbf16 = false;
   size_t total = 0;
   // byte offsets
+  int na = 1, ngv = 1;  // row-stacked operand sets (double backward uses 3 and 2)
   size_t status, counts, cursor, offsets, perm, rec, geo, D, gate, wst_hi, wst_lo, wtr_hi, wtr_lo,
-      a_hi, a_lo, V, gv_hi, gv_lo, aT_hi, aT_lo, gvT_hi, gvT_lo, Ga, Gg, h, dws, radp;
+      a_hi, a_lo, V, gv_hi, gv_lo, aT_hi, aT_lo, gvT_hi, gvT_lo, Ga, Gg, h, dws, radp, omega,
+      dgate, tA, tB;
 };
 
 size_t take(size_t &cur, size_t bytes) {
@@ -95,12 +97,17 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
   p.E = E;
   p.split = d->dtype == SO2_F32;
   p.xbf16 = d->dtype == SO2_BF16;
-  const int64_t ch = E < CHUNK_MAX ? E : CHUNK_MAX;
+  const int64_t cap = which == SO2_WS_DOUBLE_BACKWARD ? CHUNK_MAX / 2 : CHUNK_MAX;
+  const int64_t ch = E < cap ? E : cap;
   p.chunk = static_cast<int>(round_up(static_cast<int>(ch > 0 ? ch : 1), 128));
   p.chunkp = p.chunk;  // multiple of 64 already
   const Layout &y = p.y;
   const bool bwd = which >= SO2_WS_BACKWARD;
+  const bool dbl = which == SO2_WS_DOUBLE_BACKWARD;
+  p.na = dbl ? 3 : 1;
+  p.ngv = dbl ? 2 : 1;
   const int lo = p.split ? 1 : 0;
+  const size_t na = p.na, ngv = p.ngv;
   size_t c = 0;
   p.status = take(c, 256);
   p.counts = take(c, sizeof(int) * (N + 1));
@@ -115,21 +122,27 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
   p.wst_lo = take(c, 2ull * y.WR * y.WK * lo);
   p.wtr_hi = take(c, 2ull * y.WTR * y.WTK);
   p.wtr_lo = take(c, 2ull * y.WTR * y.WTK * lo);
-  p.a_hi = take(c, 2ull * p.chunk * y.KA);
-  p.a_lo = take(c, 2ull * p.chunk * y.KA * lo);
-  p.V = take(c, 4ull * p.chunk * y.KG);
+  p.a_hi = take(c, 2ull * na * p.chunk * y.KA);
+  p.a_lo = take(c, 2ull * na * p.chunk * y.KA * lo);
+  p.V = take(c, 4ull * na * p.chunk * y.KG);
   if (bwd) {
-    p.gv_hi = take(c, 2ull * p.chunk * y.KG);
-    p.gv_lo = take(c, 2ull * p.chunk * y.KG * lo);
-    p.aT_hi = take(c, 2ull * y.KA * p.chunkp);
-    p.aT_lo = take(c, 2ull * y.KA * p.chunkp * lo);
-    p.gvT_hi = take(c, 2ull * y.KG * p.chunkp);
-    p.gvT_lo = take(c, 2ull * y.KG * p.chunkp * lo);
-    p.Ga = take(c, 4ull * p.chunk * y.KA);
+    p.gv_hi = take(c, 2ull * ngv * p.chunk * y.KG);
+    p.gv_lo = take(c, 2ull * ngv * p.chunk * y.KG * lo);
+    p.aT_hi = take(c, 2ull * y.KA * na * p.chunkp);
+    p.aT_lo = take(c, 2ull * y.KA * na * p.chunkp * lo);
+    p.gvT_hi = take(c, 2ull * y.KG * ngv * p.chunkp);
+    p.gvT_lo = take(c, 2ull * y.KG * ngv * p.chunkp * lo);
+    p.Ga = take(c, 4ull * ngv * p.chunk * y.KA);
     p.Gg = take(c, 4ull * p.chunk * y.co);
     p.h = take(c, 8ull * p.chunk);
     p.dws = take(c, 4ull * y.WR * y.WK);
     p.radp = take(c, 4ull * ((p.chunk + RAD_TILE - 1) / RAD_TILE) * (y.nr + 1) * y.co);
+  }
+  if (dbl) {
+    p.omega = take(c, 16ull * p.chunk);
+    p.dgate = take(c, 4ull * p.chunk * y.co);
+    p.tA = take(c, 4ull * p.chunk * y.co);
+    p.tB = take(c, 4ull * p.chunk * y.co);
   }
   p.total = (c + 1023) & ~static_cast<size_t>(1023);
   return p;
@@ -321,19 +334,21 @@ so2_status build_maps(Ctx &c, bool bwd) {
   const Layout &y = P.y;
   void *ws = c.ws;
   bool ok = true;
-  ok &= make_map(&c.m_a_hi, at<void>(ws, P.a_hi), P.chunk, y.KA, y.KA, GEMM_BM);
-  ok &= make_map(&c.m_a_lo, at<void>(ws, P.split ? P.a_lo : P.a_hi), P.chunk, y.KA, y.KA, GEMM_BM);
+  const int64_t ra = (int64_t)P.na * P.chunk, rg = (int64_t)P.ngv * P.chunk;
+  const int64_t ca = (int64_t)P.na * P.chunkp, cg = (int64_t)P.ngv * P.chunkp;
+  ok &= make_map(&c.m_a_hi, at<void>(ws, P.a_hi), ra, y.KA, y.KA, GEMM_BM);
+  ok &= make_map(&c.m_a_lo, at<void>(ws, P.split ? P.a_lo : P.a_hi), ra, y.KA, y.KA, GEMM_BM);
   ok &= make_map(&c.m_wst_hi, at<void>(ws, P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN);
   ok &= make_map(&c.m_wst_lo, at<void>(ws, P.split ? P.wst_lo : P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN);
   if (bwd) {
-    ok &= make_map(&c.m_v_hi, at<void>(ws, P.gv_hi), P.chunk, y.KG, y.KG, GEMM_BM);
-    ok &= make_map(&c.m_v_lo, at<void>(ws, P.split ? P.gv_lo : P.gv_hi), P.chunk, y.KG, y.KG, GEMM_BM);
+    ok &= make_map(&c.m_v_hi, at<void>(ws, P.gv_hi), rg, y.KG, y.KG, GEMM_BM);
+    ok &= make_map(&c.m_v_lo, at<void>(ws, P.split ? P.gv_lo : P.gv_hi), rg, y.KG, y.KG, GEMM_BM);
     ok &= make_map(&c.m_wtr_hi, at<void>(ws, P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN);
     ok &= make_map(&c.m_wtr_lo, at<void>(ws, P.split ? P.wtr_lo : P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN);
-    ok &= make_map(&c.m_aT_hi, at<void>(ws, P.aT_hi), y.KA, P.chunkp, P.chunkp, GEMM_BN);
-    ok &= make_map(&c.m_aT_lo, at<void>(ws, P.split ? P.aT_lo : P.aT_hi), y.KA, P.chunkp, P.chunkp, GEMM_BN);
-    ok &= make_map(&c.m_gvT_hi, at<void>(ws, P.gvT_hi), y.KG, P.chunkp, P.chunkp, GEMM_BM);
-    ok &= make_map(&c.m_gvT_lo, at<void>(ws, P.split ? P.gvT_lo : P.gvT_hi), y.KG, P.chunkp, P.chunkp, GEMM_BM);
+    ok &= make_map(&c.m_aT_hi, at<void>(ws, P.aT_hi), y.KA, ca, ca, GEMM_BN);
+    ok &= make_map(&c.m_aT_lo, at<void>(ws, P.split ? P.aT_lo : P.aT_hi), y.KA, ca, ca, GEMM_BN);
+    ok &= make_map(&c.m_gvT_hi, at<void>(ws, P.gvT_hi), y.KG, cg, cg, GEMM_BM);
+    ok &= make_map(&c.m_gvT_lo, at<void>(ws, P.split ? P.gvT_lo : P.gvT_hi), y.KG, cg, cg, GEMM_BM);
   }
   return ok ? SO2_OK : SO2_ERR_CUDA;
 }
@@ -395,40 +410,115 @@ so2_status chunk_prep(Ctx &c, int64_t e0, int M, const int64_t *ei, const float 
   return SO2_OK;
 }
 
-so2_status rotate_x(Ctx &c, int M, const void *x) {
+// Rotation on gather into the grouped layout (rows of `out_*`, stride ld):
+// out = A * D X + B * Omega D X  (see k_rotate_gather).
+so2_status rotate(Ctx &c, int M, const void *X, bool xbf16, int side, int use_src, Coef A, Coef B,
+                  const float *omega, __nv_bfloat16 *hi, __nv_bfloat16 *lo, int ld) {
   const Plan &P = c.P;
-  __nv_bfloat16 *hi = at<__nv_bfloat16>(c.ws, P.a_hi), *lo = P.split ? at<__nv_bfloat16>(c.ws, P.a_lo) : nullptr;
   const EdgeRec *rec = at<EdgeRec>(c.ws, P.rec);
   const float *D = at<float>(c.ws, P.D);
-  if (P.xbf16) {
+  if (xbf16) {
     DISPATCH_MM(P.y.mmax, (k_rotate_gather<__nv_bfloat16, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
-                               P.y, M, rec, D, static_cast<const __nv_bfloat16 *>(x), 0, 1,
-                               nullptr, hi, lo, P.y.KA)));
+                               P.y, M, rec, D, static_cast<const __nv_bfloat16 *>(X), side,
+                               use_src, A, B, omega, hi, lo, ld)));
   } else {
     DISPATCH_MM(P.y.mmax, (k_rotate_gather<float, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
-                               P.y, M, rec, D, static_cast<const float *>(x), 0, 1, nullptr, hi,
-                               lo, P.y.KA)));
+                               P.y, M, rec, D, static_cast<const float *>(X), side, use_src, A,
+                               B, omega, hi, lo, ld)));
   }
   CKL();
   return SO2_OK;
 }
 
-// V = rotated features times stacked weights (one group per m).
-so2_status gemm_v(Ctx &c, int M) {
+constexpr Coef ZERO{nullptr, 0};
+constexpr Coef ONE{nullptr, 1};
+inline Coef arr(const float *p) { return Coef{p, 2}; }
+
+// x[src] rotated into rows [row0, row0 + M) of the a-operand planes.
+so2_status rotate_x(Ctx &c, int M, const void *x, bool xbf16, int row0 = 0, Coef A = ONE,
+                    Coef B = ZERO, const float *omega = nullptr) {
+  const Plan &P = c.P;
+  const size_t off = (size_t)row0 * P.y.KA;
+  __nv_bfloat16 *hi = at<__nv_bfloat16>(c.ws, P.a_hi) + off;
+  __nv_bfloat16 *lo = P.split ? at<__nv_bfloat16>(c.ws, P.a_lo) + off : nullptr;
+  return rotate(c, M, x, xbf16, 0, 1, A, B, omega, hi, lo, P.y.KA);
+}
+
+// G[dst] rotated (with coefficients) into rows [row0, row0 + M) of the
+// output-side operand planes.
+so2_status rotate_g(Ctx &c, int M, const float *G, int row0, Coef A, Coef B = ZERO,
+                    const float *omega = nullptr) {
+  const Plan &P = c.P;
+  const size_t off = (size_t)row0 * P.y.KG;
+  __nv_bfloat16 *hi = at<__nv_bfloat16>(c.ws, P.gv_hi) + off;
+  __nv_bfloat16 *lo = P.split ? at<__nv_bfloat16>(c.ws, P.gv_lo) + off : nullptr;
+  return rotate(c, M, G, false, 1, 0, A, B, omega, hi, lo, P.y.KG);
+}
+
+// Transpose rows [row0, row0 + M) of an operand plane pair into column
+// segment `seg` of its transposed planes (columns past M zero up to Kp).
+so2_status transpose_seg(Ctx &c, int M, bool out_side, int row0, int seg) {
+  const Plan &P = c.P;
+  const Layout &y = P.y;
+  const int K = out_side ? y.KG : y.KA;
+  const int nseg = out_side ? P.ngv : P.na;
+  const int ldo = nseg * P.chunkp;
+  const int Kp = round_up(M, 64);
+  const size_t ioff = (size_t)row0 * K, ooff = (size_t)seg * P.chunkp;
+  for (int plane = 0; plane < (P.split ? 2 : 1); ++plane) {
+    const __nv_bfloat16 *in = at<__nv_bfloat16>(
+        c.ws, out_side ? (plane ? P.gv_lo : P.gv_hi) : (plane ? P.a_lo : P.a_hi));
+    __nv_bfloat16 *out = at<__nv_bfloat16>(
+        c.ws, out_side ? (plane ? P.gvT_lo : P.gvT_hi) : (plane ? P.aT_lo : P.aT_hi));
+    k_transpose_bf16<<<dim3((K + 63) / 64, Kp / 64), 256, 0, c.s>>>(in + ioff, M, K, K,
+                                                                    out + ooff, Kp, ldo);
+    CKL();
+  }
+  return SO2_OK;
+}
+
+// dW (+)= (rows seg_g of the output-side operand)^T (rows seg_a of the input side).
+so2_status gemm_dw(Ctx &c, int M, int seg_g, int seg_a) {
+  const Plan &P = c.P;
+  const Layout &y = P.y;
+  const int Kp = round_up(M, 64);
+  GemmLauncher L;
+  for (int g = 0; g < y.ng; ++g)
+    L.add(y.Kout[g], y.Kin[g], Kp, y.kout_off[g], seg_g * P.chunkp, y.kin_off[g],
+          seg_a * P.chunkp, static_cast<long long>(y.wr_off[g]) * y.WK, y.WK);
+  CK(launch_gemm(2, P.split, c.m_gvT_hi, c.m_gvT_lo, c.m_aT_hi, c.m_aT_lo, L.p,
+                 at<float>(c.ws, P.dws), 1, c.st, c.s));
+  return SO2_OK;
+}
+
+// Ga rows = output-side operand rows times the transposed stacked weights.
+so2_status gemm_ga(Ctx &c, int rows) {
   const Plan &P = c.P;
   const Layout &y = P.y;
   GemmLauncher L;
   for (int g = 0; g < y.ng; ++g)
-    L.add(M, y.Kout[g], y.Kin_pad[g], 0, y.kin_off[g], y.wr_off[g], 0, y.kout_off[g], y.KG);
+    L.add(rows, y.Kin[g], y.Kout_pad[g], 0, y.kout_off[g], y.wt_off[g], 0, y.kin_off[g], y.KA);
+  CK(launch_gemm(1, P.split, c.m_v_hi, c.m_v_lo, c.m_wtr_hi, c.m_wtr_lo, L.p,
+                 at<float>(c.ws, P.Ga), 0, c.st, c.s));
+  return SO2_OK;
+}
+
+// V = rotated features times stacked weights (one group per m).
+so2_status gemm_v(Ctx &c, int rows) {
+  const Plan &P = c.P;
+  const Layout &y = P.y;
+  GemmLauncher L;
+  for (int g = 0; g < y.ng; ++g)
+    L.add(rows, y.Kout[g], y.Kin_pad[g], 0, y.kin_off[g], y.wr_off[g], 0, y.kout_off[g], y.KG);
   CK(launch_gemm(0, P.split, c.m_a_hi, c.m_a_lo, c.m_wst_hi, c.m_wst_lo, L.p, at<float>(c.ws, P.V), 0,
                  c.st, c.s));
   return SO2_OK;
 }
 
-// Node-centric inverse rotation on reduction of F (rows of the grouped
-// layout on `side`) into out, for the chunk's nodes.
-so2_status scatter(Ctx &c, int64_t e0, int M, const float *F, int ldf, int side,
-                   const float *gate, float *out) {
+// Node-centric inverse rotation on reduction (see k_scatter_nodes) for the
+// chunk's nodes, on `side` (0: input channels, 1: output channels).
+so2_status scatter(Ctx &c, int64_t e0, int M, const ScatterTerms &t, int side,
+                   const float *omega, float *out) {
   const Plan &P = c.P;
   const Layout &y = P.y;
   const int C = side ? y.co : y.ci;
@@ -441,8 +531,33 @@ so2_status scatter(Ctx &c, int64_t e0, int M, const float *F, int ldf, int side,
   bool ok = true;
   DISPATCH_MM(y.mmax, ok = allow_smem(k_scatter_nodes<MM>, smem);
               if (ok) k_scatter_nodes<MM><<<grid_for(M, 1), threads, smem, c.s>>>(
-                  y, e0, M, rec, off, D, F, ldf, side, gate, out));
+                  y, e0, M, rec, off, D, t, side, omega, out));
   if (!ok) return SO2_ERR_CUDA;
+  CKL();
+  return SO2_OK;
+}
+
+ScatterTerms one_term(const float *F, int ld, Coef A) {
+  ScatterTerms t{};
+  t.F[0] = F;
+  t.ld[0] = ld;
+  t.A[0] = A;
+  return t;
+}
+
+so2_status rad_grads(Ctx &c, int M, const float *Ag, const float *Bg, const float *omega,
+                     float *grad_w_rad, float *grad_b) {
+  const Plan &P = c.P;
+  const Layout &y = P.y;
+  const int nblk = (M + RAD_TILE - 1) / RAD_TILE;
+  const int sm = 2 * RAD_TILE * y.nr * static_cast<int>(sizeof(float));
+  if (!allow_smem(k_rad_partial, sm)) return SO2_ERR_CUDA;
+  k_rad_partial<<<nblk, 256, sm, c.s>>>(y, c.d->rbf_cutoff, M, at<float>(c.ws, P.geo), Ag, Bg,
+                                        omega, at<float>(c.ws, P.radp));
+  CKL();
+  const int Pn = (y.nr + 1) * y.co;
+  k_rad_reduce<<<(Pn + 255) / 256, 256, 0, c.s>>>(y, nblk, at<float>(c.ws, P.radp), grad_w_rad,
+                                                   grad_b);
   CKL();
   return SO2_OK;
 }
@@ -490,9 +605,10 @@ so2_status so2conv_forward(const so2conv_desc *desc, int64_t N, int64_t E, const
   for (int64_t e0 = 0; e0 < E; e0 += P.chunk) {
     const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
     if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 1, prm)) != SO2_OK) return r;
-    if ((r = rotate_x(c, M, x)) != SO2_OK) return r;
+    if ((r = rotate_x(c, M, x, P.xbf16)) != SO2_OK) return r;
     if ((r = gemm_v(c, M)) != SO2_OK) return r;
-    if ((r = scatter(c, e0, M, at<float>(ws, P.V), y.KG, 1, at<float>(ws, P.gate), out)) != SO2_OK)
+    if ((r = scatter(c, e0, M, one_term(at<float>(ws, P.V), y.KG, arr(at<float>(ws, P.gate))), 1,
+                     nullptr, out)) != SO2_OK)
       return r;
   }
   return SO2_OK;
@@ -525,59 +641,28 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
   if (E == 0) return SO2_OK;
   const bool need_v = grad_edge_vec || grad_w_rad || grad_b_rad;
   const bool need_ga = grad_x || grad_edge_vec;
-  const bool need_terms = grad_edge_vec || grad_w_rad || grad_b_rad;
   if ((r = build_maps(c, true)) != SO2_OK) return r;
   if ((r = sort_edges(c, edge_index, 0)) != SO2_OK) return r;
   if ((r = pack_weights(c, prm.w)) != SO2_OK) return r;
   float *dws = at<float>(ws, P.dws);
   if (grad_w) CK(cudaMemsetAsync(dws, 0, 4ull * y.WR * y.WK, c.s));
-  __nv_bfloat16 *gv_hi = at<__nv_bfloat16>(ws, P.gv_hi);
-  __nv_bfloat16 *gv_lo = P.split ? at<__nv_bfloat16>(ws, P.gv_lo) : nullptr;
   for (int64_t e0 = 0; e0 < E; e0 += P.chunk) {
     const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
     if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 0, prm)) != SO2_OK) return r;
-    if ((r = rotate_x(c, M, x)) != SO2_OK) return r;
+    if ((r = rotate_x(c, M, x, P.xbf16)) != SO2_OK) return r;
     // Gv = g * (D G[dst]) on the kept rows
-    DISPATCH_MM(y.mmax, (k_rotate_gather<float, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
-                            y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), grad_out, 1, 0,
-                            at<float>(ws, P.gate), gv_hi, gv_lo, y.KG)));
-    CKL();
+    if ((r = rotate_g(c, M, grad_out, 0, arr(at<float>(ws, P.gate)))) != SO2_OK) return r;
     if (need_v && (r = gemm_v(c, M)) != SO2_OK) return r;
-    if (need_ga) {
-      GemmLauncher L;
-      for (int g = 0; g < y.ng; ++g)
-        L.add(M, y.Kin[g], y.Kout_pad[g], 0, y.kout_off[g], y.wt_off[g], 0, y.kin_off[g], y.KA);
-      CK(launch_gemm(1, P.split, c.m_v_hi, c.m_v_lo, c.m_wtr_hi, c.m_wtr_lo, L.p, at<float>(ws, P.Ga),
-                     0, c.st, c.s));
-    }
+    if (need_ga && (r = gemm_ga(c, M)) != SO2_OK) return r;
     if (grad_w) {
-      const int Kp = round_up(M, 64);
-      const int mt = (Kp + 63) / 64;  // only the columns the product reads
-      k_transpose_bf16<<<dim3((y.KA + 63) / 64, mt), 256, 0, c.s>>>(
-          at<__nv_bfloat16>(ws, P.a_hi), M, y.KA, y.KA, at<__nv_bfloat16>(ws, P.aT_hi), P.chunkp);
-      CKL();
-      k_transpose_bf16<<<dim3((y.KG + 63) / 64, mt), 256, 0, c.s>>>(
-          gv_hi, M, y.KG, y.KG, at<__nv_bfloat16>(ws, P.gvT_hi), P.chunkp);
-      CKL();
-      if (P.split) {
-        k_transpose_bf16<<<dim3((y.KA + 63) / 64, mt), 256, 0, c.s>>>(
-            at<__nv_bfloat16>(ws, P.a_lo), M, y.KA, y.KA, at<__nv_bfloat16>(ws, P.aT_lo), P.chunkp);
-        CKL();
-        k_transpose_bf16<<<dim3((y.KG + 63) / 64, mt), 256, 0, c.s>>>(
-            gv_lo, M, y.KG, y.KG, at<__nv_bfloat16>(ws, P.gvT_lo), P.chunkp);
-        CKL();
-      }
-      GemmLauncher L;
-      for (int g = 0; g < y.ng; ++g)
-        L.add(y.Kout[g], y.Kin[g], Kp, y.kout_off[g], 0, y.kin_off[g], 0,
-              static_cast<long long>(y.wr_off[g]) * y.WK, y.WK);
-      CK(launch_gemm(2, P.split, c.m_gvT_hi, c.m_gvT_lo, c.m_aT_hi, c.m_aT_lo, L.p, dws, 1, c.st,
-                     c.s));
+      if ((r = transpose_seg(c, M, false, 0, 0)) != SO2_OK) return r;
+      if ((r = transpose_seg(c, M, true, 0, 0)) != SO2_OK) return r;
+      if ((r = gemm_dw(c, M, 0, 0)) != SO2_OK) return r;
     }
-    if (grad_x &&
-        (r = scatter(c, e0, M, at<float>(ws, P.Ga), y.KA, 0, nullptr, grad_x)) != SO2_OK)
+    if (grad_x && (r = scatter(c, e0, M, one_term(at<float>(ws, P.Ga), y.KA, ONE), 0, nullptr,
+                               grad_x)) != SO2_OK)
       return r;
-    if (need_terms) {
+    if (need_v) {
       if (P.xbf16) {
         DISPATCH_MM(y.mmax, (k_edge_terms<__nv_bfloat16, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
                                 y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
@@ -599,18 +684,10 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
                                                         prm.w_rad, grad_edge_vec);
         CKL();
       }
-      if (grad_w_rad || grad_b_rad) {
-        const int nblk = (M + RAD_TILE - 1) / RAD_TILE;
-        const int sm = RAD_TILE * y.nr * static_cast<int>(sizeof(float));
-        if (!allow_smem(k_rad_partial, sm)) return SO2_ERR_CUDA;
-        k_rad_partial<<<nblk, 256, sm, c.s>>>(y, desc->rbf_cutoff, M, at<float>(ws, P.geo),
-                                              at<float>(ws, P.Gg), at<float>(ws, P.radp));
-        CKL();
-        const int Pn = (y.nr + 1) * y.co;
-        k_rad_reduce<<<(Pn + 255) / 256, 256, 0, c.s>>>(y, nblk, at<float>(ws, P.radp), grad_w_rad,
-                                                         grad_b_rad);
-        CKL();
-      }
+      if ((grad_w_rad || grad_b_rad) &&
+          (r = rad_grads(c, M, at<float>(ws, P.Gg), nullptr, nullptr, grad_w_rad, grad_b_rad)) !=
+              SO2_OK)
+        return r;
     }
   }
   if (grad_w) {
@@ -620,6 +697,18 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
   return SO2_OK;
 }
 
+// Double backward.  With gg_r the cotangent on grad_edge_vec, each edge's
+// frame turns by Omega = w_x J_x + w_y J_y (dD = Omega D) and its gate moves
+// by dg; with gg_x the cotangent on grad_x.  Writing Gy~ = D G[dst] (kept
+// rows), Gv = g Gy~, a = D x[src], da = trunc(Omega D x[src]),
+// a~ = D gg_x[src], P = g trunc(Omega D G[dst]) + dg Gy~, V = M a,
+// dV = M da, V~ = M a~:
+//   Q = sum_e <P, M a> + <Gv, M da> + <Gv, M a~>
+//   d_x[src]      += D^T (M^T P - Omega M^T Gv)
+//   d_grad_out[d] += D^T (dg V + g dV + g V~ - Omega (g V))
+//   d_W           += P (x) a + Gv (x) da + Gv (x) a~
+//   dQ/dg  = sum_rows (Omega Gy~) V + Gy~ dV + Gy~ V~,  dQ/ddg = sum_rows Gy~ V
+// Pass A runs in source order (d_x), pass B in destination order (the rest).
 so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t E, const void *x,
                                    const int64_t *edge_index, const float *edge_vec,
                                    so2conv_params prm, const float *grad_out, const float *gg_x,
@@ -627,10 +716,134 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
                                    float *d_w_rad, float *d_b_rad, float *d_grad_out,
                                    float *d_edge_vec, void *ws, size_t ws_bytes,
                                    so2_stream_t stream) {
-  (void)desc; (void)N; (void)E; (void)x; (void)edge_index; (void)edge_vec; (void)prm;
-  (void)grad_out; (void)gg_x; (void)gg_edge_vec; (void)d_x; (void)d_w; (void)d_w_rad;
-  (void)d_b_rad; (void)d_grad_out; (void)d_edge_vec; (void)ws; (void)ws_bytes; (void)stream;
-  return SO2_ERR_UNSUPPORTED;
+  if (!desc) return SO2_ERR_INVALID_ARG;
+  if (d_edge_vec) return SO2_ERR_UNSUPPORTED;
+  Plan P;
+  so2_status r = common_checks(desc, N, E, x, edge_index, edge_vec, prm, ws, ws_bytes,
+                               SO2_WS_DOUBLE_BACKWARD, P);
+  if (r != SO2_OK) return r;
+  if (N > 0 && !grad_out) return SO2_ERR_INVALID_ARG;
+  Ctx c;
+  c.d = desc;
+  c.P = P;
+  c.ws = ws;
+  c.s = reinterpret_cast<cudaStream_t>(stream);
+  c.st = at<DevStatus>(ws, P.status);
+  CK(cudaMemsetAsync(c.st, 0, sizeof(DevStatus), c.s));
+  const Layout &y = P.y;
+  const int64_t nw = num_weights(y);
+  if (d_x && N > 0) CK(cudaMemsetAsync(d_x, 0, sizeof(float) * N * y.S * y.ci, c.s));
+  if (d_grad_out && N > 0) CK(cudaMemsetAsync(d_grad_out, 0, sizeof(float) * N * y.S * y.co, c.s));
+  if (d_w) CK(cudaMemsetAsync(d_w, 0, sizeof(float) * nw, c.s));
+  if (d_w_rad) CK(cudaMemsetAsync(d_w_rad, 0, sizeof(float) * y.nr * y.co, c.s));
+  if (d_b_rad) CK(cudaMemsetAsync(d_b_rad, 0, sizeof(float) * y.co, c.s));
+  const bool has_r = gg_edge_vec != nullptr, has_x = gg_x != nullptr;
+  if (E == 0 || (!has_r && !has_x)) return SO2_OK;
+  if ((r = build_maps(c, true)) != SO2_OK) return r;
+  if ((r = pack_weights(c, prm.w)) != SO2_OK) return r;
+  const Coef gate = arr(at<float>(ws, P.gate));
+  const Coef dgate = arr(at<float>(ws, P.dgate));
+  const float *omega = at<float>(ws, P.omega);
+  float *dws = at<float>(ws, P.dws);
+  if (d_w) CK(cudaMemsetAsync(dws, 0, 4ull * y.WR * y.WK, c.s));
+  const int ch = P.chunk;
+
+  // ---- pass A (source order): d_x ----
+  if (d_x && has_r) {
+    if ((r = sort_edges(c, edge_index, 0)) != SO2_OK) return r;
+    for (int64_t e0 = 0; e0 < E; e0 += ch) {
+      const int M = static_cast<int>((E - e0) < ch ? (E - e0) : ch);
+      if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 0, prm)) != SO2_OK) return r;
+      k_edge_omega<<<warp_grid(M, 8), 256, 0, c.s>>>(y, desc->rbf_cutoff, M,
+                                                     at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo),
+                                                     gg_edge_vec, prm.w_rad, at<float>(ws, P.omega),
+                                                     at<float>(ws, P.dgate));
+      CKL();
+      if ((r = rotate_g(c, M, grad_out, 0, dgate, gate, omega)) != SO2_OK) return r;  // P
+      if ((r = rotate_g(c, M, grad_out, ch, gate)) != SO2_OK) return r;              // Gv
+      if ((r = gemm_ga(c, ch + M)) != SO2_OK) return r;  // [M^T P; M^T Gv]
+      ScatterTerms t{};
+      t.F[0] = at<float>(ws, P.Ga);
+      t.ld[0] = y.KA;
+      t.A[0] = ONE;
+      t.F[1] = at<float>(ws, P.Ga) + (size_t)ch * y.KA;
+      t.ld[1] = y.KA;
+      t.B[1] = ONE;
+      if ((r = scatter(c, e0, M, t, 0, omega, d_x)) != SO2_OK) return r;
+    }
+  }
+
+  // ---- pass B (destination order): d_grad_out, radial gate, d_W ----
+  if (d_grad_out || d_w || d_w_rad || d_b_rad) {
+    if ((r = sort_edges(c, edge_index, 1)) != SO2_OK) return r;
+    for (int64_t e0 = 0; e0 < E; e0 += ch) {
+      const int M = static_cast<int>((E - e0) < ch ? (E - e0) : ch);
+      if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 1, prm)) != SO2_OK) return r;
+      if (has_r) {
+        k_edge_omega<<<warp_grid(M, 8), 256, 0, c.s>>>(
+            y, desc->rbf_cutoff, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo), gg_edge_vec,
+            prm.w_rad, at<float>(ws, P.omega), at<float>(ws, P.dgate));
+        CKL();
+      }
+      // a-operand rows: [a; da; a~]
+      if ((r = rotate_x(c, M, x, P.xbf16, 0)) != SO2_OK) return r;
+      if (has_r && (r = rotate_x(c, M, x, P.xbf16, ch, ZERO, ONE, omega)) != SO2_OK) return r;
+      if (has_x && (r = rotate_x(c, M, gg_x, false, 2 * ch)) != SO2_OK) return r;
+      if ((r = gemm_v(c, has_x ? 2 * ch + M : (has_r ? ch + M : M))) != SO2_OK) return r;
+      const float *V = at<float>(ws, P.V);
+      const float *dV = V + (size_t)ch * y.KG;
+      const float *Vt = V + (size_t)2 * ch * y.KG;
+      if (d_grad_out && N > 0) {
+        ScatterTerms t{};
+        t.F[0] = V;
+        t.ld[0] = y.KG;
+        t.A[0] = has_r ? dgate : ZERO;
+        t.B[0] = has_r ? gate : ZERO;
+        if (has_r) {
+          t.F[1] = dV;
+          t.ld[1] = y.KG;
+          t.A[1] = gate;
+        }
+        if (has_x) {
+          t.F[2] = Vt;
+          t.ld[2] = y.KG;
+          t.A[2] = gate;
+        }
+        if ((r = scatter(c, e0, M, t, 1, has_r ? omega : nullptr, d_grad_out)) != SO2_OK) return r;
+      }
+      if (d_w_rad || d_b_rad) {
+        DISPATCH_MM(y.mmax, (k_edge_terms2<MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                                y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), grad_out,
+                                has_r ? omega : nullptr, V, has_r ? dV : nullptr,
+                                has_x ? Vt : nullptr, at<float>(ws, P.tA), at<float>(ws, P.tB))));
+        CKL();
+        if ((r = rad_grads(c, M, at<float>(ws, P.tA), has_r ? at<float>(ws, P.tB) : nullptr,
+                           omega, d_w_rad, d_b_rad)) != SO2_OK)
+          return r;
+      }
+      if (d_w) {
+        if (has_r && (r = rotate_g(c, M, grad_out, 0, dgate, gate, omega)) != SO2_OK) return r;
+        if ((r = rotate_g(c, M, grad_out, ch, gate)) != SO2_OK) return r;
+        if (has_r) {
+          if ((r = transpose_seg(c, M, true, 0, 0)) != SO2_OK) return r;
+          if ((r = transpose_seg(c, M, false, 0, 0)) != SO2_OK) return r;
+          if ((r = transpose_seg(c, M, false, ch, 1)) != SO2_OK) return r;
+        }
+        if ((r = transpose_seg(c, M, true, ch, 1)) != SO2_OK) return r;
+        if (has_x && (r = transpose_seg(c, M, false, 2 * ch, 2)) != SO2_OK) return r;
+        if (has_r) {
+          if ((r = gemm_dw(c, M, 0, 0)) != SO2_OK) return r;  // P (x) a
+          if ((r = gemm_dw(c, M, 1, 1)) != SO2_OK) return r;  // Gv (x) da
+        }
+        if (has_x && (r = gemm_dw(c, M, 1, 2)) != SO2_OK) return r;  // Gv (x) a~
+      }
+    }
+  }
+  if (d_w) {
+    k_unstack_grad<<<dim3(64, y.ng), 256, 0, c.s>>>(y, block_offsets(y), dws, d_w);
+    CKL();
+  }
+  return SO2_OK;
 }
 
 so2_status so2conv_check(void *ws, so2_stream_t stream) {

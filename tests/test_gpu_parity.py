@@ -228,3 +228,54 @@ def test_device_reports_bad_index_and_zero_length_edge():
     assert B.check(DEV) == 7
     B.forward(_desc(p), d["x"], d["edge_index"], d["edge_vec"], d["w"], d["w_rad"], d["b_rad"])
     assert B.check(DEV) == 0
+
+
+# ---------------------------------------------------------------------------
+# double backward
+# ---------------------------------------------------------------------------
+DB_CASES = [
+    ("tiny", lambda: synth.make_problem("tiny")),
+    ("L3M2C32", lambda: _small(L=3, M=2, C=32, n=150, nb=20, seed=12)),
+    ("L2M1C16_two_chunks", lambda: _small(L=2, M=1, C=16, n=600, nb=30, seed=13)),  # 18000 edges
+    ("L4M2C128_bf16", lambda: _small(L=4, M=2, C=128, n=60, nb=20, seed=14, bf16=True)),
+]
+
+
+def _gpu_double_backward(p, gg_x, gg_r):
+    d = _dev(p)
+    t = lambda a: None if a is None else torch.as_tensor(np.asarray(a)).float().to(DEV)  # noqa
+    out = B.double_backward(_desc(p), d["x"], d["edge_index"], d["edge_vec"], d["w"],
+                            d["w_rad"], d["b_rad"], d["grad_out"], gg_x=t(gg_x),
+                            gg_edge_vec=t(gg_r))
+    assert B.check(DEV) == 0
+    return out
+
+
+@pytest.mark.parametrize("which", ["r", "x", "rx"])
+@pytest.mark.parametrize("name,make", DB_CASES, ids=[c[0] for c in DB_CASES])
+def test_double_backward_parity(name, make, which):
+    from helpers import oracle_double_backward
+    p = make()
+    rng = np.random.default_rng(21)
+    gg_r = rng.standard_normal(p.edge_vec.shape) if "r" in which else None
+    gg_x = rng.standard_normal(p.x.shape) if "x" in which else None
+    got = _gpu_double_backward(p, gg_x, gg_r)
+    ref = oracle_double_backward(p, gg_x=gg_x, gg_edge_vec=gg_r)
+    for k in ["d_x", "d_w", "d_w_rad", "d_b_rad", "d_grad_out"]:
+        err = rel_err(got[k], ref[k])
+        assert err < TOL[p.x_bf16], (name, which, k, err)
+
+
+def test_force_training_step_parity():
+    # energy = sum of l = 0 outputs; forces come from grad_edge_vec; a force
+    # loss cotangent on grad_edge_vec is pulled back to the weights.
+    p = synth.make_problem("force", seed=0, n_atoms=120, max_nb=20, lmax=3, mmax=2, c=32)
+    g = _gpu_backward(p, need=["grad_edge_vec"])["grad_edge_vec"]
+    ref = oracle_backward(p)["grad_edge_vec"]
+    assert rel_err(g, ref) < 1e-4
+    gg_r = np.random.default_rng(3).standard_normal(p.edge_vec.shape)
+    got = _gpu_double_backward(p, None, gg_r)
+    from helpers import oracle_double_backward
+    want = oracle_double_backward(p, gg_edge_vec=gg_r)
+    for k in ["d_w", "d_w_rad", "d_b_rad", "d_x"]:
+        assert rel_err(got[k], want[k]) < 1e-4, k
