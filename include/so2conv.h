@@ -145,6 +145,38 @@ so2_status so2conv_edge_frames(int32_t lmax, int64_t n_edges,
                                const float *edge_vec, float *R_out,
                                float *D_out, so2_stream_t stream);
 
+/* Size of the library-owned scratch array behind so2conv_forward_noalloc. */
+#define SO2_NOALLOC_WORKSPACE_BYTES (96u << 20)
+
+/* Forward that allocates nothing and needs no caller workspace.
+ *
+ * No counterpart on the pages: this exists for callers that cannot call
+ * cudaMalloc (or any allocating routine) at the point where they run the
+ * convolution -- for example code that executes inside another component's
+ * stream capture, a plugin whose host application owns all device memory, or
+ * a real-time loop that must not touch the allocator.  Such a caller still
+ * passes its own inputs and `out`; the scratch memory comes from a fixed
+ * device array of SO2_NOALLOC_WORKSPACE_BYTES inside this library, which
+ * every GPU that loads the library holds until the process exits.
+ *
+ * Same arguments and results as so2conv_forward, without ws / ws_bytes.
+ * Problems whose forward workspace (so2conv_workspace_size with
+ * SO2_WS_FORWARD) exceeds the array are rejected with SO2_ERR_WORKSPACE
+ * before anything is launched.  The first call on each device looks up the
+ * array's device address with that device current; make that first call
+ * before any stream capture.  All calls share the one array, which keeps the
+ * last call's contents (each call re-initialises what it reads), so calls
+ * that can overlap on the GPU -- different streams, or different host
+ * threads -- race and must be serialised by the caller.  Device-side input
+ * problems (bad index, zero-length edge) are recorded in the shared array,
+ * where so2conv_check cannot see them: validate inputs first, or use
+ * so2conv_forward. */
+so2_status so2conv_forward_noalloc(const so2conv_desc *desc, int64_t n_nodes,
+                                   int64_t n_edges, const void *x,
+                                   const int64_t *edge_index,
+                                   const float *edge_vec, so2conv_params params,
+                                   float *out, so2_stream_t stream);
+
 /* Number of kernels this library has launched in this process (all entry
  * points, all devices).  A plain counter, not thread safe. */
 long long so2conv_launch_count(void);

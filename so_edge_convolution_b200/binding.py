@@ -71,6 +71,8 @@ def load():
     lib.so2conv_status_string.restype = ctypes.c_char_p
     lib.so2conv_edge_frames.argtypes = [ctypes.c_int32, i64, vp, vp, vp, vp]
     lib.so2conv_edge_frames.restype = ctypes.c_int
+    lib.so2conv_forward_noalloc.argtypes = [pd, i64, i64, vp, vp, vp, Params, vp, vp]
+    lib.so2conv_forward_noalloc.restype = ctypes.c_int
     lib.so2conv_launch_count.argtypes = []
     lib.so2conv_launch_count.restype = ctypes.c_longlong
     lib.so2conv_profile_enable.argtypes = [ctypes.c_int]
@@ -260,3 +262,20 @@ def profile_read():
                     "so2conv_profile_read")
         res[k] = (n.value, ms.value)
     return res
+
+
+def forward_noalloc(desc, x, edge_index, edge_vec, w, w_rad, b_rad, out=None):
+    """so2conv_forward_noalloc: the forward on the library's own scratch array
+    (no workspace argument, nothing allocated by the library)."""
+    lib = load()
+    x, edge_index, edge_vec, w, w_rad, b_rad = map(_c, (x, edge_index, edge_vec, w, w_rad, b_rad))
+    N, E = x.shape[0], edge_index.shape[1]
+    if out is None:
+        out = torch.empty((N, (desc.lmax + 1) ** 2, desc.c_out), dtype=torch.float32,
+                          device=x.device)
+    code = lib.so2conv_forward_noalloc(ctypes.byref(desc), N, E, _ptr(x), _ptr(edge_index),
+                                       _ptr(edge_vec), Params(_ptr(w).value, _ptr(w_rad).value,
+                                                              _ptr(b_rad).value),
+                                       _ptr(out), _stream(x.device))
+    _check_call(code, "so2conv_forward_noalloc")
+    return out

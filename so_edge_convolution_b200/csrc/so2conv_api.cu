@@ -562,6 +562,11 @@ so2_status rad_grads(Ctx &c, int M, const float *Ag, const float *Bg, const floa
   return SO2_OK;
 }
 
+// Library-owned scratch for so2conv_forward_noalloc (see its declaration).
+static __device__ __align__(256) unsigned char g_noalloc_ws[SO2_NOALLOC_WORKSPACE_BYTES];
+constexpr int NOALLOC_MAX_DEVICES = 64;
+void *g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {nullptr};
+
 }  // namespace
 
 // ============================================================================
@@ -844,6 +849,28 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
     CKL();
   }
   return SO2_OK;
+}
+
+so2_status so2conv_forward_noalloc(const so2conv_desc *desc, int64_t N, int64_t E,
+                                   const void *x, const int64_t *edge_index,
+                                   const float *edge_vec, so2conv_params prm, float *out,
+                                   so2_stream_t stream) {
+  if (!desc_ok(desc)) return desc ? SO2_ERR_UNSUPPORTED : SO2_ERR_INVALID_ARG;
+  if (N < 0 || E < 0) return SO2_ERR_INVALID_ARG;
+  const size_t need = make_plan(desc, N, E, SO2_WS_FORWARD).total;
+  if (need > SO2_NOALLOC_WORKSPACE_BYTES) return SO2_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES)
+    return SO2_ERR_CUDA;
+  if (!g_noalloc_ptr[dev]) {
+    // the host-side name of the array is not a device address: ask the
+    // runtime for this device's copy (once per device, this device current)
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || !p) return SO2_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  return so2conv_forward(desc, N, E, x, edge_index, edge_vec, prm, out, g_noalloc_ptr[dev],
+                         SO2_NOALLOC_WORKSPACE_BYTES, stream);
 }
 
 so2_status so2conv_check(void *ws, so2_stream_t stream) {
