@@ -33,8 +33,19 @@ sys.path.insert(0, ROOT)
 from so_edge_convolution_b200 import synth  # noqa: E402
 
 METRIC = "SO(2)-conv edges/sec (fwd+bwd, lmax=4, C=128) and % of roofline"
-WORKLOAD = ("eSEN-like: N=2000 atoms periodic at 0.1/A^3, 30 nearest within 6 A (E=60000), "
-            "lmax=4, mmax=2, C=128, 16 RBFs, f32 features and weights, forward+backward")
+# name -> (synthetic problem, workload text, products per step, f32 split path)
+CONFIGS = {
+    "esen": ("esen", "eSEN-like: N=2000 atoms periodic at 0.1/A^3, 30 nearest within 6 A "
+             "(E=60000), lmax=4, mmax=2, C=128, 16 RBFs, f32 features and weights, "
+             "forward+backward", 4),
+    "force": ("force", "force-training step on the eSEN-like graph: forward, backward to the "
+              "edge vectors, force assembly and loss, double backward to the weights, f32", 7),
+    "uma": ("uma", "UMA-like: N=5000 atoms, 30 nearest within 6 A (E=150000), lmax=6, mmax=2, "
+            "C=128, bf16 features and weights, f32 accumulation, forward+backward", 4),
+    "large": ("large", "Large periodic: N=20000 atoms, 50 nearest within 6 A (E=1000000), "
+              "lmax=4, mmax=2, C=128, bf16 features, f32 accumulation, forward+backward", 4),
+}
+WORKLOAD = CONFIGS["esen"][1]
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 
 
@@ -200,28 +211,55 @@ def run_ours(args, world, rank, local):
     build.build()
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
-    p = synth.make_problem("esen", seed=rank)
+    prob, workload, n_products = CONFIGS[args.config]
+    p = synth.make_problem(prob, seed=rank)
     E = p.n_edges
-    desc = B.make_desc(p.lmax, p.mmax, p.c_in, p.c_out, p.n_rbf, p.rbf_cutoff, B.SO2_F32)
+    bf16 = p.x_bf16
+    xdt = torch.bfloat16 if bf16 else torch.float32
+    wdt = torch.bfloat16 if bf16 else torch.float32
+    desc = B.make_desc(p.lmax, p.mmax, p.c_in, p.c_out, p.n_rbf, p.rbf_cutoff,
+                       B.SO2_BF16 if bf16 else B.SO2_F32)
     host = {
-        "x": torch.from_numpy(p.x.astype(np.float32)).pin_memory(),
+        "x": torch.from_numpy(p.x).to(xdt).pin_memory(),
         "edge_index": torch.from_numpy(p.edge_index).pin_memory(),
         "edge_vec": torch.from_numpy(p.edge_vec.astype(np.float32)).pin_memory(),
-        "w": torch.from_numpy(p.w.astype(np.float32)).pin_memory(),
+        "w": torch.from_numpy(p.w).to(wdt).pin_memory(),
         "w_rad": torch.from_numpy(p.w_rad.astype(np.float32)).pin_memory(),
         "b_rad": torch.from_numpy(p.b_rad.astype(np.float32)).pin_memory(),
         "grad_out": torch.from_numpy(p.grad_out.astype(np.float32)).pin_memory(),
+        "f_ref": torch.from_numpy(p.f_ref.astype(np.float32)).pin_memory(),
     }
     d = {k: v.to(dev) for k, v in host.items()}
     ws = B.Workspace(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def step(t):
+    def step_fwd_bwd(t):
         out = B.forward(desc, t["x"], t["edge_index"], t["edge_vec"], t["w"], t["w_rad"],
                         t["b_rad"], ws=ws)
         g = B.backward(desc, t["x"], t["edge_index"], t["edge_vec"], t["w"], t["w_rad"],
                        t["b_rad"], t["grad_out"], ws=ws)
         return out, g
+
+    def step_force(t):
+        # energy = sum of l = 0 outputs (its cotangent is grad_out), forces from
+        # the edge-vector gradient, loss 1/2 |F - F_ref|^2 pulled back through
+        # the double backward to the weights.
+        out = B.forward(desc, t["x"], t["edge_index"], t["edge_vec"], t["w"], t["w_rad"],
+                        t["b_rad"], ws=ws)
+        gr = B.backward(desc, t["x"], t["edge_index"], t["edge_vec"], t["w"], t["w_rad"],
+                        t["b_rad"], t["grad_out"], need=["grad_edge_vec"],
+                        ws=ws)["grad_edge_vec"]
+        src, dst = t["edge_index"][0], t["edge_index"][1]
+        F = torch.zeros_like(t["f_ref"])
+        F.index_add_(0, src, -gr).index_add_(0, dst, gr)
+        dF = F - t["f_ref"]
+        gg_r = dF[dst] - dF[src]
+        g = B.double_backward(desc, t["x"], t["edge_index"], t["edge_vec"], t["w"], t["w_rad"],
+                              t["b_rad"], t["grad_out"], gg_edge_vec=gg_r,
+                              need=["d_w", "d_w_rad", "d_b_rad"], ws=ws)
+        return out, g
+
+    step = step_force if args.config == "force" else step_fwd_bwd
 
     for _ in range(max(args.warmup, 3)):
         step(d)
@@ -262,9 +300,9 @@ def run_ours(args, world, rank, local):
     fpe = mixing_flops_per_edge(p.lmax, p.mmax, p.c_in, p.c_out)
     n_gemm = sum(v[0] for v in prof.values())
     gemm_ms = sum(v[1] for v in prof.values())
-    alg_flops = 4.0 * fpe * E * args.steps  # fwd: 1 product; bwd: 3 (recompute, transpose, weights)
+    alg_flops = float(n_products) * fpe * E * args.steps
     achieved = alg_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
-    tf32_ratio = 1.1 / 2.25  # nominal dense TF32 / BF16 on B200
+    tf32_ratio = 1.0 if bf16 else 1.1 / 2.25  # nominal dense TF32 / BF16 on B200
     peak_tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * tf32_ratio
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "gemm_tc_esen_traffic.json")
@@ -276,8 +314,11 @@ def run_ours(args, world, rank, local):
             traffic = None
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                 "frac": (achieved / peak_tf) if achieved else None, "traffic": traffic,
-                "kernel": "k_gemm_tc (split-bf16 x3, f32 accumulate)",
-                "peak_basis": f"{src} bf16 sustained x nominal TF32/BF16 ratio 1.1/2.25",
+                "kernel": ("k_gemm_tc (bf16, f32 accumulate)" if bf16 else
+                           "k_gemm_tc (split-bf16 x3, f32 accumulate)"),
+                "peak_basis": (f"{src} bf16 sustained" if bf16 else
+                               f"{src} bf16 sustained x nominal TF32/BF16 ratio 1.1/2.25"),
+                "products_per_step": n_products,
                 "gemm_launches_per_step": n_gemm / args.steps,
                 "gemm_ms_per_step": gemm_ms / args.steps,
                 "step_roofline_frac": (alg_flops / (total_ms * 1e-3) / 1e12) / peak_tf}
@@ -296,6 +337,7 @@ def run_ours(args, world, rank, local):
         dd = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
         out, g = step(dd)
         res = [out] + [g[k] for k in sorted(g)]
+        res = [r for r in res if r is not None]
         if outs_host is None:
             outs_host = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in res]
         for hbuf, r in zip(outs_host, res):
@@ -309,7 +351,7 @@ def run_ours(args, world, rank, local):
 
     # ---- CPU oracle on a bounded sample (rank 0, one GPU only) ----
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "esen":
         n, ts, cores = oracle_sample_time(p, 2048, reps=1)
         cpu = {"value": n / ts[-1], "unit": "edges/s", "cores": cores, "kind": "oracle",
                "sample": f"first {n} edges (destination-major) of the same graph, float64 "
@@ -319,8 +361,8 @@ def run_ours(args, world, rank, local):
         line = {"metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f32", "data": "synthetic",
-                "config": {"workload": WORKLOAD, "edges": E, "nodes": p.n_nodes,
+                "dtype": "bf16" if bf16 else "f32", "data": "synthetic",
+                "config": {"workload": workload, "edges": E, "nodes": p.n_nodes,
                            "l2": "flushed between timed steps (256 MB write)",
                            "parallelism": f"replicas x{world}" if world > 1 else "single"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
@@ -335,6 +377,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", choices=sorted(CONFIGS), default="esen",
+                    help="workload (the headline line is esen; the others are for study)")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:
