@@ -79,16 +79,23 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Bounded wait on an mbarrier phase.  Gives up after `limit_ns` of wall time,
-// records SO2_ERR_TIMEOUT and returns false; the caller then unwinds.
+// records SO2_ERR_TIMEOUT, sets the CTA's abort flag (if given) and returns
+// false; a wait also gives up at once when another role of the CTA has set
+// the abort flag, so every role unwinds quickly.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, DevStatus *st,
+                                          volatile int *abort_flag = nullptr,
                                           uint64_t limit_ns = 2000000000ull) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) {
-      raise_error(st, SO2_ERR_TIMEOUT, 1);
-      return false;
+    if ((it & 255u) == 0) {
+      if (abort_flag && *abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        raise_error(st, SO2_ERR_TIMEOUT, 1);
+        if (abort_flag) *abort_flag = 1;
+        return false;
+      }
     }
   }
 }
@@ -170,11 +177,37 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
   return d;
 }
 
+// Same for a K-major tile with the 64-byte swizzle: rows of 32 bf16 (64 B),
+// 8-row atoms of 512 B stacked densely.  Base 512-byte aligned.
+__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(512u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(4u) << 61;  // 64-byte swizzle
+  return d;
+}
+
+// MN-major tile with the 128-byte swizzle, as a TMA box of {64 MN elements,
+// K rows} writes it: rows of 128 B (64 consecutive MN elements of one K
+// index), 8-row atoms of 1024 B along K (stride byte offset 1024), and
+// further 64-element MN chunks `lbo` bytes apart (leading byte offset).
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
 // Instruction descriptor: kind::f16 with bf16 A and B, f32 accumulator,
-// both operands K-major, shape M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
-         (static_cast<uint32_t>(M >> 4) << 24);
+// both operands K-major (or both MN-major), shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool mn_major = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (mn_major ? (1u << 15) | (1u << 16) : 0u) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 }  // namespace so2

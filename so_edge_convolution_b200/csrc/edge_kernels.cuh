@@ -92,49 +92,54 @@ __global__ void k_sort_segments(const int *__restrict__ offsets, int64_t N, int 
 struct EdgeRec {
   int eid, src, dst, key;  // key = the endpoint this order is sorted by
 };
+static_assert(sizeof(EdgeRec) == sizeof(int4), "EdgeRec is read as int4 by the fused epilogue");
 
 // Geometry record: d, r_hat[3], R[9] (row-major), 3 spare.
 constexpr int GEO = 16;
 
-// One thread per edge; the Wigner-D recursion runs in this thread's slice of
-// dynamic shared memory (blockDim.x * dsz floats) and is then copied out
-// with coalesced stores.
+// One warp per edge: lane 0 builds the record and frame, the warp runs the
+// Wigner-D recursion in its shared-memory slice (dsz floats) and copies it
+// out with coalesced stores.
 __global__ void k_edge_prep(Layout y, const int *__restrict__ perm, int64_t e0, int M,
                             const int64_t *__restrict__ ei, int64_t E, int64_t N, int key_row,
                             const float *__restrict__ edge_vec, EdgeRec *__restrict__ rec,
                             float *__restrict__ geo, float *__restrict__ D, DevStatus *st) {
-  extern __shared__ float sD[];
-  const int i0 = blockIdx.x * blockDim.x;
-  const int i = i0 + threadIdx.x;
-  float *mine = sD + threadIdx.x * y.dsz;
-  if (i < M) {
-    const int e = perm[e0 + i];
-    int64_t s = ei[e], d = ei[E + e];
-    if (s < 0 || s >= N) s = 0;  // already reported by the sort
-    if (d < 0 || d >= N) d = 0;
-    EdgeRec r;
-    r.eid = e;
-    r.src = static_cast<int>(s);
-    r.dst = static_cast<int>(d);
-    r.key = key_row == 0 ? r.src : r.dst;
-    rec[i] = r;
-    Frame f;
-    if (!make_frame(edge_vec[3 * (int64_t)e], edge_vec[3 * (int64_t)e + 1],
-                    edge_vec[3 * (int64_t)e + 2], f))
-      raise_error(st, SO2_ERR_DEGENERATE, e);
-    float *gr = geo + (int64_t)i * GEO;
-    gr[0] = f.d;
-    gr[1] = f.rh[0];
-    gr[2] = f.rh[1];
-    gr[3] = f.rh[2];
-    for (int k = 0; k < 9; ++k) gr[4 + k] = f.R[k];
-    wigner_blocks(f.R, y.L, mine);
+  extern __shared__ float sDall[];  // [warps][dsz + 16]
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  float *sD = sDall + (threadIdx.x >> 5) * (y.dsz + 16);
+  float *sR = sD + y.dsz;  // 9 floats of R
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
+    __syncwarp();
+    if (lane == 0) {
+      const int e = perm[e0 + i];
+      int64_t s = ei[e], d = ei[E + e];
+      if (s < 0 || s >= N) s = 0;  // already reported by the sort
+      if (d < 0 || d >= N) d = 0;
+      EdgeRec r;
+      r.eid = e;
+      r.src = static_cast<int>(s);
+      r.dst = static_cast<int>(d);
+      r.key = key_row == 0 ? r.src : r.dst;
+      rec[i] = r;
+      Frame f;
+      if (!make_frame(edge_vec[3 * (int64_t)e], edge_vec[3 * (int64_t)e + 1],
+                      edge_vec[3 * (int64_t)e + 2], f))
+        raise_error(st, SO2_ERR_DEGENERATE, e);
+      float *gr = geo + (int64_t)i * GEO;
+      gr[0] = f.d;
+      gr[1] = f.rh[0];
+      gr[2] = f.rh[1];
+      gr[3] = f.rh[2];
+      for (int k = 0; k < 9; ++k) {
+        gr[4 + k] = f.R[k];
+        sR[k] = f.R[k];
+      }
+    }
+    __syncwarp();
+    wigner_blocks_warp(sR, y.L, sD);
+    float *dst = D + (int64_t)i * y.dsz;
+    for (int k = lane; k < y.dsz; k += 32) dst[k] = sD[k];
   }
-  __syncthreads();
-  const int n_here = (M - i0) < (int)blockDim.x ? (M - i0) : (int)blockDim.x;
-  const int total = n_here * y.dsz;
-  float *dst = D + (int64_t)i0 * y.dsz;
-  for (int k = threadIdx.x; k < total; k += blockDim.x) dst[k] = sD[k];
 }
 
 __device__ __forceinline__ float rbf_val(float d, int k, const Layout &y, float cutoff) {
@@ -144,17 +149,28 @@ __device__ __forceinline__ float rbf_val(float d, int k, const Layout &y, float 
   return __expf(-0.5f * t * t);
 }
 
-// g[i][c'] = b[c'] + sum_k w_rad[k][c'] phi_k(d_i)
+// g[i][c'] = b[c'] + sum_k w_rad[k][c'] phi_k(d_i).  A block takes
+// GATE_EDGES edges: the basis values are computed once per edge into shared
+// memory, then threads over channels form the gates.
+constexpr int GATE_EDGES = 16;
 __global__ void k_edge_gate(Layout y, float cutoff, int M, const float *__restrict__ geo,
                             const float *__restrict__ w_rad, const float *__restrict__ b_rad,
                             float *__restrict__ gate) {
-  const int i = blockIdx.x;
-  if (i >= M) return;
-  const float d = geo[(int64_t)i * GEO];
+  extern __shared__ float phi[];  // [GATE_EDGES][nr]
+  const int i0 = blockIdx.x * GATE_EDGES;
+  const int n = (M - i0) < GATE_EDGES ? (M - i0) : GATE_EDGES;
+  for (int t = threadIdx.x; t < n * y.nr; t += blockDim.x) {
+    const int i = t / y.nr, k = t % y.nr;
+    phi[t] = rbf_val(geo[(int64_t)(i0 + i) * GEO], k, y, cutoff);
+  }
+  __syncthreads();
   for (int c = threadIdx.x; c < y.co; c += blockDim.x) {
-    float acc = b_rad[c];
-    for (int k = 0; k < y.nr; ++k) acc += w_rad[k * y.co + c] * rbf_val(d, k, y, cutoff);
-    gate[(int64_t)i * y.co + c] = acc;
+    const float b = b_rad[c];
+    for (int i = 0; i < n; ++i) {
+      float acc = b;
+      for (int k = 0; k < y.nr; ++k) acc += w_rad[k * y.co + c] * phi[i * y.nr + k];
+      gate[(int64_t)(i0 + i) * y.co + c] = acc;
+    }
   }
 }
 
@@ -190,6 +206,42 @@ __device__ __forceinline__ float2 coef2(const Coef &k, int64_t i, int C, int c) 
 // out[row (l,m)] = A * b[m] + B * (Omega b)[m],  b = D^l X[node][l, :],
 // Omega = w_x J_x + w_y J_y with (w_x, w_y) = omega[i][0..1].  With B absent
 // this is plain rotation on gather (A = 1) or gated rotation (A = g).
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void store_split4(__nv_bfloat16 *hi, __nv_bfloat16 *lo, float4 v) {
+  __nv_bfloat16 h[4], l[4];
+  split_bf16(v.x, h[0], l[0]);
+  split_bf16(v.y, h[1], l[1]);
+  split_bf16(v.z, h[2], l[2]);
+  split_bf16(v.w, h[3], l[3]);
+  uint2 uh, ul;
+  *reinterpret_cast<__nv_bfloat162 *>(&uh.x) = __halves2bfloat162(h[0], h[1]);
+  *reinterpret_cast<__nv_bfloat162 *>(&uh.y) = __halves2bfloat162(h[2], h[3]);
+  *reinterpret_cast<uint2 *>(hi) = uh;
+  if (lo) {
+    *reinterpret_cast<__nv_bfloat162 *>(&ul.x) = __halves2bfloat162(l[0], l[1]);
+    *reinterpret_cast<__nv_bfloat162 *>(&ul.y) = __halves2bfloat162(l[2], l[3]);
+    *reinterpret_cast<uint2 *>(lo) = ul;
+  }
+}
+__device__ __forceinline__ float4 coef4(const Coef &k, int64_t i, int C, int c) {
+  if (k.mode == 0) return make_float4(0.f, 0.f, 0.f, 0.f);
+  if (k.mode == 1) return make_float4(1.f, 1.f, 1.f, 1.f);
+  return load4(k.p + i * C + c);
+}
+
+// Copy one edge's Wigner-D blocks (dsz floats) into this warp's shared slice.
+__device__ __forceinline__ void stage_d(const float *De, int dsz, float *sD) {
+  const int lane = threadIdx.x & 31;
+  for (int k = lane; k < dsz; k += 32) sD[k] = De[k];
+  __syncwarp();
+}
+
 template <typename TX, int MM>
 __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec,
                                 const float *__restrict__ D, const TX *__restrict__ X, int side,
@@ -197,15 +249,18 @@ __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec
                                 __nv_bfloat16 *__restrict__ out_hi, __nv_bfloat16 *__restrict__ out_lo,
                                 int ld) {
   constexpr int W = MM + 1;
+  extern __shared__ float sDall[];  // [warps][dsz]
   const int C = side ? y.co : y.ci;
   const int *col_off = side ? y.kout_off : y.kin_off;
   const int *col_pad = side ? y.Kout_pad : y.Kin_pad;
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  float *sD = sDall + (threadIdx.x >> 5) * y.dsz;
   const bool wide = B.mode != 0;
   for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
     const EdgeRec r = rec[i];
     const int node = use_src ? r.src : r.dst;
-    const float *De = D + (int64_t)i * y.dsz;
+    __syncwarp();
+    stage_d(D + (int64_t)i * y.dsz, y.dsz, sD);
     const TX *Xn = X + (int64_t)node * y.S * C;
     __nv_bfloat16 *oh = out_hi + (int64_t)i * ld;
     __nv_bfloat16 *ol = out_lo ? out_lo + (int64_t)i * ld : nullptr;
@@ -214,23 +269,25 @@ __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec
       wx = omega[4 * (int64_t)i];
       wy = omega[4 * (int64_t)i + 1];
     }
-    for (int c = 2 * lane; c < C; c += 64) {
-      const float2 ca = coef2(A, i, C, c), cb = coef2(B, i, C, c);
+    for (int c = 4 * lane; c < C; c += 128) {
+      const float4 ca = coef4(A, i, C, c), cb = coef4(B, i, C, c);
       for (int l = 0; l <= y.L; ++l) {
-        float a0[2 * W + 1], a1[2 * W + 1];
+        float4 a[2 * W + 1];
 #pragma unroll
-        for (int k = 0; k < 2 * W + 1; ++k) a0[k] = a1[k] = 0.f;
-        const float *Dl = De + dblock_off(l);
+        for (int k = 0; k < 2 * W + 1; ++k) a[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *Dl = sD + dblock_off(l);
         const int w = 2 * l + 1;
         const int top = wide ? W : MM;
         for (int mp = -l; mp <= l; ++mp) {
-          const float2 xv = load2(Xn + (l * l + l + mp) * C + c);
+          const float4 xv = load4(Xn + (l * l + l + mp) * C + c);
 #pragma unroll
           for (int m = -W; m <= W; ++m) {
             if (m < -l || m > l || m < -top || m > top) continue;
             const float dv = Dl[(m + l) * w + mp + l];
-            a0[m + W] += dv * xv.x;
-            a1[m + W] += dv * xv.y;
+            a[m + W].x += dv * xv.x;
+            a[m + W].y += dv * xv.y;
+            a[m + W].z += dv * xv.z;
+            a[m + W].w += dv * xv.w;
           }
         }
 #pragma unroll
@@ -239,48 +296,28 @@ __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec
           int g, j;
           lm_group_row(y, l, m, g, j);
           const int col = col_off[g] + j * C + c;
-          float o0 = ca.x * a0[m + W], o1 = ca.y * a1[m + W];
+          float4 o = make_float4(ca.x * a[m + W].x, ca.y * a[m + W].y, ca.z * a[m + W].z,
+                                 ca.w * a[m + W].w);
           if (wide) {
-            float jx0, jy0, jx1, jy1;
-            gen_xy(l, m, [&](int q) { return a0[q + W]; }, jx0, jy0);
-            gen_xy(l, m, [&](int q) { return a1[q + W]; }, jx1, jy1);
-            o0 += cb.x * (wx * jx0 + wy * jy0);
-            o1 += cb.y * (wx * jx1 + wy * jy1);
+            float jx, jy;
+            gen_xy(l, m, [&](int q) { return a[q + W].x; }, jx, jy);
+            o.x += cb.x * (wx * jx + wy * jy);
+            gen_xy(l, m, [&](int q) { return a[q + W].y; }, jx, jy);
+            o.y += cb.y * (wx * jx + wy * jy);
+            gen_xy(l, m, [&](int q) { return a[q + W].z; }, jx, jy);
+            o.z += cb.z * (wx * jx + wy * jy);
+            gen_xy(l, m, [&](int q) { return a[q + W].w; }, jx, jy);
+            o.w += cb.w * (wx * jx + wy * jy);
           }
-          store_split2(oh + col, ol ? ol + col : nullptr, o0, o1);
+          store_split4(oh + col, ol ? ol + col : nullptr, o);
         }
       }
     }
     for (int g = 0; g < y.ng; ++g) {
       const int width = y.rows[g] * C;
-      for (int k = width + 2 * lane; k < col_pad[g]; k += 64)
-        store_split2(oh + col_off[g] + k, ol ? ol + col_off[g] + k : nullptr, 0.f, 0.f);
-    }
-  }
-}
-
-// [M x K] bf16 row-major -> [K x Mp] (row stride ld_out), columns in [M, Mp) zero.
-// 64 x 64 tiles through shared memory, 32-bit accesses.
-__global__ void k_transpose_bf16(const __nv_bfloat16 *__restrict__ in, int M, int K, int ld_in,
-                                 __nv_bfloat16 *__restrict__ out, int Mp, int ld_out) {
-  __shared__ __nv_bfloat16 tile[64][66];
-  const int k0 = blockIdx.x * 64, m0 = blockIdx.y * 64;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-  for (int r = ty; r < 64; r += 8) {
-    const int m = m0 + r, k = k0 + 2 * tx;
-    __nv_bfloat162 v = __floats2bfloat162_rn(0.f, 0.f);
-    if (m < M && k < K) v = *reinterpret_cast<const __nv_bfloat162 *>(in + (int64_t)m * ld_in + k);
-    tile[r][2 * tx] = v.x;
-    tile[r][2 * tx + 1] = v.y;
-  }
-  __syncthreads();
-  for (int r = ty; r < 64; r += 8) {
-    const int k = k0 + r, m = m0 + 2 * tx;
-    if (k < K && m < Mp) {
-      __nv_bfloat162 v;
-      v.x = tile[2 * tx][r];
-      v.y = tile[2 * tx + 1][r];
-      *reinterpret_cast<__nv_bfloat162 *>(out + (int64_t)k * ld_out + m) = v;
+      for (int k = width + 4 * lane; k < col_pad[g]; k += 128)
+        store_split4(oh + col_off[g] + k, ol ? ol + col_off[g] + k : nullptr,
+                     make_float4(0.f, 0.f, 0.f, 0.f));
     }
   }
 }
@@ -488,31 +525,36 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
                              const float *__restrict__ V, const float *__restrict__ Ga,
                              float *__restrict__ Gg, float *__restrict__ h) {
   constexpr int W = MM + 1;  // widest |m| needed by the generators
+  extern __shared__ float sDall[];  // [warps][dsz]
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  float *sD = sDall + (threadIdx.x >> 5) * y.dsz;
   for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
     const EdgeRec r = rec[i];
-    const float *De = D + (int64_t)i * y.dsz;
+    __syncwarp();
+    stage_d(D + (int64_t)i * y.dsz, y.dsz, sD);
     float hx = 0.f, hy = 0.f;
     // output side
     const float *Gn = G + (int64_t)r.dst * y.S * y.co;
     const float *Vi = V + (int64_t)i * y.KG;
-    for (int c = 2 * lane; c < y.co; c += 64) {
-      const float2 gv = load2(gate + (int64_t)i * y.co + c);
-      float gg0 = 0.f, gg1 = 0.f;
+    for (int c = 4 * lane; c < y.co; c += 128) {
+      const float4 gv = load4(gate + (int64_t)i * y.co + c);
+      float4 gg = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int l = 0; l <= y.L; ++l) {
-        float b0[2 * W + 1], b1[2 * W + 1];
+        float4 b[2 * W + 1];
 #pragma unroll
-        for (int k = 0; k < 2 * W + 1; ++k) b0[k] = b1[k] = 0.f;
-        const float *Dl = De + dblock_off(l);
+        for (int k = 0; k < 2 * W + 1; ++k) b[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *Dl = sD + dblock_off(l);
         const int w = 2 * l + 1;
         for (int mp = -l; mp <= l; ++mp) {
-          const float2 gx = load2(Gn + (l * l + l + mp) * y.co + c);
+          const float4 gx = load4(Gn + (l * l + l + mp) * y.co + c);
 #pragma unroll
           for (int m = -W; m <= W; ++m) {
             if (m < -l || m > l) continue;
             const float dv = Dl[(m + l) * w + mp + l];
-            b0[m + W] += dv * gx.x;
-            b1[m + W] += dv * gx.y;
+            b[m + W].x += dv * gx.x;
+            b[m + W].y += dv * gx.y;
+            b[m + W].z += dv * gx.z;
+            b[m + W].w += dv * gx.w;
           }
         }
 #pragma unroll
@@ -520,36 +562,48 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
           if (m < -l || m > l) continue;
           int g, j;
           lm_group_row(y, l, m, g, j);
-          const float2 v = load2(Vi + y.kout_off[g] + j * y.co + c);
-          gg0 += b0[m + W] * v.x;
-          gg1 += b1[m + W] * v.y;
-          float jx0, jy0, jx1, jy1;
-          gen_xy(l, m, [&](int q) { return b0[q + W]; }, jx0, jy0);
-          gen_xy(l, m, [&](int q) { return b1[q + W]; }, jx1, jy1);
-          hx += gv.x * v.x * jx0 + gv.y * v.y * jx1;
-          hy += gv.x * v.x * jy0 + gv.y * v.y * jy1;
+          const float4 v = load4(Vi + y.kout_off[g] + j * y.co + c);
+          gg.x += b[m + W].x * v.x;
+          gg.y += b[m + W].y * v.y;
+          gg.z += b[m + W].z * v.z;
+          gg.w += b[m + W].w * v.w;
+          float jx, jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].x; }, jx, jy);
+          hx += gv.x * v.x * jx;
+          hy += gv.x * v.x * jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].y; }, jx, jy);
+          hx += gv.y * v.y * jx;
+          hy += gv.y * v.y * jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].z; }, jx, jy);
+          hx += gv.z * v.z * jx;
+          hy += gv.z * v.z * jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].w; }, jx, jy);
+          hx += gv.w * v.w * jx;
+          hy += gv.w * v.w * jy;
         }
       }
-      *reinterpret_cast<float2 *>(Gg + (int64_t)i * y.co + c) = make_float2(gg0, gg1);
+      *reinterpret_cast<float4 *>(Gg + (int64_t)i * y.co + c) = gg;
     }
     // input side
     const TX *Xn = X + (int64_t)r.src * y.S * y.ci;
     const float *Gai = Ga + (int64_t)i * y.KA;
-    for (int c = 2 * lane; c < y.ci; c += 64) {
+    for (int c = 4 * lane; c < y.ci; c += 128) {
       for (int l = 0; l <= y.L; ++l) {
-        float b0[2 * W + 1], b1[2 * W + 1];
+        float4 b[2 * W + 1];
 #pragma unroll
-        for (int k = 0; k < 2 * W + 1; ++k) b0[k] = b1[k] = 0.f;
-        const float *Dl = De + dblock_off(l);
+        for (int k = 0; k < 2 * W + 1; ++k) b[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *Dl = sD + dblock_off(l);
         const int w = 2 * l + 1;
         for (int mp = -l; mp <= l; ++mp) {
-          const float2 xv = load2(Xn + (l * l + l + mp) * y.ci + c);
+          const float4 xv = load4(Xn + (l * l + l + mp) * y.ci + c);
 #pragma unroll
           for (int m = -W; m <= W; ++m) {
             if (m < -l || m > l) continue;
             const float dv = Dl[(m + l) * w + mp + l];
-            b0[m + W] += dv * xv.x;
-            b1[m + W] += dv * xv.y;
+            b[m + W].x += dv * xv.x;
+            b[m + W].y += dv * xv.y;
+            b[m + W].z += dv * xv.z;
+            b[m + W].w += dv * xv.w;
           }
         }
 #pragma unroll
@@ -557,12 +611,20 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
           if (m < -l || m > l) continue;
           int g, j;
           lm_group_row(y, l, m, g, j);
-          const float2 ga = load2(Gai + y.kin_off[g] + j * y.ci + c);
-          float jx0, jy0, jx1, jy1;
-          gen_xy(l, m, [&](int q) { return b0[q + W]; }, jx0, jy0);
-          gen_xy(l, m, [&](int q) { return b1[q + W]; }, jx1, jy1);
-          hx += ga.x * jx0 + ga.y * jx1;
-          hy += ga.x * jy0 + ga.y * jy1;
+          const float4 ga = load4(Gai + y.kin_off[g] + j * y.ci + c);
+          float jx, jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].x; }, jx, jy);
+          hx += ga.x * jx;
+          hy += ga.x * jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].y; }, jx, jy);
+          hx += ga.y * jx;
+          hy += ga.y * jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].z; }, jx, jy);
+          hx += ga.z * jx;
+          hy += ga.z * jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].w; }, jx, jy);
+          hx += ga.w * jx;
+          hy += ga.w * jy;
         }
       }
     }
@@ -655,18 +717,29 @@ __global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__rest
   }
 }
 
+// Stage 2: block = 32 consecutive (k, c') entries x 8 warps; each warp sums a
+// strided share of the blocks' partials, then the 8 shares are added in a
+// fixed order.
 __global__ void k_rad_reduce(Layout y, int nblk, const float *__restrict__ part,
                              float *__restrict__ grad_w_rad, float *__restrict__ grad_b) {
+  __shared__ float red[8][32];
   const int P = (y.nr + 1) * y.co;
-  const int pidx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (pidx >= P) return;
+  const int pidx = blockIdx.x * 32 + (threadIdx.x & 31);
+  const int w = threadIdx.x >> 5;
   float s = 0.f;
-  for (int b = 0; b < nblk; ++b) s += part[(int64_t)b * P + pidx];
-  const int k = pidx / y.co, c = pidx % y.co;
-  if (k < y.nr) {
-    if (grad_w_rad) grad_w_rad[k * y.co + c] += s;
-  } else if (grad_b) {
-    grad_b[c] += s;
+  if (pidx < P)
+    for (int b = w; b < nblk; b += 8) s += part[(int64_t)b * P + pidx];
+  red[w][threadIdx.x & 31] = s;
+  __syncthreads();
+  if (w == 0 && pidx < P) {
+    float t = 0.f;
+    for (int u = 0; u < 8; ++u) t += red[u][threadIdx.x];
+    const int k = pidx / y.co, c = pidx % y.co;
+    if (k < y.nr) {
+      if (grad_w_rad) grad_w_rad[k * y.co + c] += t;
+    } else if (grad_b) {
+      grad_b[c] += t;
+    }
   }
 }
 
@@ -784,20 +857,27 @@ __global__ void k_edge_terms2(Layout y, int M, const EdgeRec *__restrict__ rec,
   }
 }
 
-// Frames and full Wigner-D for inspection.
+// Frames and full Wigner-D for inspection (the same recursion the op uses).
 __global__ void k_frames(int lmax, int64_t E, const float *__restrict__ edge_vec, float *__restrict__ Rout,
                          float *__restrict__ Dout) {
-  const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (e >= E) return;
-  Frame f;
-  make_frame(edge_vec[3 * e], edge_vec[3 * e + 1], edge_vec[3 * e + 2], f);
-  if (Rout)
-    for (int k = 0; k < 9; ++k) Rout[9 * e + k] = f.R[k];
-  if (Dout) {
-    float Dl[dsize(LMAX_SUPPORTED)];
-    wigner_blocks(f.R, lmax, Dl);
-    const int n = dsize(lmax);
-    for (int k = 0; k < n; ++k) Dout[e * n + k] = Dl[k];
+  extern __shared__ float sDall[];  // [warps][dsz + 16]
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  const int dsz = dsize(lmax);
+  float *sD = sDall + (threadIdx.x >> 5) * (dsz + 16);
+  float *sR = sD + dsz;
+  for (int64_t e = blockIdx.x * (int64_t)wpb + (threadIdx.x >> 5); e < E; e += (int64_t)gridDim.x * wpb) {
+    __syncwarp();
+    if (lane == 0) {
+      Frame f;
+      make_frame(edge_vec[3 * e], edge_vec[3 * e + 1], edge_vec[3 * e + 2], f);
+      for (int k = 0; k < 9; ++k) sR[k] = f.R[k];
+    }
+    __syncwarp();
+    if (Rout && lane < 9) Rout[9 * e + lane] = sR[lane];
+    if (Dout) {
+      wigner_blocks_warp(sR, lmax, sD);
+      for (int k = lane; k < dsz; k += 32) Dout[e * dsz + k] = sD[k];
+    }
   }
 }
 

@@ -1,35 +1,60 @@
-// gemm_tc.cuh -- grouped tcgen05 GEMM for the per-m mixing.
+// gemm_tc.cuh -- grouped, persistent tcgen05 GEMM for the per-m mixing.
 //
 // C[M x N] (+)= A[M x K] * B[N x K]^T, A and B bf16 and K-major, f32
-// accumulation in tensor memory.  With `split`, A and B are each given as a
+// accumulation in tensor memory.  With SPLIT, A and B are each given as a
 // (hi, lo) pair of bf16 planes whose sum carries 16 significant bits, and the
-// product is hi*hi + hi*lo + lo*hi (the lo*lo term is below f32-level
-// accuracy for the tolerances the f32 path is held to).  This is how the f32
-// configurations reach ~1e-5 relative error on bf16 tensor cores.
+// product is hi*hi + hi*lo + lo*hi (the lo*lo term is below the f32 path's
+// tolerance).  This is how the f32 configurations reach ~1e-5 relative error
+// on bf16 tensor cores.
 //
-// Several independent problems (one per m, for the dense per-m
-// multiplications named in "TrimSO(2): Fast and Memory-Efficient Training of
-// Equivariant Interatomic Potentials", Abstract) run in one launch: each
-// group addresses its own rectangle of the same A and B tensors.
+// Several independent problems (one per m, the dense per-m multiplications
+// named in "TrimSO(2): Fast and Memory-Efficient Training of Equivariant
+// Interatomic Potentials", Abstract) share one launch: each group addresses
+// its own rectangle of the same A and B tensors.
+//
+// Structure: one CTA per SM loops over 128 x 256 output tiles.  Warp 0 issues
+// the TMA loads into a STAGES-deep shared-memory ring, warp 1 issues the MMAs
+// (one thread) into one of two TMEM accumulators (2 x 256 columns), warps 2..9
+// (two per TMEM lane quadrant) drain the other accumulator -- to global memory
+// and/or through the fused reduction epilogue -- so a tile's epilogue overlaps
+// the next tile's main loop.  Every wait is bounded (see mbar_wait).
 #pragma once
 
 #include "common.cuh"
 
+#ifndef SO2_EPI_WARPS
+#define SO2_EPI_WARPS 8
+#endif
+
 namespace so2 {
 
 constexpr int GEMM_BM = 128;
-constexpr int GEMM_BN = 128;
-constexpr int GEMM_BK = 64;
+constexpr int GEMM_BN = 256;
 constexpr int GEMM_MAX_GROUPS = 8;
-constexpr int GEMM_THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int GEMM_THREADS = 64 + 32 * SO2_EPI_WARPS;  // warp 0 TMA, warp 1 MMA, then epilogue
 
 struct GemmGroup {
-  int M, N, K;           // K is a multiple of GEMM_BK
+  int M, N, K;           // K is a multiple of the K block
   int a_row, a_col;      // origin of this group's A rectangle (rows, K cols)
   int b_row, b_col;      // origin of this group's B rectangle
   int tiles_n, tile_begin;
   long long c_off;       // element offset of C[0][0] for this group
   int ldc;               // row stride of C in elements
+  int mgroup;            // |m| of this group (fused reduction epilogue)
+  int tiles_mn;          // tiles per K split
+  int klen;              // K per split (multiple of the K block); ksplit = ceil(K / klen)
+};
+
+// Fused epilogue "inverse rotation on reduction": instead of (or besides)
+// storing a tile of the product, multiply it by the per-edge gate, rotate
+// each edge-frame row (l, m) back with D^l[m][:] and add it onto the node
+// key[edge] of out[node][(l, m')][c].  Requires rows = edges and C % 32 == 0.
+struct GemmScatter {
+  const int4 *rec;     // per edge: (eid, src, dst, key)
+  const float *gate;   // [rows][C] or null
+  const float *D;      // [rows][dsz] full Wigner-D blocks
+  float *out;          // [N][S][C]
+  int C, L, dsz;
 };
 
 struct GemmParams {
@@ -39,54 +64,203 @@ struct GemmParams {
   float *C;
   int beta;   // 0: C = AB^T, 1: C += AB^T
   int split;  // 1: hi/lo planes (3 products), 0: hi only
+  int store;  // write C
+  int scatter;  // fused reduction epilogue (GemmScatter)
+  GemmScatter sc;
   DevStatus *status;
 };
 
-template <int STAGES, bool SPLIT>
-struct GemmSmem {
-  static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
-  static constexpr int B_BYTES = GEMM_BN * GEMM_BK * 2;
-  static constexpr int PLANES = SPLIT ? 2 : 1;
-  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES) * PLANES;
-  static constexpr int TOTAL = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int EPI_WARPS = SO2_EPI_WARPS;  // 4 or 8: one or two per TMEM lane quadrant
+static_assert(EPI_WARPS == 4 || EPI_WARPS == 8, "epilogue warps per TMEM quadrant");
+constexpr int EPI_SMEM_PER_WARP = (32 * 33 + 32 * 16 + 32) * 4;  // multiple of 16 B
+constexpr int EPI_SMEM = EPI_WARPS * EPI_SMEM_PER_WARP;
+
+// Row j of an m-group (|m| = g) of an lmax-L layout -> (l, m); rows of group
+// g >= 1 are (l, +g) for l = g..L then (l, -g).
+__device__ __forceinline__ void gemm_row_lm(int L, int g, int j, int &l, int &m) {
+  if (g == 0) {
+    l = j;
+    m = 0;
+    return;
+  }
+  const int half = L + 1 - g;
+  if (j < half) {
+    l = g + j;
+    m = g;
+  } else {
+    l = g + (j - half);
+    m = -g;
+  }
+}
+
+// Per-warp scratch of the fused reduction epilogue.
+struct EpiScratch {
+  float *T;     // [32][33] product values, edge-major
+  float *Dw;    // [32][16] D^l[m][:] of the warp's edges for the current row
+  int *keys;    // [32] node of each edge (-1 past the end)
 };
 
-template <int STAGES, bool SPLIT>
+static_assert((32 * 33 * 4) % 16 == 0 && EPI_SMEM_PER_WARP % 16 == 0,
+              "float4 reads of the staged D rows need 16-byte alignment");
+__device__ __forceinline__ EpiScratch epi_scratch(float *base) {
+  EpiScratch e;
+  e.T = base;
+  e.Dw = base + 32 * 33;  // 32 * 33 floats = 4224 B: rows of 16 stay 16-byte aligned
+  e.keys = reinterpret_cast<int *>(base + 32 * 33 + 32 * 16);
+  return e;
+}
+
+// Stage D^l[m][:] for the warp's 32 edges (rows row_base..) into Dw.
+__device__ __forceinline__ void epi_stage_d(const GemmParams &p, const GemmGroup &G, int row_base,
+                                            int l, int m, const EpiScratch &x) {
+  const int lane = threadIdx.x & 31;
+  const int w = 2 * l + 1;
+  const int doff = l * (4 * l * l - 1) / 3 + (m + l) * w;
+  for (int idx = lane; idx < 32 * w; idx += 32) {
+    const int el = idx / w, k = idx % w;
+    const int ee = row_base + el;
+    x.Dw[el * 16 + k] = (ee < G.M) ? p.sc.D[(int64_t)ee * p.sc.dsz + doff + k] : 0.f;
+  }
+}
+
+// The sums of one warp-chunk for a fixed width W = 2l + 1 (see below).
+template <int W>
+__device__ __forceinline__ void epi_rotate_reduce(const GemmScatter &S, int row_base, int l, int c,
+                                                  const EpiScratch &x, const float (&g)[32]) {
+  const int lane = threadIdx.x & 31;
+  const int S_ = (S.L + 1) * (S.L + 1);
+  float acc[W];
+#pragma unroll
+  for (int k = 0; k < W; ++k) acc[k] = 0.f;
+  int cur = x.keys[0];
+#pragma unroll
+  for (int el = 0; el < 32; ++el) {
+    const int k_e = x.keys[el];
+    if (k_e != cur) {
+      if (cur >= 0) {
+        float *o = S.out + ((int64_t)cur * S_ + l * l) * S.C + c;
+#pragma unroll
+        for (int k = 0; k < W; ++k) atomicAdd(o + k * S.C, acc[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < W; ++k) acc[k] = 0.f;
+      cur = k_e;
+    }
+    const float v = x.T[el * 33 + lane] * g[el];
+    const float4 *d4 = reinterpret_cast<const float4 *>(x.Dw + el * 16);
+#pragma unroll
+    for (int k4 = 0; k4 < (W + 3) / 4; ++k4) {
+      const float4 d = d4[k4];
+      if (4 * k4 + 0 < W) acc[4 * k4 + 0] += d.x * v;
+      if (4 * k4 + 1 < W) acc[4 * k4 + 1] += d.y * v;
+      if (4 * k4 + 2 < W) acc[4 * k4 + 2] += d.z * v;
+      if (4 * k4 + 3 < W) acc[4 * k4 + 3] += d.w * v;
+    }
+  }
+  if (cur >= 0) {
+    float *o = S.out + ((int64_t)cur * S_ + l * l) * S.C + c;
+#pragma unroll
+    for (int k = 0; k < W; ++k) atomicAdd(o + k * S.C, acc[k]);
+  }
+}
+
+// One warp, one 32-column chunk (channels c0.. of edge-frame row (l, m)) of
+// its 32 edges: adds sum_e D_e^l[m][m'] g_e[c] v_e[c] onto
+// out[key_e][(l, m')][c], one coalesced atomic per (node run, m', c).
+// keys and Dw must be staged; r holds one edge's 32 values per lane.
+__device__ __forceinline__ void epi_scatter_chunk(const GemmParams &p, int row_base, int l, int c0,
+                                                  const uint32_t (&r)[32], const EpiScratch &x) {
+  const GemmScatter &S = p.sc;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) x.T[lane * 33 + k] = __uint_as_float(r[k]);
+  __syncwarp();
+  // lane = channel from here on
+  const int c = c0 + lane;
+  float g[32];
+#pragma unroll
+  for (int el = 0; el < 32; ++el)
+    g[el] = (S.gate && x.keys[el] >= 0) ? S.gate[(int64_t)(row_base + el) * S.C + c] : 1.f;
+  switch (2 * l + 1) {
+    case 1: epi_rotate_reduce<1>(S, row_base, l, c, x, g); break;
+    case 3: epi_rotate_reduce<3>(S, row_base, l, c, x, g); break;
+    case 5: epi_rotate_reduce<5>(S, row_base, l, c, x, g); break;
+    case 7: epi_rotate_reduce<7>(S, row_base, l, c, x, g); break;
+    case 9: epi_rotate_reduce<9>(S, row_base, l, c, x, g); break;
+    case 11: epi_rotate_reduce<11>(S, row_base, l, c, x, g); break;
+    default: epi_rotate_reduce<13>(S, row_base, l, c, x, g); break;
+  }
+  __syncwarp();
+}
+
+// BK = 32 uses the 64-byte swizzle (4 stages of 48 KB with hi/lo planes),
+// BK = 64 the 128-byte swizzle.
+template <int BK, int STAGES, bool SPLIT, bool SCATTER>
+struct GemmCfg {
+  static constexpr int A_BYTES = GEMM_BM * BK * 2;
+  static constexpr int B_BYTES = GEMM_BN * BK * 2;
+  static constexpr int PLANES = SPLIT ? 2 : 1;
+  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES) * PLANES;
+  static constexpr int SMEM =
+      STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + (SCATTER ? EPI_SMEM : 0);
+  static constexpr int TMEM_COLS = 2 * GEMM_BN;
+  static_assert(SMEM <= 232448, "shared memory per CTA");
+};
+
+__device__ __forceinline__ uint64_t sdesc_k(uint32_t saddr, int bk) {
+  return bk == 32 ? sdesc_k_sw64(saddr) : sdesc_k_sw128(saddr);
+}
+
+// Tile -> group, output origin and K range [k0, k0 + klen_t).  K splits are
+// outermost inside a group so that concurrent tiles share operand rows in L2.
+__device__ __forceinline__ void tile_coords(const GemmParams &p, int tile, int &gi, int &m0,
+                                            int &n0, int &k0, int &kl) {
+  gi = 0;
+  while (gi + 1 < p.n_groups && tile >= p.g[gi + 1].tile_begin) ++gi;
+  const GemmGroup &G = p.g[gi];
+  const int local = tile - G.tile_begin;
+  const int ks = local / G.tiles_mn, mn = local % G.tiles_mn;
+  m0 = (mn / G.tiles_n) * GEMM_BM;
+  n0 = (mn % G.tiles_n) * GEMM_BN;
+  k0 = ks * G.klen;
+  kl = (G.K - k0) < G.klen ? (G.K - k0) : G.klen;
+}
+
+template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool MN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
               const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
               const __grid_constant__ GemmParams p) {
-  using L = GemmSmem<STAGES, SPLIT>;
+  using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER>;
+  static_assert(!MN || BK % 16 == 0, "MN-major K block");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * L::STAGE_BYTES);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * Cfg::STAGE_BYTES);
   uint64_t *empty = full + STAGES;
-  uint64_t *tmem_full = empty + STAGES;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tmem_full + 1);
+  uint64_t *tfull = empty + STAGES;  // [2]
+  uint64_t *tempty = tfull + 2;      // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *epi_smem = reinterpret_cast<float *>(smem + STAGES * Cfg::STAGE_BYTES + 256);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // which group / tile
-  int gi = 0;
-  while (gi + 1 < p.n_groups && static_cast<int>(blockIdx.x) >= p.g[gi + 1].tile_begin) ++gi;
-  const GemmGroup &G = p.g[gi];
-  const int local = blockIdx.x - G.tile_begin;
-  const int m0 = (local / G.tiles_n) * GEMM_BM;
-  const int n0 = (local % G.tiles_n) * GEMM_BN;
-  const int nk = G.K / GEMM_BK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(tmem_full, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], EPI_WARPS);  // one arrive per epilogue warp
+    }
+    *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, GEMM_BN);
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -96,71 +270,144 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (!mbar_wait(&empty[s], ph ^ 1, p.status)) break;
-      uint8_t *st = smem + s * L::STAGE_BYTES;
-      mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
-      const int kc = kb * GEMM_BK;
-      tma_load_2d(st, &tA_hi, &full[s], G.a_col + kc, G.a_row + m0);
-      tma_load_2d(st + L::A_BYTES, &tB_hi, &full[s], G.b_col + kc, G.b_row + n0);
-      if (SPLIT) {
-        tma_load_2d(st + L::A_BYTES + L::B_BYTES, &tA_lo, &full[s], G.a_col + kc, G.a_row + m0);
-        tma_load_2d(st + 2 * L::A_BYTES + L::B_BYTES, &tB_lo, &full[s], G.b_col + kc,
-                    G.b_row + n0);
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+      int gi, m0, n0, k0, kl;
+      tile_coords(p, tile, gi, m0, n0, k0, kl);
+      const GemmGroup &G = p.g[gi];
+      const int nk = kl / BK;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t *st = smem + s * Cfg::STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[s], Cfg::STAGE_BYTES);
+        const int kc = k0 + kb * BK;
+        if (!MN) {
+          tma_load_2d(st, &tA_hi, &full[s], G.a_col + kc, G.a_row + m0);
+          tma_load_2d(st + Cfg::A_BYTES, &tB_hi, &full[s], G.b_col + kc, G.b_row + n0);
+          if (SPLIT) {
+            tma_load_2d(st + Cfg::A_BYTES + Cfg::B_BYTES, &tA_lo, &full[s], G.a_col + kc,
+                        G.a_row + m0);
+            tma_load_2d(st + 2 * Cfg::A_BYTES + Cfg::B_BYTES, &tB_lo, &full[s], G.b_col + kc,
+                        G.b_row + n0);
+          }
+        } else {
+          // MN-major operands: the inner TMA coordinate is the M / N index, the
+          // outer one the K index; one box per 64 M / N elements
+          constexpr int BOX = 64 * BK * 2;
+          for (int h = 0; h < GEMM_BM / 64; ++h)
+            tma_load_2d(st + h * BOX, &tA_hi, &full[s], G.a_row + m0 + 64 * h, G.a_col + kc);
+          for (int h = 0; h < GEMM_BN / 64; ++h)
+            tma_load_2d(st + Cfg::A_BYTES + h * BOX, &tB_hi, &full[s], G.b_row + n0 + 64 * h,
+                        G.b_col + kc);
+          if (SPLIT) {
+            for (int h = 0; h < GEMM_BM / 64; ++h)
+              tma_load_2d(st + Cfg::A_BYTES + Cfg::B_BYTES + h * BOX, &tA_lo, &full[s],
+                          G.a_row + m0 + 64 * h, G.a_col + kc);
+            for (int h = 0; h < GEMM_BN / 64; ++h)
+              tma_load_2d(st + 2 * Cfg::A_BYTES + Cfg::B_BYTES + h * BOX, &tB_lo, &full[s],
+                          G.b_row + n0 + 64 * h, G.b_col + kc);
+          }
+        }
       }
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
-    constexpr uint32_t idesc = idesc_bf16_f32(GEMM_BM, GEMM_BN);
+    constexpr uint32_t idesc = idesc_bf16_f32(GEMM_BM, GEMM_BN, MN);
+    constexpr uint32_t LBO = 64 * BK * 2;  // MN-major: bytes between 64-element MN chunks
+    int it = 0, tcount = 0;
     bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (!mbar_wait(&full[s], ph, p.status)) {
-        ok = false;
-        break;
-      }
+    for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tcount) {
+      int gi, m0, n0, k0, kl;
+      tile_coords(p, tile, gi, m0, n0, k0, kl);
+      const int nk = kl / BK;
+      const int acc = tcount & 1;
+      const uint32_t aph = (tcount >> 1) & 1;
+      if (!mbar_wait(&tempty[acc], aph ^ 1, p.status, abort_flag)) break;
       tc_fence_after();
-      const uint32_t base = smem_u32(smem + s * L::STAGE_BYTES);
-      const uint64_t a_hi = sdesc_k_sw128(base);
-      const uint64_t b_hi = sdesc_k_sw128(base + L::A_BYTES);
-      const uint64_t a_lo = sdesc_k_sw128(base + L::A_BYTES + L::B_BYTES);
-      const uint64_t b_lo = sdesc_k_sw128(base + 2 * L::A_BYTES + L::B_BYTES);
-#pragma unroll
-      for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-        const uint64_t step = static_cast<uint64_t>(kk * 2);  // 32 bytes, in 16-byte units
-        umma_bf16(tmem, a_hi + step, b_hi + step, idesc, (kb | kk) != 0);
-        if (SPLIT) {
-          umma_bf16(tmem, a_hi + step, b_lo + step, idesc, 1);
-          umma_bf16(tmem, a_lo + step, b_hi + step, idesc, 1);
+      const uint32_t d_tmem = tmem + acc * GEMM_BN;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(&full[s], ph, p.status, abort_flag)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        const uint32_t base = smem_u32(smem + s * Cfg::STAGE_BYTES);
+        const uint32_t oa = base, ob = base + Cfg::A_BYTES;
+        const uint32_t oal = base + Cfg::A_BYTES + Cfg::B_BYTES;
+        const uint32_t obl = base + 2 * Cfg::A_BYTES + Cfg::B_BYTES;
+        const uint64_t a_hi = MN ? sdesc_mn_sw128(oa, LBO) : sdesc_k(oa, BK);
+        const uint64_t b_hi = MN ? sdesc_mn_sw128(ob, LBO) : sdesc_k(ob, BK);
+        const uint64_t a_lo = MN ? sdesc_mn_sw128(oal, LBO) : sdesc_k(oal, BK);
+        const uint64_t b_lo = MN ? sdesc_mn_sw128(obl, LBO) : sdesc_k(obl, BK);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          // next 16 K: 32 bytes along a K-major row, or two 1024-byte atoms of
+          // an MN-major tile (in 16-byte units)
+          const uint64_t step = static_cast<uint64_t>(MN ? kk * 128 : kk * 2);
+          umma_bf16(d_tmem, a_hi + step, b_hi + step, idesc, (kb | kk) != 0);
+          if (SPLIT) {
+            umma_bf16(d_tmem, a_hi + step, b_lo + step, idesc, 1);
+            umma_bf16(d_tmem, a_lo + step, b_hi + step, idesc, 1);
+          }
+        }
+        umma_commit(&empty[s]);
       }
-      umma_commit(&empty[s]);
+      if (ok) umma_commit(&tfull[acc]);
     }
-    if (ok) umma_commit(tmem_full);
   } else if (warp >= 2) {
-    // ---------------- epilogue: TMEM -> registers -> C ----------------
-    const int q = warp & 3;  // TMEM lane quadrant this warp may read
-    const int row = m0 + q * 32 + lane;
-    bool ready = (nk > 0) ? mbar_wait(tmem_full, 0, p.status) : true;
-    tc_fence_after();
-    if (ready) {
+    // ---------------- epilogue: TMEM -> registers -> C and/or node sums ----------------
+    const int q = warp & 3;           // TMEM lane quadrant this warp may read
+    const int half = (warp - 2) >> 2;  // which half of the tile's column chunks (8 warps)
+    const EpiScratch xs = epi_scratch(epi_smem + (warp - 2) * (EPI_SMEM_PER_WARP / 4));
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tcount) {
+      int gi, m0, n0, k0, kl;
+      tile_coords(p, tile, gi, m0, n0, k0, kl);
+      const GemmGroup &G = p.g[gi];
+      const bool atomic_c = G.klen < G.K;  // split K: partial sums meet in C
+      const int acc = tcount & 1;
+      const uint32_t aph = (tcount >> 1) & 1;
+      const int row_base = m0 + q * 32;
+      if (SCATTER && p.scatter) {
+        const int e = row_base + lane;
+        xs.keys[lane] = (e < G.M) ? p.sc.rec[e].w : -1;
+      }
+      if (!mbar_wait(&tfull[acc], aph, p.status, abort_flag)) break;
+      tc_fence_after();
+      const int row = row_base + lane;
       float *Cg = p.C + G.c_off;
-      for (int cc = 0; cc < GEMM_BN / 32; ++cc) {
-        uint32_t r[32];
-        if (nk > 0) {
-          tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + cc * 32, r);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = 0u;
-        }
+      int staged = -1;  // edge-frame row whose D rows are in Dw
+      for (int cc = half; cc < GEMM_BN / 32; cc += EPI_WARPS / 4) {
         const int col0 = n0 + cc * 32;
-        if (row < G.M && col0 < G.N) {
+        if (col0 >= G.N) break;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * GEMM_BN + cc * 32, r);
+        if (SCATTER && p.scatter) {
+          const int j = col0 / p.sc.C, c0 = col0 % p.sc.C;
+          int l, m;
+          gemm_row_lm(p.sc.L, G.mgroup, j, l, m);
+          if (j != staged) {
+            __syncwarp();
+            epi_stage_d(p, G, row_base, l, m, xs);
+            staged = j;
+          }
+          __syncwarp();
+          epi_scatter_chunk(p, row_base, l, c0, r, xs);
+        }
+        if (p.store && row < G.M) {
           float *crow = Cg + static_cast<long long>(row) * G.ldc + col0;
-          const bool full_vec = (col0 + 32 <= G.N) && ((reinterpret_cast<uintptr_t>(crow) & 15) == 0);
-          if (full_vec) {
+          const bool vec = (col0 + 32 <= G.N) && ((reinterpret_cast<uintptr_t>(crow) & 15) == 0);
+          if (atomic_c) {
+            for (int j = 0; j < 32 && col0 + j < G.N; ++j) atomicAdd(crow + j, __uint_as_float(r[j]));
+          } else if (vec) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
               float4 v = make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
@@ -183,13 +430,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
     }
-    tc_fence_before();
   }
+  tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, GEMM_BN);
+    tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
 }
 

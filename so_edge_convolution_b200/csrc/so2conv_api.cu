@@ -12,6 +12,10 @@
 
 using namespace so2;
 
+#ifndef SO2_SCATTER_STAGES
+#define SO2_SCATTER_STAGES 3
+#endif
+
 namespace {
 
 constexpr int CHUNK_MAX = 32768;  // edges per chunk of per-edge intermediates
@@ -39,20 +43,50 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-// bf16 matrix [rows x cols] with row stride ld (elements); box 64 x box_rows,
-// 128-byte swizzle, zero fill outside.
+// bf16 matrix [rows x cols] with row stride ld (elements); box bk x box_rows
+// with the swizzle that matches bk (32 -> 64 B rows, 64 -> 128 B rows), zero
+// fill outside the matrix.
 bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld,
-              int box_rows) {
+              int box_rows, int bk) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
-  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(bk), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             bk == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The same bf16 matrix read MN-major: box of 64 columns (inner, 128 B) by bk
+// rows, 128-byte swizzle.
+bool make_map_mn(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld,
+                 int bk) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bk)};
   cuuint32_t estr[2] = {1u, 1u};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// K block of the product kernel: 32 (64-byte swizzle) for the split path so
+// that four stages of hi/lo planes fit in shared memory, 64 otherwise.
+inline int gemm_bk(bool split) { return split ? 32 : 64; }
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+    return n;
+  return 148;
 }
 
 // --------------------------------------------------------------------------
@@ -61,13 +95,13 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int6
 struct Plan {
   Layout y;
   int64_t N = 0, E = 0;
-  int chunk = 0, chunkp = 0;
+  int chunk = 0;
   bool split = true, xbf16 = false;
   size_t total = 0;
   // byte offsets
   int na = 1, ngv = 1;  // row-stacked operand sets (double backward uses 3 and 2)
   size_t status, counts, cursor, offsets, perm, rec, geo, D, gate, wst_hi, wst_lo, wtr_hi, wtr_lo,
-      a_hi, a_lo, V, gv_hi, gv_lo, aT_hi, aT_lo, gvT_hi, gvT_lo, Ga, Gg, h, dws, radp, omega,
+      a_hi, a_lo, V, gv_hi, gv_lo, Ga, Gg, h, dws, radp, omega,
       dgate, tA, tB;
 };
 
@@ -100,7 +134,6 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
   const int64_t cap = which == SO2_WS_DOUBLE_BACKWARD ? CHUNK_MAX / 2 : CHUNK_MAX;
   const int64_t ch = E < cap ? E : cap;
   p.chunk = static_cast<int>(round_up(static_cast<int>(ch > 0 ? ch : 1), 128));
-  p.chunkp = p.chunk;  // multiple of 64 already
   const Layout &y = p.y;
   const bool bwd = which >= SO2_WS_BACKWARD;
   const bool dbl = which == SO2_WS_DOUBLE_BACKWARD;
@@ -128,10 +161,6 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
   if (bwd) {
     p.gv_hi = take(c, 2ull * ngv * p.chunk * y.KG);
     p.gv_lo = take(c, 2ull * ngv * p.chunk * y.KG * lo);
-    p.aT_hi = take(c, 2ull * y.KA * na * p.chunkp);
-    p.aT_lo = take(c, 2ull * y.KA * na * p.chunkp * lo);
-    p.gvT_hi = take(c, 2ull * y.KG * ngv * p.chunkp);
-    p.gvT_lo = take(c, 2ull * y.KG * ngv * p.chunkp * lo);
     p.Ga = take(c, 4ull * ngv * p.chunk * y.KA);
     p.Gg = take(c, 4ull * p.chunk * y.co);
     p.h = take(c, 8ull * p.chunk);
@@ -246,8 +275,10 @@ int warp_grid(int M, int warps_per_block) {
 // --------------------------------------------------------------------------
 struct GemmLauncher {
   GemmParams p{};
+  // ksplit > 1 splits K into that many ranges (multiples of 64) whose
+  // partial products are added into C atomically (C must hold the base).
   void add(int M, int N, int K, int a_row, int a_col, int b_row, int b_col, long long c_off,
-           int ldc) {
+           int ldc, int ksplit = 1) {
     if (M <= 0 || N <= 0) return;
     GemmGroup &g = p.g[p.n_groups++];
     g.M = M;
@@ -259,35 +290,48 @@ struct GemmLauncher {
     g.b_col = b_col;
     g.c_off = c_off;
     g.ldc = ldc;
+    g.mgroup = p.n_groups - 1;
     g.tiles_n = (N + GEMM_BN - 1) / GEMM_BN;
+    g.tiles_mn = ((M + GEMM_BM - 1) / GEMM_BM) * g.tiles_n;
+    if (ksplit < 1) ksplit = 1;
+    g.klen = round_up((K + ksplit - 1) / ksplit, 64);
+    if (g.klen > K) g.klen = K;
+    const int nsplit = (K + g.klen - 1) / g.klen;
     g.tile_begin = p.total_tiles;
-    p.total_tiles += ((M + GEMM_BM - 1) / GEMM_BM) * g.tiles_n;
+    p.total_tiles += g.tiles_mn * nsplit;
   }
 };
 
-template <int STAGES, bool SPLIT>
+template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool MN>
 cudaError_t launch_gemm_t(const CUtensorMap &a_hi, const CUtensorMap &a_lo, const CUtensorMap &b_hi,
                           const CUtensorMap &b_lo, const GemmParams &p, cudaStream_t s) {
-  using L = GemmSmem<STAGES, SPLIT>;
+  using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER>;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<STAGES, SPLIT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BK, STAGES, SPLIT, SCATTER, MN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  k_gemm_tc<STAGES, SPLIT><<<p.total_tiles, GEMM_THREADS, L::TOTAL, s>>>(a_hi, a_lo, b_hi, b_lo, p);
+  static int sms = num_sms();
+  const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+  k_gemm_tc<BK, STAGES, SPLIT, SCATTER, MN><<<grid, GEMM_THREADS, Cfg::SMEM, s>>>(a_hi, a_lo,
+                                                                               b_hi, b_lo, p);
   return cudaPeekAtLastError();
 }
 
 cudaError_t launch_gemm(int kind, bool split, const CUtensorMap &a_hi, const CUtensorMap &a_lo,
                         const CUtensorMap &b_hi, const CUtensorMap &b_lo, GemmParams p,
-                        float *C, int beta, DevStatus *st, cudaStream_t s) {
+                        float *C, int beta, DevStatus *st, cudaStream_t s,
+                        const GemmScatter *sc = nullptr, bool store = true, bool mn = false) {
   if (p.total_tiles == 0) return cudaSuccess;
   p.C = C;
   p.beta = beta;
   p.split = split ? 1 : 0;
   p.status = st;
+  p.store = store ? 1 : 0;
+  p.scatter = sc ? 1 : 0;
+  if (sc) p.sc = *sc;
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   if (g_prof.on) {
     e0 = prof_event(kind);
@@ -295,8 +339,18 @@ cudaError_t launch_gemm(int kind, bool split, const CUtensorMap &a_hi, const CUt
     if (e0) cudaEventRecord(e0, s);
   }
   ++g_launches;
-  cudaError_t r = split ? launch_gemm_t<3, true>(a_hi, a_lo, b_hi, b_lo, p, s)
-                        : launch_gemm_t<6, false>(a_hi, a_lo, b_hi, b_lo, p, s);
+  // the fused reduction epilogue's scratch (6.4 KB per epilogue warp) can cost
+  // a pipeline stage
+  cudaError_t r;
+  if (sc)
+    r = split ? launch_gemm_t<32, SO2_SCATTER_STAGES, true, true, false>(a_hi, a_lo, b_hi, b_lo, p, s)
+              : launch_gemm_t<64, SO2_SCATTER_STAGES, false, true, false>(a_hi, a_lo, b_hi, b_lo, p, s);
+  else if (mn)
+    r = split ? launch_gemm_t<32, 4, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
+              : launch_gemm_t<64, 4, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
+  else
+    r = split ? launch_gemm_t<32, 4, true, false, false>(a_hi, a_lo, b_hi, b_lo, p, s)
+              : launch_gemm_t<64, 4, false, false, false>(a_hi, a_lo, b_hi, b_lo, p, s);
   if (e1) cudaEventRecord(e1, s);
   return r;
 }
@@ -310,8 +364,8 @@ struct Ctx {
   void *ws;
   cudaStream_t s;
   DevStatus *st;
-  CUtensorMap m_a_hi, m_a_lo, m_v_hi, m_v_lo, m_wst_hi, m_wst_lo, m_wtr_hi, m_wtr_lo, m_aT_hi,
-      m_aT_lo, m_gvT_hi, m_gvT_lo;
+  CUtensorMap m_a_hi, m_a_lo, m_v_hi, m_v_lo, m_wst_hi, m_wst_lo, m_wtr_hi, m_wtr_lo;
+  CUtensorMap m_amn_hi, m_amn_lo, m_vmn_hi, m_vmn_lo;  // the same planes, MN-major boxes
 };
 
 so2_status common_checks(const so2conv_desc *d, int64_t N, int64_t E, const void *x,
@@ -333,22 +387,22 @@ so2_status build_maps(Ctx &c, bool bwd) {
   const Plan &P = c.P;
   const Layout &y = P.y;
   void *ws = c.ws;
+  const int bk = gemm_bk(P.split);
   bool ok = true;
   const int64_t ra = (int64_t)P.na * P.chunk, rg = (int64_t)P.ngv * P.chunk;
-  const int64_t ca = (int64_t)P.na * P.chunkp, cg = (int64_t)P.ngv * P.chunkp;
-  ok &= make_map(&c.m_a_hi, at<void>(ws, P.a_hi), ra, y.KA, y.KA, GEMM_BM);
-  ok &= make_map(&c.m_a_lo, at<void>(ws, P.split ? P.a_lo : P.a_hi), ra, y.KA, y.KA, GEMM_BM);
-  ok &= make_map(&c.m_wst_hi, at<void>(ws, P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN);
-  ok &= make_map(&c.m_wst_lo, at<void>(ws, P.split ? P.wst_lo : P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN);
+  ok &= make_map(&c.m_a_hi, at<void>(ws, P.a_hi), ra, y.KA, y.KA, GEMM_BM, bk);
+  ok &= make_map(&c.m_a_lo, at<void>(ws, P.split ? P.a_lo : P.a_hi), ra, y.KA, y.KA, GEMM_BM, bk);
+  ok &= make_map(&c.m_wst_hi, at<void>(ws, P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN, bk);
+  ok &= make_map(&c.m_wst_lo, at<void>(ws, P.split ? P.wst_lo : P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN, bk);
   if (bwd) {
-    ok &= make_map(&c.m_v_hi, at<void>(ws, P.gv_hi), rg, y.KG, y.KG, GEMM_BM);
-    ok &= make_map(&c.m_v_lo, at<void>(ws, P.split ? P.gv_lo : P.gv_hi), rg, y.KG, y.KG, GEMM_BM);
-    ok &= make_map(&c.m_wtr_hi, at<void>(ws, P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN);
-    ok &= make_map(&c.m_wtr_lo, at<void>(ws, P.split ? P.wtr_lo : P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN);
-    ok &= make_map(&c.m_aT_hi, at<void>(ws, P.aT_hi), y.KA, ca, ca, GEMM_BN);
-    ok &= make_map(&c.m_aT_lo, at<void>(ws, P.split ? P.aT_lo : P.aT_hi), y.KA, ca, ca, GEMM_BN);
-    ok &= make_map(&c.m_gvT_hi, at<void>(ws, P.gvT_hi), y.KG, cg, cg, GEMM_BM);
-    ok &= make_map(&c.m_gvT_lo, at<void>(ws, P.split ? P.gvT_lo : P.gvT_hi), y.KG, cg, cg, GEMM_BM);
+    ok &= make_map(&c.m_v_hi, at<void>(ws, P.gv_hi), rg, y.KG, y.KG, GEMM_BM, bk);
+    ok &= make_map(&c.m_v_lo, at<void>(ws, P.split ? P.gv_lo : P.gv_hi), rg, y.KG, y.KG, GEMM_BM, bk);
+    ok &= make_map(&c.m_wtr_hi, at<void>(ws, P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN, bk);
+    ok &= make_map(&c.m_wtr_lo, at<void>(ws, P.split ? P.wtr_lo : P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN, bk);
+    ok &= make_map_mn(&c.m_amn_hi, at<void>(ws, P.a_hi), ra, y.KA, y.KA, bk);
+    ok &= make_map_mn(&c.m_amn_lo, at<void>(ws, P.split ? P.a_lo : P.a_hi), ra, y.KA, y.KA, bk);
+    ok &= make_map_mn(&c.m_vmn_hi, at<void>(ws, P.gv_hi), rg, y.KG, y.KG, bk);
+    ok &= make_map_mn(&c.m_vmn_lo, at<void>(ws, P.split ? P.gv_lo : P.gv_hi), rg, y.KG, y.KG, bk);
   }
   return ok ? SO2_OK : SO2_ERR_CUDA;
 }
@@ -396,16 +450,15 @@ so2_status pack_weights(Ctx &c, const void *w) {
 so2_status chunk_prep(Ctx &c, int64_t e0, int M, const int64_t *ei, const float *ev, int key_row,
                       so2conv_params prm) {
   const Plan &P = c.P;
-  const int tpb = P.y.dsz <= 200 ? 64 : 32;
-  const int smem = tpb * P.y.dsz * static_cast<int>(sizeof(float));
-  if (!allow_smem(k_edge_prep, smem)) return SO2_ERR_CUDA;
-  k_edge_prep<<<(M + tpb - 1) / tpb, tpb, smem, c.s>>>(P.y, at<int>(c.ws, P.perm), e0, M, ei, P.E,
-                                                       P.N, key_row, ev, at<EdgeRec>(c.ws, P.rec),
-                                                       at<float>(c.ws, P.geo),
-                                                       at<float>(c.ws, P.D), c.st);
+  const int smem = 8 * (P.y.dsz + 16) * static_cast<int>(sizeof(float));
+  k_edge_prep<<<warp_grid(M, 8), 256, smem, c.s>>>(P.y, at<int>(c.ws, P.perm), e0, M, ei, P.E, P.N,
+                                                   key_row, ev, at<EdgeRec>(c.ws, P.rec),
+                                                   at<float>(c.ws, P.geo), at<float>(c.ws, P.D),
+                                                   c.st);
   CKL();
-  k_edge_gate<<<M, 128, 0, c.s>>>(P.y, c.d->rbf_cutoff, M, at<float>(c.ws, P.geo), prm.w_rad,
-                                  prm.b_rad, at<float>(c.ws, P.gate));
+  k_edge_gate<<<(M + GATE_EDGES - 1) / GATE_EDGES, 128, GATE_EDGES * P.y.nr * sizeof(float),
+                c.s>>>(P.y, c.d->rbf_cutoff, M, at<float>(c.ws, P.geo), prm.w_rad, prm.b_rad,
+                       at<float>(c.ws, P.gate));
   CKL();
   return SO2_OK;
 }
@@ -417,12 +470,13 @@ so2_status rotate(Ctx &c, int M, const void *X, bool xbf16, int side, int use_sr
   const Plan &P = c.P;
   const EdgeRec *rec = at<EdgeRec>(c.ws, P.rec);
   const float *D = at<float>(c.ws, P.D);
+  const int dsm = 8 * P.y.dsz * static_cast<int>(sizeof(float));  // staged D per warp
   if (xbf16) {
-    DISPATCH_MM(P.y.mmax, (k_rotate_gather<__nv_bfloat16, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+    DISPATCH_MM(P.y.mmax, (k_rotate_gather<__nv_bfloat16, MM><<<warp_grid(M, 8), 256, dsm, c.s>>>(
                                P.y, M, rec, D, static_cast<const __nv_bfloat16 *>(X), side,
                                use_src, A, B, omega, hi, lo, ld)));
   } else {
-    DISPATCH_MM(P.y.mmax, (k_rotate_gather<float, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+    DISPATCH_MM(P.y.mmax, (k_rotate_gather<float, MM><<<warp_grid(M, 8), 256, dsm, c.s>>>(
                                P.y, M, rec, D, static_cast<const float *>(X), side, use_src, A,
                                B, omega, hi, lo, ld)));
   }
@@ -455,64 +509,85 @@ so2_status rotate_g(Ctx &c, int M, const float *G, int row0, Coef A, Coef B = ZE
   return rotate(c, M, G, false, 1, 0, A, B, omega, hi, lo, P.y.KG);
 }
 
-// Transpose rows [row0, row0 + M) of an operand plane pair into column
-// segment `seg` of its transposed planes (columns past M zero up to Kp).
-so2_status transpose_seg(Ctx &c, int M, bool out_side, int row0, int seg) {
+// Zero rows [row0 + M, row0 + roundup(M, 64)) of both planes of the input
+// (out_side = false) or output side operand, so that a weight-gradient
+// product over the padded edge range adds nothing for them.
+so2_status zero_tail(Ctx &c, int M, bool out_side, int row0) {
   const Plan &P = c.P;
-  const Layout &y = P.y;
-  const int K = out_side ? y.KG : y.KA;
-  const int nseg = out_side ? P.ngv : P.na;
-  const int ldo = nseg * P.chunkp;
+  const int K = out_side ? P.y.KG : P.y.KA;
   const int Kp = round_up(M, 64);
-  const size_t ioff = (size_t)row0 * K, ooff = (size_t)seg * P.chunkp;
-  for (int plane = 0; plane < (P.split ? 2 : 1); ++plane) {
-    const __nv_bfloat16 *in = at<__nv_bfloat16>(
-        c.ws, out_side ? (plane ? P.gv_lo : P.gv_hi) : (plane ? P.a_lo : P.a_hi));
-    __nv_bfloat16 *out = at<__nv_bfloat16>(
-        c.ws, out_side ? (plane ? P.gvT_lo : P.gvT_hi) : (plane ? P.aT_lo : P.aT_hi));
-    k_transpose_bf16<<<dim3((K + 63) / 64, Kp / 64), 256, 0, c.s>>>(in + ioff, M, K, K,
-                                                                    out + ooff, Kp, ldo);
-    CKL();
+  if (Kp == M) return SO2_OK;
+  const size_t off = (size_t)(row0 + M) * K * 2, bytes = (size_t)(Kp - M) * K * 2;
+  char *hi = at<char>(c.ws, out_side ? P.gv_hi : P.a_hi);
+  CK(cudaMemsetAsync(hi + off, 0, bytes, c.s));
+  if (P.split) {
+    char *lo = at<char>(c.ws, out_side ? P.gv_lo : P.a_lo);
+    CK(cudaMemsetAsync(lo + off, 0, bytes, c.s));
   }
   return SO2_OK;
 }
 
-// dW (+)= (rows seg_g of the output-side operand)^T (rows seg_a of the input side).
+// dW (+)= (rows of segment seg_g of the output-side planes)^T x (rows of
+// segment seg_a of the input-side planes): K = edges, both operands read
+// MN-major straight from the edge-major planes.
 so2_status gemm_dw(Ctx &c, int M, int seg_g, int seg_a) {
   const Plan &P = c.P;
   const Layout &y = P.y;
   const int Kp = round_up(M, 64);
+  // the output is small (a few hundred tiles at most) and K long: split K
+  // until the launch covers about two waves of SMs
+  int tiles = 0;
+  for (int g = 0; g < y.ng; ++g)
+    tiles += ((y.Kout[g] + GEMM_BM - 1) / GEMM_BM) * ((y.Kin[g] + GEMM_BN - 1) / GEMM_BN);
+  int ksplit = (2 * num_sms() + tiles - 1) / tiles;
+  if (ksplit > Kp / 512) ksplit = Kp / 512 > 0 ? Kp / 512 : 1;  // keep >= 512 edges per split
   GemmLauncher L;
   for (int g = 0; g < y.ng; ++g)
-    L.add(y.Kout[g], y.Kin[g], Kp, y.kout_off[g], seg_g * P.chunkp, y.kin_off[g],
-          seg_a * P.chunkp, static_cast<long long>(y.wr_off[g]) * y.WK, y.WK);
-  CK(launch_gemm(2, P.split, c.m_gvT_hi, c.m_gvT_lo, c.m_aT_hi, c.m_aT_lo, L.p,
-                 at<float>(c.ws, P.dws), 1, c.st, c.s));
+    L.add(y.Kout[g], y.Kin[g], Kp, y.kout_off[g], seg_g * P.chunk, y.kin_off[g], seg_a * P.chunk,
+          static_cast<long long>(y.wr_off[g]) * y.WK, y.WK, ksplit);
+  CK(launch_gemm(2, P.split, c.m_vmn_hi, c.m_vmn_lo, c.m_amn_hi, c.m_amn_lo, L.p,
+                 at<float>(c.ws, P.dws), 1, c.st, c.s, nullptr, true, true));
   return SO2_OK;
 }
 
 // Ga rows = output-side operand rows times the transposed stacked weights.
-so2_status gemm_ga(Ctx &c, int rows) {
+so2_status gemm_ga(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store = true) {
   const Plan &P = c.P;
   const Layout &y = P.y;
   GemmLauncher L;
   for (int g = 0; g < y.ng; ++g)
     L.add(rows, y.Kin[g], y.Kout_pad[g], 0, y.kout_off[g], y.wt_off[g], 0, y.kin_off[g], y.KA);
   CK(launch_gemm(1, P.split, c.m_v_hi, c.m_v_lo, c.m_wtr_hi, c.m_wtr_lo, L.p,
-                 at<float>(c.ws, P.Ga), 0, c.st, c.s));
+                 at<float>(c.ws, P.Ga), 0, c.st, c.s, sc, store));
   return SO2_OK;
 }
 
 // V = rotated features times stacked weights (one group per m).
-so2_status gemm_v(Ctx &c, int rows) {
+so2_status gemm_v(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store = true) {
   const Plan &P = c.P;
   const Layout &y = P.y;
   GemmLauncher L;
   for (int g = 0; g < y.ng; ++g)
     L.add(rows, y.Kout[g], y.Kin_pad[g], 0, y.kin_off[g], y.wr_off[g], 0, y.kout_off[g], y.KG);
   CK(launch_gemm(0, P.split, c.m_a_hi, c.m_a_lo, c.m_wst_hi, c.m_wst_lo, L.p, at<float>(c.ws, P.V), 0,
-                 c.st, c.s));
+                 c.st, c.s, sc, store));
   return SO2_OK;
+}
+
+// The fused gate + inverse rotation + reduction epilogue needs whole 32-wide
+// channel chunks inside one edge-frame row.
+bool fusable(int C) { return C % 32 == 0; }
+
+GemmScatter make_scatter(Ctx &c, const float *gate, float *out, int C) {
+  GemmScatter sc;
+  sc.rec = at<int4>(c.ws, c.P.rec);
+  sc.gate = gate;
+  sc.D = at<float>(c.ws, c.P.D);
+  sc.out = out;
+  sc.C = C;
+  sc.L = c.P.y.L;
+  sc.dsz = c.P.y.dsz;
+  return sc;
 }
 
 // Node-centric inverse rotation on reduction (see k_scatter_nodes) for the
@@ -556,8 +631,8 @@ so2_status rad_grads(Ctx &c, int M, const float *Ag, const float *Bg, const floa
                                         omega, at<float>(c.ws, P.radp));
   CKL();
   const int Pn = (y.nr + 1) * y.co;
-  k_rad_reduce<<<(Pn + 255) / 256, 256, 0, c.s>>>(y, nblk, at<float>(c.ws, P.radp), grad_w_rad,
-                                                   grad_b);
+  k_rad_reduce<<<(Pn + 31) / 32, 256, 0, c.s>>>(y, nblk, at<float>(c.ws, P.radp), grad_w_rad,
+                                                 grad_b);
   CKL();
   return SO2_OK;
 }
@@ -611,10 +686,16 @@ so2_status so2conv_forward(const so2conv_desc *desc, int64_t N, int64_t E, const
     const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
     if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 1, prm)) != SO2_OK) return r;
     if ((r = rotate_x(c, M, x, P.xbf16)) != SO2_OK) return r;
-    if ((r = gemm_v(c, M)) != SO2_OK) return r;
-    if ((r = scatter(c, e0, M, one_term(at<float>(ws, P.V), y.KG, arr(at<float>(ws, P.gate))), 1,
-                     nullptr, out)) != SO2_OK)
-      return r;
+    if (fusable(y.co)) {
+      // product, gate, inverse rotation and reduction in one kernel
+      const GemmScatter sc = make_scatter(c, at<float>(ws, P.gate), out, y.co);
+      if ((r = gemm_v(c, M, &sc, false)) != SO2_OK) return r;
+    } else {
+      if ((r = gemm_v(c, M)) != SO2_OK) return r;
+      if ((r = scatter(c, e0, M, one_term(at<float>(ws, P.V), y.KG, arr(at<float>(ws, P.gate))),
+                       1, nullptr, out)) != SO2_OK)
+        return r;
+    }
   }
   return SO2_OK;
 }
@@ -658,24 +739,31 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
     // Gv = g * (D G[dst]) on the kept rows
     if ((r = rotate_g(c, M, grad_out, 0, arr(at<float>(ws, P.gate)))) != SO2_OK) return r;
     if (need_v && (r = gemm_v(c, M)) != SO2_OK) return r;
-    if (need_ga && (r = gemm_ga(c, M)) != SO2_OK) return r;
+    const bool fuse_gx = grad_x && fusable(y.ci);
+    if (need_ga) {
+      const GemmScatter sc = make_scatter(c, nullptr, grad_x, y.ci);
+      if ((r = gemm_ga(c, M, fuse_gx ? &sc : nullptr, grad_edge_vec != nullptr || !fuse_gx)) !=
+          SO2_OK)
+        return r;
+    }
     if (grad_w) {
-      if ((r = transpose_seg(c, M, false, 0, 0)) != SO2_OK) return r;
-      if ((r = transpose_seg(c, M, true, 0, 0)) != SO2_OK) return r;
+      if ((r = zero_tail(c, M, false, 0)) != SO2_OK) return r;
+      if ((r = zero_tail(c, M, true, 0)) != SO2_OK) return r;
       if ((r = gemm_dw(c, M, 0, 0)) != SO2_OK) return r;
     }
-    if (grad_x && (r = scatter(c, e0, M, one_term(at<float>(ws, P.Ga), y.KA, ONE), 0, nullptr,
-                               grad_x)) != SO2_OK)
+    if (grad_x && !fuse_gx &&
+        (r = scatter(c, e0, M, one_term(at<float>(ws, P.Ga), y.KA, ONE), 0, nullptr, grad_x)) !=
+            SO2_OK)
       return r;
     if (need_v) {
       if (P.xbf16) {
-        DISPATCH_MM(y.mmax, (k_edge_terms<__nv_bfloat16, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+        DISPATCH_MM(y.mmax, (k_edge_terms<__nv_bfloat16, MM><<<warp_grid(M, 8), 256, 8 * y.dsz * 4, c.s>>>(
                                 y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
                                 at<float>(ws, P.gate), grad_out,
                                 static_cast<const __nv_bfloat16 *>(x), at<float>(ws, P.V),
                                 at<float>(ws, P.Ga), at<float>(ws, P.Gg), at<float>(ws, P.h))));
       } else {
-        DISPATCH_MM(y.mmax, (k_edge_terms<float, MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+        DISPATCH_MM(y.mmax, (k_edge_terms<float, MM><<<warp_grid(M, 8), 256, 8 * y.dsz * 4, c.s>>>(
                                 y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
                                 at<float>(ws, P.gate), grad_out, static_cast<const float *>(x),
                                 at<float>(ws, P.V), at<float>(ws, P.Ga), at<float>(ws, P.Gg),
@@ -830,12 +918,12 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
         if (has_r && (r = rotate_g(c, M, grad_out, 0, dgate, gate, omega)) != SO2_OK) return r;
         if ((r = rotate_g(c, M, grad_out, ch, gate)) != SO2_OK) return r;
         if (has_r) {
-          if ((r = transpose_seg(c, M, true, 0, 0)) != SO2_OK) return r;
-          if ((r = transpose_seg(c, M, false, 0, 0)) != SO2_OK) return r;
-          if ((r = transpose_seg(c, M, false, ch, 1)) != SO2_OK) return r;
+          if ((r = zero_tail(c, M, true, 0)) != SO2_OK) return r;
+          if ((r = zero_tail(c, M, false, 0)) != SO2_OK) return r;
+          if ((r = zero_tail(c, M, false, ch)) != SO2_OK) return r;
         }
-        if ((r = transpose_seg(c, M, true, ch, 1)) != SO2_OK) return r;
-        if (has_x && (r = transpose_seg(c, M, false, 2 * ch, 2)) != SO2_OK) return r;
+        if ((r = zero_tail(c, M, true, ch)) != SO2_OK) return r;
+        if (has_x && (r = zero_tail(c, M, false, 2 * ch)) != SO2_OK) return r;
         if (has_r) {
           if ((r = gemm_dw(c, M, 0, 0)) != SO2_OK) return r;  // P (x) a
           if ((r = gemm_dw(c, M, 1, 1)) != SO2_OK) return r;  // Gv (x) da
@@ -930,8 +1018,9 @@ so2_status so2conv_edge_frames(int32_t lmax, int64_t E, const float *edge_vec, f
   if (lmax < 0 || lmax > LMAX_SUPPORTED || E < 0) return SO2_ERR_UNSUPPORTED;
   if (E == 0) return SO2_OK;
   if (!edge_vec) return SO2_ERR_INVALID_ARG;
-  k_frames<<<(E + 127) / 128, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(lmax, E, edge_vec,
-                                                                             R_out, D_out);
+  const int smem = 8 * (dsize(lmax) + 16) * static_cast<int>(sizeof(float));
+  k_frames<<<warp_grid(static_cast<int>(E < (1 << 30) ? E : (1 << 30)), 8), 256, smem,
+             reinterpret_cast<cudaStream_t>(stream)>>>(lmax, E, edge_vec, R_out, D_out);
   return cudaPeekAtLastError() == cudaSuccess ? SO2_OK : SO2_ERR_CUDA;
 }
 

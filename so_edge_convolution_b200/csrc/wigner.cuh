@@ -67,65 +67,71 @@ __device__ __forceinline__ bool make_frame(float rx, float ry, float rz, Frame &
   return true;
 }
 
-// Full blocks D^0..D^lmax, each (2l+1)^2 row-major, concatenated into D.
-__device__ inline void wigner_blocks(const float *R, int lmax, float *D) {
-  D[0] = 1.f;
-  if (lmax < 1) return;
-  // (y, z, x) ordering: sh index 0 <- y(1), 1 <- z(2), 2 <- x(0)
-  const int pm[3] = {1, 2, 0};
-  float *D1 = D + dblock_off(1);
-  for (int a = 0; a < 3; ++a)
-    for (int b = 0; b < 3; ++b) D1[a * 3 + b] = R[pm[a] * 3 + pm[b]];
+// Entry (m, n) of D^l (l >= 2) from D^1 (row-major 3x3, index (i+1)*3+(j+1))
+// and D^{l-1} (row-major (2l-1)^2): the Ivanic-Ruedenberg recursion.
+__device__ __forceinline__ float ir_entry(int l, int m, int n, const float *D1, const float *Dp) {
+  const int wp = 2 * l - 1;
+  auto r1 = [&](int i, int j) { return D1[(i + 1) * 3 + (j + 1)]; };
+  auto rp = [&](int a, int b) { return Dp[(a + l - 1) * wp + (b + l - 1)]; };
+  auto P = [&](int i, int a, int b) -> float {
+    if (b == -l) return r1(i, 1) * rp(a, -l + 1) + r1(i, -1) * rp(a, l - 1);
+    if (b == l) return r1(i, 1) * rp(a, l - 1) - r1(i, -1) * rp(a, -l + 1);
+    return r1(i, 0) * rp(a, b);
+  };
+  const int am = m < 0 ? -m : m;
+  const int an = n < 0 ? -n : n;
+  const int dm0 = (m == 0);
+  const float den = (an == l) ? static_cast<float>((2 * l) * (2 * l - 1))
+                              : static_cast<float>((l + n) * (l - n));
+  const float u = sqrtf(static_cast<float>((l + m) * (l - m)) / den);
+  const float v = 0.5f * sqrtf(static_cast<float>((1 + dm0) * (l + am - 1) * (l + am)) / den) *
+                  static_cast<float>(1 - 2 * dm0);
+  const float wc = -0.5f * sqrtf(static_cast<float>((l - am - 1) * (l - am)) / den) *
+                   static_cast<float>(1 - dm0);
+  float val = 0.f;
+  if (u != 0.f) val += u * P(0, m, n);
+  if (v != 0.f) {
+    float V;
+    if (m == 0) {
+      V = P(1, 1, n) + P(-1, -1, n);
+    } else if (m > 0) {
+      V = P(1, m - 1, n) * (m == 1 ? 1.41421356237f : 1.f) - (m == 1 ? 0.f : P(-1, -m + 1, n));
+    } else {
+      V = (m == -1 ? 0.f : P(1, m + 1, n)) + P(-1, -m - 1, n) * (m == -1 ? 1.41421356237f : 1.f);
+    }
+    val += v * V;
+  }
+  if (wc != 0.f) {
+    float Wv;
+    if (m > 0)
+      Wv = P(1, m + 1, n) + P(-1, -m - 1, n);
+    else
+      Wv = P(1, m - 1, n) - P(-1, -m + 1, n);
+    val += wc * Wv;
+  }
+  return val;
+}
+
+// Full blocks D^0..D^lmax (each (2l+1)^2 row-major, concatenated) of the
+// rotation R, computed by one warp into D (shared memory): the lanes share
+// the entries of each level, levels one after another.
+__device__ inline void wigner_blocks_warp(const float *R, int lmax, float *D) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) D[0] = 1.f;
+  if (lmax >= 1 && lane < 9) {
+    // (y, z, x) ordering: sh index 0 <- y(1), 1 <- z(2), 2 <- x(0)
+    const int pm[3] = {1, 2, 0};
+    const int a = lane / 3, b = lane % 3;
+    D[dblock_off(1) + lane] = R[pm[a] * 3 + pm[b]];
+  }
+  __syncwarp();
+  const float *D1 = D + dblock_off(1);
   for (int l = 2; l <= lmax; ++l) {
     const float *Dp = D + dblock_off(l - 1);
     float *Dl = D + dblock_off(l);
-    const int wp = 2 * l - 1;  // width of D^{l-1}
     const int w = 2 * l + 1;
-    auto r1 = [&](int i, int j) { return D1[(i + 1) * 3 + (j + 1)]; };
-    auto rp = [&](int a, int b) { return Dp[(a + l - 1) * wp + (b + l - 1)]; };
-    auto P = [&](int i, int a, int b) -> float {
-      if (b == -l) return r1(i, 1) * rp(a, -l + 1) + r1(i, -1) * rp(a, l - 1);
-      if (b == l) return r1(i, 1) * rp(a, l - 1) - r1(i, -1) * rp(a, -l + 1);
-      return r1(i, 0) * rp(a, b);
-    };
-    for (int m = -l; m <= l; ++m) {
-      const int am = m < 0 ? -m : m;
-      const int dm0 = (m == 0);
-      for (int n = -l; n <= l; ++n) {
-        const int an = n < 0 ? -n : n;
-        const float den = (an == l) ? static_cast<float>((2 * l) * (2 * l - 1))
-                                    : static_cast<float>((l + n) * (l - n));
-        const float u = sqrtf(static_cast<float>((l + m) * (l - m)) / den);
-        const float v = 0.5f * sqrtf(static_cast<float>((1 + dm0) * (l + am - 1) * (l + am)) / den) *
-                        static_cast<float>(1 - 2 * dm0);
-        const float wc = -0.5f * sqrtf(static_cast<float>((l - am - 1) * (l - am)) / den) *
-                         static_cast<float>(1 - dm0);
-        float val = 0.f;
-        if (u != 0.f) val += u * P(0, m, n);
-        if (v != 0.f) {
-          float V;
-          if (m == 0) {
-            V = P(1, 1, n) + P(-1, -1, n);
-          } else if (m > 0) {
-            V = P(1, m - 1, n) * (m == 1 ? 1.41421356237f : 1.f) -
-                (m == 1 ? 0.f : P(-1, -m + 1, n));
-          } else {
-            V = (m == -1 ? 0.f : P(1, m + 1, n)) +
-                P(-1, -m - 1, n) * (m == -1 ? 1.41421356237f : 1.f);
-          }
-          val += v * V;
-        }
-        if (wc != 0.f) {
-          float W;
-          if (m > 0)
-            W = P(1, m + 1, n) + P(-1, -m - 1, n);
-          else
-            W = P(1, m - 1, n) - P(-1, -m + 1, n);
-          val += wc * W;
-        }
-        Dl[(m + l) * w + (n + l)] = val;
-      }
-    }
+    for (int idx = lane; idx < w * w; idx += 32) Dl[idx] = ir_entry(l, idx / w - l, idx % w - l, D1, Dp);
+    __syncwarp();
   }
 }
 

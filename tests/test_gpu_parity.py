@@ -153,7 +153,8 @@ def test_backward_partial_outputs():
         part = _gpu_backward(p, need=need)
         assert set(part) == set(need)
         for k in need:
-            assert torch.equal(part[k], full[k]), k
+            # node sums are reduced with atomics: the order may differ per run
+            assert rel_err(part[k], full[k]) < 1e-6, k
 
 
 def _integer_problem(n=200, nb=20, seed=7):
