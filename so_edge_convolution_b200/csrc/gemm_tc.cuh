@@ -23,7 +23,7 @@
 #include "common.cuh"
 
 #ifndef SO2_EPI_WARPS
-#define SO2_EPI_WARPS 8
+#define SO2_EPI_WARPS 12
 #endif
 
 namespace so2 {
@@ -70,8 +70,8 @@ struct GemmParams {
   DevStatus *status;
 };
 
-constexpr int EPI_WARPS = SO2_EPI_WARPS;  // 4 or 8: one or two per TMEM lane quadrant
-static_assert(EPI_WARPS == 4 || EPI_WARPS == 8, "epilogue warps per TMEM quadrant");
+constexpr int EPI_WARPS = SO2_EPI_WARPS;  // 4, 8 or 12: one to three per TMEM lane quadrant
+static_assert(EPI_WARPS % 4 == 0 && EPI_WARPS <= 12, "epilogue warps per TMEM quadrant");
 constexpr int EPI_SMEM_PER_WARP = (32 * 33 + 32 * 16 + 32) * 4;  // multiple of 16 B
 constexpr int EPI_SMEM = EPI_WARPS * EPI_SMEM_PER_WARP;
 
@@ -123,42 +123,41 @@ __device__ __forceinline__ void epi_stage_d(const GemmParams &p, const GemmGroup
   }
 }
 
-// The sums of one warp-chunk for a fixed width W = 2l + 1 (see below).
+// The sums of one warp-chunk for a fixed width W = 2l + 1 (see below).  The
+// warp's 32 edges split into runs of equal node (a ballot finds the run
+// starts); each run is summed branch-free and flushed with W coalesced
+// atomics.
 template <int W>
 __device__ __forceinline__ void epi_rotate_reduce(const GemmScatter &S, int row_base, int l, int c,
-                                                  const EpiScratch &x, const float (&g)[32]) {
+                                                  const EpiScratch &x) {
   const int lane = threadIdx.x & 31;
   const int S_ = (S.L + 1) * (S.L + 1);
-  float acc[W];
+  const int my_key = x.keys[lane];
+  const int prev_key = lane ? x.keys[lane - 1] : -2;
+  unsigned starts = __ballot_sync(0xffffffffu, my_key != prev_key && my_key >= 0);
+  while (starts) {
+    const int s0 = __ffs(starts) - 1;
+    starts &= starts - 1;
+    const int s1 = starts ? __ffs(starts) - 1 : 32;
+    const int key = x.keys[s0];
+    float acc[W];
 #pragma unroll
-  for (int k = 0; k < W; ++k) acc[k] = 0.f;
-  int cur = x.keys[0];
+    for (int k = 0; k < W; ++k) acc[k] = 0.f;
+#pragma unroll 4
+    for (int el = s0; el < s1; ++el) {
+      if (x.keys[el] < 0) break;  // past the end of the chunk (uniform)
+      const float v = x.T[el * 33 + lane];
+      const float4 *d4 = reinterpret_cast<const float4 *>(x.Dw + el * 16);
 #pragma unroll
-  for (int el = 0; el < 32; ++el) {
-    const int k_e = x.keys[el];
-    if (k_e != cur) {
-      if (cur >= 0) {
-        float *o = S.out + ((int64_t)cur * S_ + l * l) * S.C + c;
-#pragma unroll
-        for (int k = 0; k < W; ++k) atomicAdd(o + k * S.C, acc[k]);
+      for (int k4 = 0; k4 < (W + 3) / 4; ++k4) {
+        const float4 d = d4[k4];
+        if (4 * k4 + 0 < W) acc[4 * k4 + 0] += d.x * v;
+        if (4 * k4 + 1 < W) acc[4 * k4 + 1] += d.y * v;
+        if (4 * k4 + 2 < W) acc[4 * k4 + 2] += d.z * v;
+        if (4 * k4 + 3 < W) acc[4 * k4 + 3] += d.w * v;
       }
-#pragma unroll
-      for (int k = 0; k < W; ++k) acc[k] = 0.f;
-      cur = k_e;
     }
-    const float v = x.T[el * 33 + lane] * g[el];
-    const float4 *d4 = reinterpret_cast<const float4 *>(x.Dw + el * 16);
-#pragma unroll
-    for (int k4 = 0; k4 < (W + 3) / 4; ++k4) {
-      const float4 d = d4[k4];
-      if (4 * k4 + 0 < W) acc[4 * k4 + 0] += d.x * v;
-      if (4 * k4 + 1 < W) acc[4 * k4 + 1] += d.y * v;
-      if (4 * k4 + 2 < W) acc[4 * k4 + 2] += d.z * v;
-      if (4 * k4 + 3 < W) acc[4 * k4 + 3] += d.w * v;
-    }
-  }
-  if (cur >= 0) {
-    float *o = S.out + ((int64_t)cur * S_ + l * l) * S.C + c;
+    float *o = S.out + ((int64_t)key * S_ + l * l) * S.C + c;
 #pragma unroll
     for (int k = 0; k < W; ++k) atomicAdd(o + k * S.C, acc[k]);
   }
@@ -177,18 +176,24 @@ __device__ __forceinline__ void epi_scatter_chunk(const GemmParams &p, int row_b
   __syncwarp();
   // lane = channel from here on
   const int c = c0 + lane;
-  float g[32];
+  if (S.gate) {
+    // all 32 gate loads in flight at once (coalesced per edge), then scale
+    float g[32];
 #pragma unroll
-  for (int el = 0; el < 32; ++el)
-    g[el] = (S.gate && x.keys[el] >= 0) ? S.gate[(int64_t)(row_base + el) * S.C + c] : 1.f;
+    for (int el = 0; el < 32; ++el)
+      g[el] = (x.keys[el] >= 0) ? S.gate[(int64_t)(row_base + el) * S.C + c] : 0.f;
+#pragma unroll
+    for (int el = 0; el < 32; ++el) x.T[el * 33 + lane] *= g[el];
+    __syncwarp();
+  }
   switch (2 * l + 1) {
-    case 1: epi_rotate_reduce<1>(S, row_base, l, c, x, g); break;
-    case 3: epi_rotate_reduce<3>(S, row_base, l, c, x, g); break;
-    case 5: epi_rotate_reduce<5>(S, row_base, l, c, x, g); break;
-    case 7: epi_rotate_reduce<7>(S, row_base, l, c, x, g); break;
-    case 9: epi_rotate_reduce<9>(S, row_base, l, c, x, g); break;
-    case 11: epi_rotate_reduce<11>(S, row_base, l, c, x, g); break;
-    default: epi_rotate_reduce<13>(S, row_base, l, c, x, g); break;
+    case 1: epi_rotate_reduce<1>(S, row_base, l, c, x); break;
+    case 3: epi_rotate_reduce<3>(S, row_base, l, c, x); break;
+    case 5: epi_rotate_reduce<5>(S, row_base, l, c, x); break;
+    case 7: epi_rotate_reduce<7>(S, row_base, l, c, x); break;
+    case 9: epi_rotate_reduce<9>(S, row_base, l, c, x); break;
+    case 11: epi_rotate_reduce<11>(S, row_base, l, c, x); break;
+    default: epi_rotate_reduce<13>(S, row_base, l, c, x); break;
   }
   __syncwarp();
 }
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp >= 2) {
     // ---------------- epilogue: TMEM -> registers -> C and/or node sums ----------------
     const int q = warp & 3;           // TMEM lane quadrant this warp may read
-    const int half = (warp - 2) >> 2;  // which half of the tile's column chunks (8 warps)
+    const int half = (warp - 2) >> 2;  // which share of the tile's column chunks
     const EpiScratch xs = epi_scratch(epi_smem + (warp - 2) * (EPI_SMEM_PER_WARP / 4));
     int tcount = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tcount) {
