@@ -242,7 +242,9 @@ __device__ __forceinline__ void stage_d(const float *De, int dsz, float *sD) {
   __syncwarp();
 }
 
-template <typename TX, int MM>
+// LC >= 0 fixes lmax at compile time (loops fully unrolled); -1 reads it
+// from the layout.
+template <typename TX, int MM, int LC = -1>
 __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec,
                                 const float *__restrict__ D, const TX *__restrict__ X, int side,
                                 int use_src, Coef A, Coef B, const float *__restrict__ omega,
@@ -271,13 +273,16 @@ __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec
     }
     for (int c = 4 * lane; c < C; c += 128) {
       const float4 ca = coef4(A, i, C, c), cb = coef4(B, i, C, c);
-      for (int l = 0; l <= y.L; ++l) {
+      const int L = LC >= 0 ? LC : y.L;
+#pragma unroll
+      for (int l = 0; l <= L; ++l) {
         float4 a[2 * W + 1];
 #pragma unroll
         for (int k = 0; k < 2 * W + 1; ++k) a[k] = make_float4(0.f, 0.f, 0.f, 0.f);
         const float *Dl = sD + dblock_off(l);
         const int w = 2 * l + 1;
         const int top = wide ? W : MM;
+#pragma unroll
         for (int mp = -l; mp <= l; ++mp) {
           const float4 xv = load4(Xn + (l * l + l + mp) * C + c);
 #pragma unroll
@@ -518,7 +523,9 @@ __global__ void k_unstack_grad(Layout y, BlockOffsets bo, const float *__restric
 // where v (mixing output) and Ga (gradient of the rotated input) come from
 // the two products.  h_x, h_y give the frame part of dL/dr.
 // ---------------------------------------------------------------------------
-template <typename TX, int MM>
+// PART: 3 = both sides in one pass; 1 = output side only (writes Gg and h);
+// 2 = input side only (adds its share to h).
+template <typename TX, int MM, int LC = -1, int PART = 3>
 __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
                              const float *__restrict__ D, const float *__restrict__ gate,
                              const float *__restrict__ G, const TX *__restrict__ X,
@@ -536,15 +543,17 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
     // output side
     const float *Gn = G + (int64_t)r.dst * y.S * y.co;
     const float *Vi = V + (int64_t)i * y.KG;
-    for (int c = 4 * lane; c < y.co; c += 128) {
+    for (int c = 4 * lane; (PART & 1) && c < y.co; c += 128) {
       const float4 gv = load4(gate + (int64_t)i * y.co + c);
       float4 gg = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int l = 0; l <= y.L; ++l) {
+#pragma unroll
+      for (int l = 0; l <= (LC >= 0 ? LC : y.L); ++l) {
         float4 b[2 * W + 1];
 #pragma unroll
         for (int k = 0; k < 2 * W + 1; ++k) b[k] = make_float4(0.f, 0.f, 0.f, 0.f);
         const float *Dl = sD + dblock_off(l);
         const int w = 2 * l + 1;
+#pragma unroll
         for (int mp = -l; mp <= l; ++mp) {
           const float4 gx = load4(Gn + (l * l + l + mp) * y.co + c);
 #pragma unroll
@@ -587,13 +596,15 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
     // input side
     const TX *Xn = X + (int64_t)r.src * y.S * y.ci;
     const float *Gai = Ga + (int64_t)i * y.KA;
-    for (int c = 4 * lane; c < y.ci; c += 128) {
-      for (int l = 0; l <= y.L; ++l) {
+    for (int c = 4 * lane; (PART & 2) && c < y.ci; c += 128) {
+#pragma unroll
+      for (int l = 0; l <= (LC >= 0 ? LC : y.L); ++l) {
         float4 b[2 * W + 1];
 #pragma unroll
         for (int k = 0; k < 2 * W + 1; ++k) b[k] = make_float4(0.f, 0.f, 0.f, 0.f);
         const float *Dl = sD + dblock_off(l);
         const int w = 2 * l + 1;
+#pragma unroll
         for (int mp = -l; mp <= l; ++mp) {
           const float4 xv = load4(Xn + (l * l + l + mp) * y.ci + c);
 #pragma unroll
@@ -633,8 +644,13 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
       hy += __shfl_xor_sync(0xffffffffu, hy, o);
     }
     if (lane == 0) {
-      h[2 * (int64_t)i] = hx;
-      h[2 * (int64_t)i + 1] = hy;
+      if (PART & 1) {
+        h[2 * (int64_t)i] = hx;
+        h[2 * (int64_t)i + 1] = hy;
+      } else {
+        h[2 * (int64_t)i] += hx;
+        h[2 * (int64_t)i + 1] += hy;
+      }
     }
   }
 }

@@ -244,6 +244,23 @@ int grid_for(int64_t n, int block) {
   return static_cast<int>(g);
 }
 
+// Common shapes get kernels with lmax fixed at compile time (LC), the rest
+// the generic ones (LC = -1).
+#define DISPATCH_LM(L_, mm, ...)                                        \
+  if ((L_) == 4 && (mm) == 2) {                                         \
+    constexpr int MM = 2, LC = 4;                                       \
+    __VA_ARGS__;                                                        \
+  } else if ((L_) == 6 && (mm) == 2) {                                  \
+    constexpr int MM = 2, LC = 6;                                       \
+    __VA_ARGS__;                                                        \
+  } else if ((L_) == 2 && (mm) == 2) {                                  \
+    constexpr int MM = 2, LC = 2;                                       \
+    __VA_ARGS__;                                                        \
+  } else {                                                              \
+    constexpr int LC = -1;                                              \
+    DISPATCH_MM(mm, __VA_ARGS__);                                       \
+  }
+
 #define DISPATCH_MM(mm, ...)                  \
   switch (mm) {                               \
     case 0: { constexpr int MM = 0; __VA_ARGS__; } break; \
@@ -472,11 +489,11 @@ so2_status rotate(Ctx &c, int M, const void *X, bool xbf16, int side, int use_sr
   const float *D = at<float>(c.ws, P.D);
   const int dsm = 8 * P.y.dsz * static_cast<int>(sizeof(float));  // staged D per warp
   if (xbf16) {
-    DISPATCH_MM(P.y.mmax, (k_rotate_gather<__nv_bfloat16, MM><<<warp_grid(M, 8), 256, dsm, c.s>>>(
+    DISPATCH_LM(P.y.L, P.y.mmax, (k_rotate_gather<__nv_bfloat16, MM, LC><<<warp_grid(M, 8), 256, dsm, c.s>>>(
                                P.y, M, rec, D, static_cast<const __nv_bfloat16 *>(X), side,
                                use_src, A, B, omega, hi, lo, ld)));
   } else {
-    DISPATCH_MM(P.y.mmax, (k_rotate_gather<float, MM><<<warp_grid(M, 8), 256, dsm, c.s>>>(
+    DISPATCH_LM(P.y.L, P.y.mmax, (k_rotate_gather<float, MM, LC><<<warp_grid(M, 8), 256, dsm, c.s>>>(
                                P.y, M, rec, D, static_cast<const float *>(X), side, use_src, A,
                                B, omega, hi, lo, ld)));
   }
@@ -756,18 +773,37 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
             SO2_OK)
       return r;
     if (need_v) {
-      if (P.xbf16) {
-        DISPATCH_MM(y.mmax, (k_edge_terms<__nv_bfloat16, MM><<<warp_grid(M, 8), 256, 8 * y.dsz * 4, c.s>>>(
-                                y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
-                                at<float>(ws, P.gate), grad_out,
-                                static_cast<const __nv_bfloat16 *>(x), at<float>(ws, P.V),
-                                at<float>(ws, P.Ga), at<float>(ws, P.Gg), at<float>(ws, P.h))));
-      } else {
-        DISPATCH_MM(y.mmax, (k_edge_terms<float, MM><<<warp_grid(M, 8), 256, 8 * y.dsz * 4, c.s>>>(
-                                y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
-                                at<float>(ws, P.gate), grad_out, static_cast<const float *>(x),
-                                at<float>(ws, P.V), at<float>(ws, P.Ga), at<float>(ws, P.Gg),
-                                at<float>(ws, P.h))));
+      {
+        const int sm = 8 * y.dsz * 4;
+        const int g = warp_grid(M, 8);
+        EdgeRec *rec = at<EdgeRec>(ws, P.rec);
+        float *Dp = at<float>(ws, P.D), *gate = at<float>(ws, P.gate), *Vp = at<float>(ws, P.V);
+        float *Gap = at<float>(ws, P.Ga), *Ggp = at<float>(ws, P.Gg), *hp = at<float>(ws, P.h);
+        if (P.xbf16) {
+          const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+          DISPATCH_LM(y.L, y.mmax,
+                      if (LC >= 0 && LC <= 4) {  // lmax 6 unrolled spills
+                        k_edge_terms<__nv_bfloat16, MM, LC, 1><<<g, 256, sm, c.s>>>(
+                            y, M, rec, Dp, gate, grad_out, xb, Vp, Gap, Ggp, hp);
+                        k_edge_terms<__nv_bfloat16, MM, LC, 2><<<g, 256, sm, c.s>>>(
+                            y, M, rec, Dp, gate, grad_out, xb, Vp, Gap, Ggp, hp);
+                      } else {
+                        k_edge_terms<__nv_bfloat16, MM><<<g, 256, sm, c.s>>>(
+                            y, M, rec, Dp, gate, grad_out, xb, Vp, Gap, Ggp, hp);
+                      });
+        } else {
+          const float *xf = static_cast<const float *>(x);
+          DISPATCH_LM(y.L, y.mmax,
+                      if (LC >= 0 && LC <= 4) {  // lmax 6 unrolled spills
+                        k_edge_terms<float, MM, LC, 1><<<g, 256, sm, c.s>>>(
+                            y, M, rec, Dp, gate, grad_out, xf, Vp, Gap, Ggp, hp);
+                        k_edge_terms<float, MM, LC, 2><<<g, 256, sm, c.s>>>(
+                            y, M, rec, Dp, gate, grad_out, xf, Vp, Gap, Ggp, hp);
+                      } else {
+                        k_edge_terms<float, MM><<<g, 256, sm, c.s>>>(
+                            y, M, rec, Dp, gate, grad_out, xf, Vp, Gap, Ggp, hp);
+                      });
+        }
       }
       CKL();
       if (grad_edge_vec) {
