@@ -68,20 +68,32 @@ __global__ void k_place(const int64_t *__restrict__ keys, int64_t E, int64_t N,
   }
 }
 
-// Within each key's segment, order the edge ids ascending (insertion sort by
-// one thread per segment), which makes the sort stable and deterministic.
+// Within each key's segment, order the edge ids ascending, which makes the
+// sort stable and deterministic.  One warp per segment: segments of up to 32
+// edges are placed by rank (each lane counts the smaller ids); longer ones
+// fall back to an insertion sort by lane 0.
 __global__ void k_sort_segments(const int *__restrict__ offsets, int64_t N, int *__restrict__ perm) {
-  for (int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; n < N;
-       n += (int64_t)gridDim.x * blockDim.x) {
-    const int b = offsets[n], e = offsets[n + 1];
-    for (int i = b + 1; i < e; ++i) {
-      const int v = perm[i];
-      int j = i - 1;
-      while (j >= b && perm[j] > v) {
-        perm[j + 1] = perm[j];
-        --j;
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  for (int64_t n = blockIdx.x * (int64_t)wpb + (threadIdx.x >> 5); n < N;
+       n += (int64_t)gridDim.x * wpb) {
+    const int b = offsets[n], e = offsets[n + 1], len = e - b;
+    if (len <= 1) continue;
+    if (len <= 32) {
+      const int v = lane < len ? perm[b + lane] : 0x7fffffff;
+      int rank = 0;
+      for (int j = 0; j < len; ++j) rank += (__shfl_sync(0xffffffffu, v, j) < v);
+      __syncwarp();
+      if (lane < len) perm[b + rank] = v;
+    } else if (lane == 0) {
+      for (int i = b + 1; i < e; ++i) {
+        const int v = perm[i];
+        int j = i - 1;
+        while (j >= b && perm[j] > v) {
+          perm[j + 1] = perm[j];
+          --j;
+        }
+        perm[j + 1] = v;
       }
-      perm[j + 1] = v;
     }
   }
 }
@@ -103,7 +115,8 @@ constexpr int GEO = 16;
 __global__ void k_edge_prep(Layout y, const int *__restrict__ perm, int64_t e0, int M,
                             const int64_t *__restrict__ ei, int64_t E, int64_t N, int key_row,
                             const float *__restrict__ edge_vec, EdgeRec *__restrict__ rec,
-                            float *__restrict__ geo, float *__restrict__ D, DevStatus *st) {
+                            float *__restrict__ geo, float *__restrict__ D,
+                            const float *__restrict__ ir_table, DevStatus *st) {
   extern __shared__ float sDall[];  // [warps][dsz + 16]
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
   float *sD = sDall + (threadIdx.x >> 5) * (y.dsz + 16);
@@ -136,7 +149,7 @@ __global__ void k_edge_prep(Layout y, const int *__restrict__ perm, int64_t e0, 
       }
     }
     __syncwarp();
-    wigner_blocks_warp(sR, y.L, sD);
+    wigner_blocks_warp(sR, y.L, sD, ir_table);
     float *dst = D + (int64_t)i * y.dsz;
     for (int k = lane; k < y.dsz; k += 32) dst[k] = sD[k];
   }
@@ -464,27 +477,31 @@ struct BlockOffsets {
   long long off[2 * MAX_GROUPS];
 };
 
+// transposed = 0: stacked [n][k] planes (coalesced over k); transposed = 1:
+// their transposes [k][n] (coalesced over n).
 template <typename TW>
-__global__ void k_pack_weights(Layout y, BlockOffsets bo, const TW *__restrict__ w,
-                               __nv_bfloat16 *__restrict__ wst_hi, __nv_bfloat16 *__restrict__ wst_lo,
-                               __nv_bfloat16 *__restrict__ wtr_hi, __nv_bfloat16 *__restrict__ wtr_lo) {
+__global__ void k_pack_weights(Layout y, BlockOffsets bo, const TW *__restrict__ w, int transposed,
+                               __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo) {
   const int g = blockIdx.y;
   if (g >= y.ng) return;
   const int64_t total = (int64_t)y.Kout[g] * y.Kin[g];
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total;
        t += (int64_t)gridDim.x * blockDim.x) {
-    const int n = static_cast<int>(t / y.Kin[g]), k = static_cast<int>(t % y.Kin[g]);
+    int n, k;
+    if (transposed) {
+      k = static_cast<int>(t / y.Kout[g]);
+      n = static_cast<int>(t % y.Kout[g]);
+    } else {
+      n = static_cast<int>(t / y.Kin[g]);
+      k = static_cast<int>(t % y.Kin[g]);
+    }
     const float v = stacked_w(y, w, bo.off, g, n, k);
     __nv_bfloat16 h, l;
     split_bf16(v, h, l);
-    const int64_t a = (int64_t)(y.wr_off[g] + n) * y.WK + k;
-    const int64_t b = (int64_t)(y.wt_off[g] + k) * y.WTK + n;
-    wst_hi[a] = h;
-    wtr_hi[b] = h;
-    if (wst_lo) {
-      wst_lo[a] = l;
-      wtr_lo[b] = l;
-    }
+    const int64_t a = transposed ? (int64_t)(y.wt_off[g] + k) * y.WTK + n
+                                 : (int64_t)(y.wr_off[g] + n) * y.WK + k;
+    hi[a] = h;
+    if (lo) lo[a] = l;
   }
 }
 
@@ -698,8 +715,11 @@ __global__ void k_edge_final(Layout y, float cutoff, int M, const EdgeRec *__res
 // Radial-gate gradients, stage 1: each block sums, over a tile of RAD_TILE
 // edges, phi_k(d_i) A[i][c'] + phi'_k(d_i) dd_i B[i][c'] (rows k < nr) and
 // A[i][c'] (bias row k = nr) into part[block][k][c'].  B (and dd_i =
-// omega[i][2]) is optional.  Stage 2 adds the blocks in order.
+// omega[i][2]) is optional.  One thread per channel keeps all nr + 1 sums
+// in registers and reads each product once.  Stage 2 adds the blocks in
+// order.
 constexpr int RAD_TILE = 256;
+constexpr int RAD_MAX_NR = 64;
 __global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__restrict__ geo,
                               const float *__restrict__ Ag, const float *__restrict__ Bg,
                               const float *__restrict__ omega, float *__restrict__ part) {
@@ -719,17 +739,28 @@ __global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__rest
   }
   __syncthreads();
   const int P = (y.nr + 1) * y.co;
-  for (int pidx = threadIdx.x; pidx < P; pidx += blockDim.x) {
-    const int k = pidx / y.co, c = pidx % y.co;
-    float s = 0.f;
-    if (k < y.nr) {
-      for (int i = 0; i < n; ++i) s += phi[i * y.nr + k] * Ag[(int64_t)(i0 + i) * y.co + c];
-      if (Bg)
-        for (int i = 0; i < n; ++i) s += dphi[i * y.nr + k] * Bg[(int64_t)(i0 + i) * y.co + c];
-    } else {
-      for (int i = 0; i < n; ++i) s += Ag[(int64_t)(i0 + i) * y.co + c];
+  for (int c = threadIdx.x; c < y.co; c += blockDim.x) {
+    for (int k0 = 0; k0 < y.nr; k0 += 16) {  // 16 radial sums per pass
+      float acc[16], bias = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+      for (int i = 0; i < n; ++i) {
+        const float a = Ag[(int64_t)(i0 + i) * y.co + c];
+        const float b = Bg ? Bg[(int64_t)(i0 + i) * y.co + c] : 0.f;
+        bias += a;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          if (k0 + k < y.nr) {
+            acc[k] += phi[i * y.nr + k0 + k] * a;
+            if (Bg) acc[k] += dphi[i * y.nr + k0 + k] * b;
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        if (k0 + k < y.nr) part[(int64_t)blockIdx.x * P + (k0 + k) * y.co + c] = acc[k];
+      if (k0 == 0) part[(int64_t)blockIdx.x * P + y.nr * y.co + c] = bias;
     }
-    part[(int64_t)blockIdx.x * P + pidx] = s;
   }
 }
 

@@ -101,7 +101,7 @@ struct Plan {
   // byte offsets
   int na = 1, ngv = 1;  // row-stacked operand sets (double backward uses 3 and 2)
   size_t status, counts, cursor, offsets, perm, rec, geo, D, gate, wst_hi, wst_lo, wtr_hi, wtr_lo,
-      a_hi, a_lo, V, gv_hi, gv_lo, Ga, Gg, h, dws, radp, omega,
+      a_hi, a_lo, V, gv_hi, gv_lo, Ga, Gg, h, dws, radp, irt, omega,
       dgate, tA, tB;
 };
 
@@ -151,6 +151,7 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
   p.geo = take(c, sizeof(float) * GEO * p.chunk);
   p.D = take(c, sizeof(float) * (size_t)y.dsz * p.chunk);
   p.gate = take(c, sizeof(float) * (size_t)y.co * p.chunk);
+  p.irt = take(c, sizeof(float) * 2 * IR_TERMS * (ir_table_entries(y.L) + 1));
   p.wst_hi = take(c, 2ull * y.WR * y.WK);
   p.wst_lo = take(c, 2ull * y.WR * y.WK * lo);
   p.wtr_hi = take(c, 2ull * y.WTR * y.WTK);
@@ -438,28 +439,34 @@ so2_status sort_edges(Ctx &c, const int64_t *ei, int key_row) {
   CKL();
   k_place<<<grid_for(P.E, 256), 256, 0, c.s>>>(keys, P.E, P.N, offsets, cursor, perm);
   CKL();
-  k_sort_segments<<<grid_for(P.N, 128), 128, 0, c.s>>>(offsets, P.N, perm);
+  k_sort_segments<<<warp_grid(static_cast<int>(P.N), 8), 256, 0, c.s>>>(offsets, P.N, perm);
   CKL();
   return SO2_OK;
 }
 
-so2_status pack_weights(Ctx &c, const void *w) {
+// Stacked weight planes (and, when the call needs them, their transposes).
+so2_status pack_weights(Ctx &c, const void *w, bool transposes) {
   const Plan &P = c.P;
   const Layout &y = P.y;
   __nv_bfloat16 *wh = at<__nv_bfloat16>(c.ws, P.wst_hi), *wl = P.split ? at<__nv_bfloat16>(c.ws, P.wst_lo) : nullptr;
   __nv_bfloat16 *th = at<__nv_bfloat16>(c.ws, P.wtr_hi), *tl = P.split ? at<__nv_bfloat16>(c.ws, P.wtr_lo) : nullptr;
   // zero padding first
   CK(cudaMemsetAsync(wh, 0, 2ull * y.WR * y.WK, c.s));
-  CK(cudaMemsetAsync(th, 0, 2ull * y.WTR * y.WTK, c.s));
   if (wl) CK(cudaMemsetAsync(wl, 0, 2ull * y.WR * y.WK, c.s));
-  if (tl) CK(cudaMemsetAsync(tl, 0, 2ull * y.WTR * y.WTK, c.s));
+  if (transposes) {
+    CK(cudaMemsetAsync(th, 0, 2ull * y.WTR * y.WTK, c.s));
+    if (tl) CK(cudaMemsetAsync(tl, 0, 2ull * y.WTR * y.WTK, c.s));
+  }
   dim3 grid(64, y.ng);
   BlockOffsets bo = block_offsets(y);
-  if (P.xbf16)
-    k_pack_weights<__nv_bfloat16><<<grid, 256, 0, c.s>>>(y, bo, static_cast<const __nv_bfloat16 *>(w), wh, wl, th, tl);
-  else
-    k_pack_weights<float><<<grid, 256, 0, c.s>>>(y, bo, static_cast<const float *>(w), wh, wl, th, tl);
-  CKL();
+  for (int t = 0; t < (transposes ? 2 : 1); ++t) {
+    __nv_bfloat16 *h = t ? th : wh, *l = t ? tl : wl;
+    if (P.xbf16)
+      k_pack_weights<__nv_bfloat16><<<grid, 256, 0, c.s>>>(y, bo, static_cast<const __nv_bfloat16 *>(w), t, h, l);
+    else
+      k_pack_weights<float><<<grid, 256, 0, c.s>>>(y, bo, static_cast<const float *>(w), t, h, l);
+    CKL();
+  }
   return SO2_OK;
 }
 
@@ -468,9 +475,17 @@ so2_status chunk_prep(Ctx &c, int64_t e0, int M, const int64_t *ei, const float 
                       so2conv_params prm) {
   const Plan &P = c.P;
   const int smem = 8 * (P.y.dsz + 16) * static_cast<int>(sizeof(float));
+  if (e0 == 0) {  // the recursion's term table, once per call
+    const int ne = ir_table_entries(P.y.L);
+    if (ne > 0) {
+      k_ir_table<<<(ne + 127) / 128, 128, 0, c.s>>>(P.y.L, at<float>(c.ws, P.irt));
+      CKL();
+    }
+  }
   k_edge_prep<<<warp_grid(M, 8), 256, smem, c.s>>>(P.y, at<int>(c.ws, P.perm), e0, M, ei, P.E, P.N,
                                                    key_row, ev, at<EdgeRec>(c.ws, P.rec),
                                                    at<float>(c.ws, P.geo), at<float>(c.ws, P.D),
+                                                   P.y.L >= 2 ? at<float>(c.ws, P.irt) : nullptr,
                                                    c.st);
   CKL();
   k_edge_gate<<<(M + GATE_EDGES - 1) / GATE_EDGES, 128, GATE_EDGES * P.y.nr * sizeof(float),
@@ -644,7 +659,7 @@ so2_status rad_grads(Ctx &c, int M, const float *Ag, const float *Bg, const floa
   const int nblk = (M + RAD_TILE - 1) / RAD_TILE;
   const int sm = 2 * RAD_TILE * y.nr * static_cast<int>(sizeof(float));
   if (!allow_smem(k_rad_partial, sm)) return SO2_ERR_CUDA;
-  k_rad_partial<<<nblk, 256, sm, c.s>>>(y, c.d->rbf_cutoff, M, at<float>(c.ws, P.geo), Ag, Bg,
+  k_rad_partial<<<nblk, 128, sm, c.s>>>(y, c.d->rbf_cutoff, M, at<float>(c.ws, P.geo), Ag, Bg,
                                         omega, at<float>(c.ws, P.radp));
   CKL();
   const int Pn = (y.nr + 1) * y.co;
@@ -698,7 +713,7 @@ so2_status so2conv_forward(const so2conv_desc *desc, int64_t N, int64_t E, const
   if (E == 0) return SO2_OK;
   if ((r = build_maps(c, false)) != SO2_OK) return r;
   if ((r = sort_edges(c, edge_index, 1)) != SO2_OK) return r;
-  if ((r = pack_weights(c, prm.w)) != SO2_OK) return r;
+  if ((r = pack_weights(c, prm.w, false)) != SO2_OK) return r;
   for (int64_t e0 = 0; e0 < E; e0 += P.chunk) {
     const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
     if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 1, prm)) != SO2_OK) return r;
@@ -746,7 +761,7 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
   const bool need_ga = grad_x || grad_edge_vec;
   if ((r = build_maps(c, true)) != SO2_OK) return r;
   if ((r = sort_edges(c, edge_index, 0)) != SO2_OK) return r;
-  if ((r = pack_weights(c, prm.w)) != SO2_OK) return r;
+  if ((r = pack_weights(c, prm.w, true)) != SO2_OK) return r;
   float *dws = at<float>(ws, P.dws);
   if (grad_w) CK(cudaMemsetAsync(dws, 0, 4ull * y.WR * y.WK, c.s));
   for (int64_t e0 = 0; e0 < E; e0 += P.chunk) {
@@ -869,7 +884,7 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
   const bool has_r = gg_edge_vec != nullptr, has_x = gg_x != nullptr;
   if (E == 0 || (!has_r && !has_x)) return SO2_OK;
   if ((r = build_maps(c, true)) != SO2_OK) return r;
-  if ((r = pack_weights(c, prm.w)) != SO2_OK) return r;
+  if ((r = pack_weights(c, prm.w, true)) != SO2_OK) return r;
   const Coef gate = arr(at<float>(ws, P.gate));
   const Coef dgate = arr(at<float>(ws, P.dgate));
   const float *omega = at<float>(ws, P.omega);

@@ -67,16 +67,32 @@ __device__ __forceinline__ bool make_frame(float rx, float ry, float rz, Frame &
   return true;
 }
 
-// Entry (m, n) of D^l (l >= 2) from D^1 (row-major 3x3, index (i+1)*3+(j+1))
-// and D^{l-1} (row-major (2l-1)^2): the Ivanic-Ruedenberg recursion.
-__device__ __forceinline__ float ir_entry(int l, int m, int n, const float *D1, const float *Dp) {
+// The Ivanic-Ruedenberg recursion writes entry (m, n) of D^l (l >= 2) as a
+// sum of at most IR_TERMS products coef * D^1[i] * D^{l-1}[j], with D^1
+// row-major 3x3 (index (a+1)*3+(b+1)) and D^{l-1} row-major (2l-1)^2.
+// ir_terms lists them (unused slots have coef 0 and indices 0).
+constexpr int IR_TERMS = 10;
+
+__host__ __device__ inline int ir_terms(int l, int m, int n, float *coef, int *i1, int *i2) {
   const int wp = 2 * l - 1;
-  auto r1 = [&](int i, int j) { return D1[(i + 1) * 3 + (j + 1)]; };
-  auto rp = [&](int a, int b) { return Dp[(a + l - 1) * wp + (b + l - 1)]; };
-  auto P = [&](int i, int a, int b) -> float {
-    if (b == -l) return r1(i, 1) * rp(a, -l + 1) + r1(i, -1) * rp(a, l - 1);
-    if (b == l) return r1(i, 1) * rp(a, l - 1) - r1(i, -1) * rp(a, -l + 1);
-    return r1(i, 0) * rp(a, b);
+  int nt = 0;
+  auto put = [&](float c, int i, int j, int a, int b) {
+    coef[nt] = c;
+    i1[nt] = (i + 1) * 3 + (j + 1);
+    i2[nt] = (a + l - 1) * wp + (b + l - 1);
+    ++nt;
+  };
+  // c * P(i, a, b)
+  auto P = [&](float c, int i, int a, int b) {
+    if (b == -l) {
+      put(c, i, 1, a, -l + 1);
+      put(c, i, -1, a, l - 1);
+    } else if (b == l) {
+      put(c, i, 1, a, l - 1);
+      put(-c, i, -1, a, -l + 1);
+    } else {
+      put(c, i, 0, a, b);
+    }
   };
   const int am = m < 0 ? -m : m;
   const int an = n < 0 ? -n : n;
@@ -88,34 +104,80 @@ __device__ __forceinline__ float ir_entry(int l, int m, int n, const float *D1, 
                   static_cast<float>(1 - 2 * dm0);
   const float wc = -0.5f * sqrtf(static_cast<float>((l - am - 1) * (l - am)) / den) *
                    static_cast<float>(1 - dm0);
-  float val = 0.f;
-  if (u != 0.f) val += u * P(0, m, n);
+  const float r2 = 1.41421356237f;
+  if (u != 0.f) P(u, 0, m, n);
   if (v != 0.f) {
-    float V;
     if (m == 0) {
-      V = P(1, 1, n) + P(-1, -1, n);
+      P(v, 1, 1, n);
+      P(v, -1, -1, n);
     } else if (m > 0) {
-      V = P(1, m - 1, n) * (m == 1 ? 1.41421356237f : 1.f) - (m == 1 ? 0.f : P(-1, -m + 1, n));
+      P(v * (m == 1 ? r2 : 1.f), 1, m - 1, n);
+      if (m != 1) P(-v, -1, -m + 1, n);
     } else {
-      V = (m == -1 ? 0.f : P(1, m + 1, n)) + P(-1, -m - 1, n) * (m == -1 ? 1.41421356237f : 1.f);
+      if (m != -1) P(v, 1, m + 1, n);
+      P(v * (m == -1 ? r2 : 1.f), -1, -m - 1, n);
     }
-    val += v * V;
   }
   if (wc != 0.f) {
-    float Wv;
-    if (m > 0)
-      Wv = P(1, m + 1, n) + P(-1, -m - 1, n);
-    else
-      Wv = P(1, m - 1, n) - P(-1, -m + 1, n);
-    val += wc * Wv;
+    if (m > 0) {
+      P(wc, 1, m + 1, n);
+      P(wc, -1, -m - 1, n);
+    } else {
+      P(wc, 1, m - 1, n);
+      P(-wc, -1, -m + 1, n);
+    }
   }
+  for (int t = nt; t < IR_TERMS; ++t) {
+    coef[t] = 0.f;
+    i1[t] = 0;
+    i2[t] = 0;
+  }
+  return nt;
+}
+
+// Entry (m, n) of D^l (l >= 2) evaluated directly from the term list.
+__device__ __forceinline__ float ir_entry(int l, int m, int n, const float *D1, const float *Dp) {
+  float c[IR_TERMS];
+  int a[IR_TERMS], b[IR_TERMS];
+  const int nt = ir_terms(l, m, n, c, a, b);
+  float val = 0.f;
+  for (int t = 0; t < nt; ++t) val += c[t] * D1[a[t]] * Dp[b[t]];
   return val;
+}
+
+// Number of tabulated entries for levels 2..lmax (entry index of (l, m, n)
+// is dblock_off(l) - dblock_off(2) + (m+l)(2l+1) + (n+l)).
+__host__ __device__ constexpr int ir_table_entries(int lmax) {
+  return lmax < 2 ? 0 : dblock_off(lmax + 1) - dblock_off(2);
+}
+
+// Table layout (structure of arrays, NE = ir_table_entries(lmax)):
+// coef[t * NE + e] floats, then idx[t * NE + e] ints with i1 | i2 << 8.
+__global__ void k_ir_table(int lmax, float *table) {
+  const int NE = ir_table_entries(lmax);
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= NE) return;
+  int l = 2;
+  while (l < lmax && e >= dblock_off(l + 1) - dblock_off(2)) ++l;
+  const int local = e - (dblock_off(l) - dblock_off(2));
+  const int w = 2 * l + 1;
+  float c[IR_TERMS];
+  int a[IR_TERMS], b[IR_TERMS];
+  ir_terms(l, local / w - l, local % w - l, c, a, b);
+  int *idx = reinterpret_cast<int *>(table + IR_TERMS * NE);
+  for (int t = 0; t < IR_TERMS; ++t) {
+    table[t * NE + e] = c[t];
+    idx[t * NE + e] = a[t] | (b[t] << 8);
+  }
 }
 
 // Full blocks D^0..D^lmax (each (2l+1)^2 row-major, concatenated) of the
 // rotation R, computed by one warp into D (shared memory): the lanes share
-// the entries of each level, levels one after another.
-__device__ inline void wigner_blocks_warp(const float *R, int lmax, float *D) {
+// the entries of each level, levels one after another.  With a term table
+// (k_ir_table) every entry is the same branch-free 10-term sum; without one
+// the terms are enumerated per entry.
+__device__ inline void wigner_blocks_warp(const float *R, int lmax, float *D,
+                                          const float *table = nullptr) {
   const int lane = threadIdx.x & 31;
   if (lane == 0) D[0] = 1.f;
   if (lmax >= 1 && lane < 9) {
@@ -130,7 +192,23 @@ __device__ inline void wigner_blocks_warp(const float *R, int lmax, float *D) {
     const float *Dp = D + dblock_off(l - 1);
     float *Dl = D + dblock_off(l);
     const int w = 2 * l + 1;
-    for (int idx = lane; idx < w * w; idx += 32) Dl[idx] = ir_entry(l, idx / w - l, idx % w - l, D1, Dp);
+    if (table) {
+      const int NE = ir_table_entries(lmax);
+      const int *tidx = reinterpret_cast<const int *>(table + IR_TERMS * NE);
+      const int base = dblock_off(l) - dblock_off(2);
+      for (int idx = lane; idx < w * w; idx += 32) {
+        float val = 0.f;
+#pragma unroll
+        for (int t = 0; t < IR_TERMS; ++t) {
+          const int pk = __ldg(tidx + t * NE + base + idx);
+          val += __ldg(table + t * NE + base + idx) * D1[pk & 0xff] * Dp[pk >> 8];
+        }
+        Dl[idx] = val;
+      }
+    } else {
+      for (int idx = lane; idx < w * w; idx += 32)
+        Dl[idx] = ir_entry(l, idx / w - l, idx % w - l, D1, Dp);
+    }
     __syncwarp();
   }
 }
