@@ -57,6 +57,36 @@ def mixing_flops_per_edge(L, M, ci, co):
     return f
 
 
+def kernel_sources_sha256():
+    """Hash of the CUDA sources and the C header, to tell whether recorded
+    counters still describe the kernels that are built now."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "so_edge_convolution_b200", "csrc")
+    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    for path in files + [os.path.join(ROOT, "include", "so2conv.h")]:
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def kernel_traffic(config):
+    """DRAM bytes (read + write) per launch of the mixing kernel, averaged over
+    the launches of one step, from the ncu record committed for this workload;
+    None when there is none or the kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"gemm_tc_{config}_traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("sources_sha256") != kernel_sources_sha256():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -298,20 +328,13 @@ def run_ours(args, world, rank, local):
     # ---- roofline of the dominant kernel (the tcgen05 mixing GEMM) ----
     pk, src = peaks()
     fpe = mixing_flops_per_edge(p.lmax, p.mmax, p.c_in, p.c_out)
-    n_gemm = sum(v[0] for v in prof.values())
-    gemm_ms = sum(v[1] for v in prof.values())
+    n_gemm = sum(prof[k][0] for k in B.TENSOR_KINDS)
+    gemm_ms = sum(prof[k][1] for k in B.TENSOR_KINDS)
     alg_flops = float(n_products) * fpe * E * args.steps
     achieved = alg_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
     tf32_ratio = 1.0 if bf16 else 1.1 / 2.25  # nominal dense TF32 / BF16 on B200
     peak_tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * tf32_ratio
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "gemm_tc_esen_traffic.json")
-    if os.path.exists(tpath):
-        try:
-            with open(tpath) as f:
-                traffic = json.load(f).get("dram_bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = kernel_traffic(args.config)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                 "frac": (achieved / peak_tf) if achieved else None, "traffic": traffic,
                 "kernel": ("k_gemm_tc (bf16, f32 accumulate)" if bf16 else
@@ -322,6 +345,17 @@ def run_ours(args, world, rank, local):
                 "gemm_launches_per_step": n_gemm / args.steps,
                 "gemm_ms_per_step": gemm_ms / args.steps,
                 "step_roofline_frac": (alg_flops / (total_ms * 1e-3) / 1e12) / peak_tf}
+    # where the step's time goes: CUDA events around every launch group, in a
+    # few extra steps after the timed ones (so they add nothing to its time)
+    n_bd = 3
+    torch.cuda.synchronize()
+    B.profile_enable(True, all_kinds=True)
+    for _ in range(n_bd):
+        flush.zero_()
+        step(d)
+    torch.cuda.synchronize()
+    B.profile_enable(False)
+    breakdown = {B.PROFILE_KINDS[k]: round(v[1] / n_bd, 4) for k, v in B.profile_read().items()}
 
     # ---- end to end through the C ABI from pinned host buffers ----
     outs_host = None
@@ -366,7 +400,7 @@ def run_ours(args, world, rank, local):
                            "l2": "flushed between timed steps (256 MB write)",
                            "parallelism": f"replicas x{world}" if world > 1 else "single"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches, "clocks": clk}
+                "gpu_launches": launches, "clocks": clk, "breakdown_ms_per_step": breakdown}
         print(json.dumps(line), flush=True)
 
 

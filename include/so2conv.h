@@ -181,14 +181,21 @@ so2_status so2conv_forward_noalloc(const so2conv_desc *desc, int64_t n_nodes,
  * points, all devices).  A plain counter, not thread safe. */
 long long so2conv_launch_count(void);
 
-/* Live timing of the tensor-core launches.  so2conv_profile_enable(1) clears
+/* Live timing of the library's launches.  so2conv_profile_enable(1) clears
  * the record and starts recording a pair of CUDA events around every
- * tensor-core launch, on the stream it is launched on; (0) stops recording
- * and keeps the record for so2conv_profile_read.
+ * tensor-core launch, on the stream it is launched on; (2) does the same and
+ * also brackets each group of CUDA-core launches; (0) stops recording and
+ * keeps the record for so2conv_profile_read.
  * so2conv_profile_read waits for the recorded events and returns, for one
- * kind (0: products with the stacked weights, 1: with their transposes,
- * 2: weight-gradient products), the number of launches and their summed
- * duration in milliseconds.  Process-wide state, not thread safe. */
+ * kind, the number of recorded ranges and their summed duration in
+ * milliseconds.  Kinds (SO2_PROFILE_KINDS of them): 0 products with the
+ * stacked weights, 1 products with their transposes, 2 weight-gradient
+ * products (0-2: the tcgen05 kernel, one range per launch), 3 rotation on
+ * gather, 4 edge preparation (sort, records, frames, Wigner-D, gates),
+ * 5 per-edge gradient terms, 6 radial-weight sums, 7 weight packing and
+ * unpacking and the node-side scatter.  Process-wide state, not thread
+ * safe. */
+#define SO2_PROFILE_KINDS 8
 void so2conv_profile_enable(int on);
 so2_status so2conv_profile_read(int kind, int *n_launches, double *total_ms);
 

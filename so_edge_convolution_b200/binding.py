@@ -245,15 +245,21 @@ def launch_count():
     return int(load().so2conv_launch_count())
 
 
-def profile_enable(on=True):
-    load().so2conv_profile_enable(1 if on else 0)
+def profile_enable(on=True, all_kinds=False):
+    """Record CUDA events around the tensor-core launches (and, with
+    all_kinds, around every group of CUDA-core launches too)."""
+    load().so2conv_profile_enable((2 if all_kinds else 1) if on else 0)
 
 
-PROFILE_KINDS = {0: "mixing (x W^T)", 1: "mixing transposed (g W)", 2: "weight gradient"}
+PROFILE_KINDS = {0: "mixing (x W^T)", 1: "mixing transposed (g W)", 2: "weight gradient",
+                 3: "rotation on gather", 4: "edge preparation", 5: "edge gradient terms",
+                 6: "radial sums", 7: "weight packing and node scatter"}
+TENSOR_KINDS = (0, 1, 2)
 
 
 def profile_read():
-    """{kind: (launches, total_ms)} of the recorded tensor-core launches."""
+    """{kind: (ranges, total_ms)} of the recorded launches (kinds 0-2: one
+    range per tcgen05 launch; 3-7: groups of CUDA-core launches)."""
     lib = load()
     res = {}
     for k in PROFILE_KINDS:

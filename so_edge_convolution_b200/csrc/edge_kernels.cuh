@@ -13,6 +13,60 @@
 
 namespace so2 {
 
+// Resident 256-thread blocks per SM that the generic-degree (runtime lmax)
+// gather kernels are compiled for: caps their registers, since they are
+// latency bound and every level is instantiated in one function.
+#ifndef SO2_GATHER_MINB
+#define SO2_GATHER_MINB 2
+#endif
+// Rows of x / G whose loads may be in flight at once in the generic-degree
+// edge-term kernels (0: no limit).
+#ifndef SO2_ET_BATCH
+#define SO2_ET_BATCH 2
+#endif
+
+// Keeps the compiler from moving loads across this point.
+__device__ __forceinline__ void load_fence() { asm volatile("" ::: "memory"); }
+
+// Degree l as a compile-time value.
+template <int N>
+struct Lv {
+  static constexpr int value = N;
+};
+
+template <int I, int N, typename F>
+__device__ __forceinline__ void static_levels(F &f) {
+  if constexpr (I < N) {
+    f(Lv<I>{});
+    static_levels<I + 1, N>(f);
+  }
+}
+
+// f(Lv<l>{}) for l = 0..L.  LC >= 0 (then L = LC): every level inlined in
+// sequence, so loads of one level can be scheduled early in the previous
+// one.  LC = -1: a runtime loop whose body switches to the level's
+// compile-time instance, so no level keeps registers live in another.
+template <int LC, typename F>
+__device__ __forceinline__ void each_level(int L, F &&f) {
+  if constexpr (LC >= 0) {
+    static_levels<0, LC + 1>(f);
+  } else {
+#pragma unroll 1
+    for (int l = 0; l <= L; ++l) {
+      switch (l) {
+        case 0: f(Lv<0>{}); break;
+        case 1: f(Lv<1>{}); break;
+        case 2: f(Lv<2>{}); break;
+        case 3: f(Lv<3>{}); break;
+        case 4: f(Lv<4>{}); break;
+        case 5: f(Lv<5>{}); break;
+        default: f(Lv<6>{}); break;
+      }
+    }
+  }
+}
+static_assert(LMAX_SUPPORTED == 6, "each_level instantiates degrees 0..6");
+
 // ---------------------------------------------------------------------------
 // Graph preparation: stable counting sort of edges by one endpoint.
 // ---------------------------------------------------------------------------
@@ -220,6 +274,14 @@ __device__ __forceinline__ float2 coef2(const Coef &k, int64_t i, int C, int c) 
 // Omega = w_x J_x + w_y J_y with (w_x, w_y) = omega[i][0..1].  With B absent
 // this is plain rotation on gather (A = 1) or gated rotation (A = g).
 __device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+// Read-only (non-coherent) loads, free to move across the kernel's stores.
+__device__ __forceinline__ float4 load4_ro(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+__device__ __forceinline__ float4 load4_ro(const __nv_bfloat16 *p) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
 __device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
   const uint2 u = *reinterpret_cast<const uint2 *>(p);
   const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
@@ -258,7 +320,7 @@ __device__ __forceinline__ void stage_d(const float *De, int dsz, float *sD) {
 // LC >= 0 fixes lmax at compile time (loops fully unrolled); -1 reads it
 // from the layout.
 template <typename TX, int MM, int LC = -1>
-__global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec,
+__global__ void __launch_bounds__(256, LC >= 0 ? 2 : SO2_GATHER_MINB) k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec,
                                 const float *__restrict__ D, const TX *__restrict__ X, int side,
                                 int use_src, Coef A, Coef B, const float *__restrict__ omega,
                                 __nv_bfloat16 *__restrict__ out_hi, __nv_bfloat16 *__restrict__ out_lo,
@@ -284,51 +346,102 @@ __global__ void k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec
       wx = omega[4 * (int64_t)i];
       wy = omega[4 * (int64_t)i + 1];
     }
-    for (int c = 4 * lane; c < C; c += 128) {
-      const float4 ca = coef4(A, i, C, c), cb = coef4(B, i, C, c);
-      const int L = LC >= 0 ? LC : y.L;
+    // Two schedules, each chosen by measurement for the degrees it serves:
+    // lmax 6 runs every level inlined with plain loads; the others run
+    // per-level bodies with read-only loads the compiler may hoist.
+    if constexpr (LC == 6) {
+      for (int c = 4 * lane; c < C; c += 128) {
+        const float4 ca = coef4(A, i, C, c), cb = coef4(B, i, C, c);
 #pragma unroll
-      for (int l = 0; l <= L; ++l) {
-        float4 a[2 * W + 1];
+        for (int l = 0; l <= LC; ++l) {
+          float4 a[2 * W + 1];
 #pragma unroll
-        for (int k = 0; k < 2 * W + 1; ++k) a[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float *Dl = sD + dblock_off(l);
-        const int w = 2 * l + 1;
-        const int top = wide ? W : MM;
+          for (int k = 0; k < 2 * W + 1; ++k) a[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          const float *Dl = sD + dblock_off(l);
+          const int w = 2 * l + 1;
+          const int top = wide ? W : MM;
 #pragma unroll
-        for (int mp = -l; mp <= l; ++mp) {
-          const float4 xv = load4(Xn + (l * l + l + mp) * C + c);
+          for (int mp = -l; mp <= l; ++mp) {
+            const float4 xv = load4(Xn + (l * l + l + mp) * C + c);
 #pragma unroll
-          for (int m = -W; m <= W; ++m) {
-            if (m < -l || m > l || m < -top || m > top) continue;
-            const float dv = Dl[(m + l) * w + mp + l];
-            a[m + W].x += dv * xv.x;
-            a[m + W].y += dv * xv.y;
-            a[m + W].z += dv * xv.z;
-            a[m + W].w += dv * xv.w;
+            for (int m = -W; m <= W; ++m) {
+              if (m < -l || m > l || m < -top || m > top) continue;
+              const float dv = Dl[(m + l) * w + mp + l];
+              a[m + W].x += dv * xv.x;
+              a[m + W].y += dv * xv.y;
+              a[m + W].z += dv * xv.z;
+              a[m + W].w += dv * xv.w;
+            }
+          }
+#pragma unroll
+          for (int m = -MM; m <= MM; ++m) {
+            if (m < -l || m > l) continue;
+            int g, j;
+            lm_group_row(y, l, m, g, j);
+            const int col = col_off[g] + j * C + c;
+            float4 o = make_float4(ca.x * a[m + W].x, ca.y * a[m + W].y, ca.z * a[m + W].z,
+                                   ca.w * a[m + W].w);
+            if (wide) {
+              float jx, jy;
+              gen_xy(l, m, [&](int q) { return a[q + W].x; }, jx, jy);
+              o.x += cb.x * (wx * jx + wy * jy);
+              gen_xy(l, m, [&](int q) { return a[q + W].y; }, jx, jy);
+              o.y += cb.y * (wx * jx + wy * jy);
+              gen_xy(l, m, [&](int q) { return a[q + W].z; }, jx, jy);
+              o.z += cb.z * (wx * jx + wy * jy);
+              gen_xy(l, m, [&](int q) { return a[q + W].w; }, jx, jy);
+              o.w += cb.w * (wx * jx + wy * jy);
+            }
+            store_split4(oh + col, ol ? ol + col : nullptr, o);
           }
         }
+      }
+    } else {
+      for (int c = 4 * lane; c < C; c += 128) {
+        const float4 ca = coef4(A, i, C, c), cb = coef4(B, i, C, c);
+        each_level<LC>(y.L, [&](auto lv) {
+          constexpr int l = decltype(lv)::value;
+          constexpr int w = 2 * l + 1;
+          constexpr int mlo = -(W < l ? W : l), mhi = (W < l ? W : l);
+          float4 a[2 * W + 1];
 #pragma unroll
-        for (int m = -MM; m <= MM; ++m) {
-          if (m < -l || m > l) continue;
-          int g, j;
-          lm_group_row(y, l, m, g, j);
-          const int col = col_off[g] + j * C + c;
-          float4 o = make_float4(ca.x * a[m + W].x, ca.y * a[m + W].y, ca.z * a[m + W].z,
-                                 ca.w * a[m + W].w);
-          if (wide) {
-            float jx, jy;
-            gen_xy(l, m, [&](int q) { return a[q + W].x; }, jx, jy);
-            o.x += cb.x * (wx * jx + wy * jy);
-            gen_xy(l, m, [&](int q) { return a[q + W].y; }, jx, jy);
-            o.y += cb.y * (wx * jx + wy * jy);
-            gen_xy(l, m, [&](int q) { return a[q + W].z; }, jx, jy);
-            o.z += cb.z * (wx * jx + wy * jy);
-            gen_xy(l, m, [&](int q) { return a[q + W].w; }, jx, jy);
-            o.w += cb.w * (wx * jx + wy * jy);
+          for (int k = 0; k < 2 * W + 1; ++k) a[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          const float *Dl = sD + dblock_off(l);
+          const int top = wide ? W : MM;
+#pragma unroll
+          for (int mp = -l; mp <= l; ++mp) {
+            const float4 xv = load4_ro(Xn + (l * l + l + mp) * C + c);
+#pragma unroll
+            for (int m = mlo; m <= mhi; ++m) {
+              if (m < -top || m > top) continue;
+              const float dv = Dl[(m + l) * w + mp + l];
+              a[m + W].x += dv * xv.x;
+              a[m + W].y += dv * xv.y;
+              a[m + W].z += dv * xv.z;
+              a[m + W].w += dv * xv.w;
+            }
           }
-          store_split4(oh + col, ol ? ol + col : nullptr, o);
-        }
+#pragma unroll
+          for (int m = -(MM < l ? MM : l); m <= (MM < l ? MM : l); ++m) {
+            int g, j;
+            lm_group_row(y, l, m, g, j);
+            const int col = col_off[g] + j * C + c;
+            float4 o = make_float4(ca.x * a[m + W].x, ca.y * a[m + W].y, ca.z * a[m + W].z,
+                                   ca.w * a[m + W].w);
+            if (wide) {
+              float jx, jy;
+              gen_xy(l, m, [&](int q) { return a[q + W].x; }, jx, jy);
+              o.x += cb.x * (wx * jx + wy * jy);
+              gen_xy(l, m, [&](int q) { return a[q + W].y; }, jx, jy);
+              o.y += cb.y * (wx * jx + wy * jy);
+              gen_xy(l, m, [&](int q) { return a[q + W].z; }, jx, jy);
+              o.z += cb.z * (wx * jx + wy * jy);
+              gen_xy(l, m, [&](int q) { return a[q + W].w; }, jx, jy);
+              o.w += cb.w * (wx * jx + wy * jy);
+            }
+            store_split4(oh + col, ol ? ol + col : nullptr, o);
+          }
+        });
       }
     }
     for (int g = 0; g < y.ng; ++g) {
@@ -543,7 +656,7 @@ __global__ void k_unstack_grad(Layout y, BlockOffsets bo, const float *__restric
 // PART: 3 = both sides in one pass; 1 = output side only (writes Gg and h);
 // 2 = input side only (adds its share to h).
 template <typename TX, int MM, int LC = -1, int PART = 3>
-__global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
+__global__ void __launch_bounds__(256, LC >= 0 ? 1 : SO2_GATHER_MINB) k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
                              const float *__restrict__ D, const float *__restrict__ gate,
                              const float *__restrict__ G, const TX *__restrict__ X,
                              const float *__restrict__ V, const float *__restrict__ Ga,
@@ -563,19 +676,20 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
     for (int c = 4 * lane; (PART & 1) && c < y.co; c += 128) {
       const float4 gv = load4(gate + (int64_t)i * y.co + c);
       float4 gg = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int l = 0; l <= (LC >= 0 ? LC : y.L); ++l) {
+      each_level<LC>(y.L, [&](auto lv) {
+        constexpr int l = decltype(lv)::value;
+        constexpr int w = 2 * l + 1;
+        constexpr int mw = W < l ? W : l, mm = MM < l ? MM : l;
         float4 b[2 * W + 1];
 #pragma unroll
         for (int k = 0; k < 2 * W + 1; ++k) b[k] = make_float4(0.f, 0.f, 0.f, 0.f);
         const float *Dl = sD + dblock_off(l);
-        const int w = 2 * l + 1;
 #pragma unroll
         for (int mp = -l; mp <= l; ++mp) {
+          if (LC < 0 && SO2_ET_BATCH > 0 && mp > -l && (mp + l) % SO2_ET_BATCH == 0) load_fence();
           const float4 gx = load4(Gn + (l * l + l + mp) * y.co + c);
 #pragma unroll
-          for (int m = -W; m <= W; ++m) {
-            if (m < -l || m > l) continue;
+          for (int m = -mw; m <= mw; ++m) {
             const float dv = Dl[(m + l) * w + mp + l];
             b[m + W].x += dv * gx.x;
             b[m + W].y += dv * gx.y;
@@ -584,8 +698,7 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
           }
         }
 #pragma unroll
-        for (int m = -MM; m <= MM; ++m) {
-          if (m < -l || m > l) continue;
+        for (int m = -mm; m <= mm; ++m) {
           int g, j;
           lm_group_row(y, l, m, g, j);
           const float4 v = load4(Vi + y.kout_off[g] + j * y.co + c);
@@ -607,26 +720,27 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
           hx += gv.w * v.w * jx;
           hy += gv.w * v.w * jy;
         }
-      }
+      });
       *reinterpret_cast<float4 *>(Gg + (int64_t)i * y.co + c) = gg;
     }
     // input side
     const TX *Xn = X + (int64_t)r.src * y.S * y.ci;
     const float *Gai = Ga + (int64_t)i * y.KA;
     for (int c = 4 * lane; (PART & 2) && c < y.ci; c += 128) {
-#pragma unroll
-      for (int l = 0; l <= (LC >= 0 ? LC : y.L); ++l) {
+      each_level<LC>(y.L, [&](auto lv) {
+        constexpr int l = decltype(lv)::value;
+        constexpr int w = 2 * l + 1;
+        constexpr int mw = W < l ? W : l, mm = MM < l ? MM : l;
         float4 b[2 * W + 1];
 #pragma unroll
         for (int k = 0; k < 2 * W + 1; ++k) b[k] = make_float4(0.f, 0.f, 0.f, 0.f);
         const float *Dl = sD + dblock_off(l);
-        const int w = 2 * l + 1;
 #pragma unroll
         for (int mp = -l; mp <= l; ++mp) {
+          if (LC < 0 && SO2_ET_BATCH > 0 && mp > -l && (mp + l) % SO2_ET_BATCH == 0) load_fence();
           const float4 xv = load4(Xn + (l * l + l + mp) * y.ci + c);
 #pragma unroll
-          for (int m = -W; m <= W; ++m) {
-            if (m < -l || m > l) continue;
+          for (int m = -mw; m <= mw; ++m) {
             const float dv = Dl[(m + l) * w + mp + l];
             b[m + W].x += dv * xv.x;
             b[m + W].y += dv * xv.y;
@@ -635,8 +749,7 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
           }
         }
 #pragma unroll
-        for (int m = -MM; m <= MM; ++m) {
-          if (m < -l || m > l) continue;
+        for (int m = -mm; m <= mm; ++m) {
           int g, j;
           lm_group_row(y, l, m, g, j);
           const float4 ga = load4(Gai + y.kin_off[g] + j * y.ci + c);
@@ -654,7 +767,7 @@ __global__ void k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
           hx += ga.w * jx;
           hy += ga.w * jy;
         }
-      }
+      });
     }
     for (int o = 16; o > 0; o >>= 1) {
       hx += __shfl_xor_sync(0xffffffffu, hx, o);

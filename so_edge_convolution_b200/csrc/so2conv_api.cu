@@ -219,12 +219,16 @@ long long g_launches = 0;
     if (cudaPeekAtLastError() != cudaSuccess) return SO2_ERR_CUDA; \
   } while (0)
 
-// Optional CUDA-event timing of the tensor-core launches, by kind.
-constexpr int PROF_KINDS = 3;  // 0: products with W, 1: with W^T, 2: weight gradients
+// Optional CUDA-event timing of the launches, by kind: 0 products with W,
+// 1 with W^T, 2 weight gradients (the tensor-core kinds), 3 rotation on
+// gather, 4 edge preparation (sort, records, frames, Wigner-D, gates),
+// 5 per-edge gradient terms, 6 radial-weight sums, 7 weight packing and
+// node-side scatter.
+constexpr int PROF_KINDS = 8;
 struct Prof {
-  bool on = false;
+  int on = 0;  // 0 off, 1 tensor-core launches, 2 every kind
   std::vector<cudaEvent_t> ev[PROF_KINDS];  // start/stop pairs
-  int used[PROF_KINDS] = {0, 0, 0};
+  int used[PROF_KINDS] = {};
 };
 Prof g_prof;
 
@@ -237,6 +241,21 @@ cudaEvent_t prof_event(int kind) {
   }
   return P.ev[kind][P.used[kind]++];
 }
+
+// Records a start/stop event pair around the launches of its lifetime.
+struct ProfScope {
+  cudaEvent_t e1 = nullptr;
+  cudaStream_t s;
+  ProfScope(int kind, cudaStream_t s_) : s(s_) {
+    if (g_prof.on < 2) return;
+    cudaEvent_t e0 = prof_event(kind);
+    e1 = prof_event(kind);
+    if (e0) cudaEventRecord(e0, s);
+  }
+  ~ProfScope() {
+    if (e1) cudaEventRecord(e1, s);
+  }
+};
 
 int grid_for(int64_t n, int block) {
   int64_t g = (n + block - 1) / block;
@@ -430,6 +449,7 @@ so2_status sort_edges(Ctx &c, const int64_t *ei, int key_row) {
   const Plan &P = c.P;
   int *counts = at<int>(c.ws, P.counts), *cursor = at<int>(c.ws, P.cursor);
   int *offsets = at<int>(c.ws, P.offsets), *perm = at<int>(c.ws, P.perm);
+  ProfScope ps(4, c.s);
   CK(cudaMemsetAsync(counts, 0, sizeof(int) * (P.N + 1), c.s));
   CK(cudaMemsetAsync(cursor, 0, sizeof(int) * (P.N + 1), c.s));
   const int64_t *keys = ei + key_row * P.E;
@@ -450,6 +470,7 @@ so2_status pack_weights(Ctx &c, const void *w, bool transposes) {
   const Layout &y = P.y;
   __nv_bfloat16 *wh = at<__nv_bfloat16>(c.ws, P.wst_hi), *wl = P.split ? at<__nv_bfloat16>(c.ws, P.wst_lo) : nullptr;
   __nv_bfloat16 *th = at<__nv_bfloat16>(c.ws, P.wtr_hi), *tl = P.split ? at<__nv_bfloat16>(c.ws, P.wtr_lo) : nullptr;
+  ProfScope ps(7, c.s);
   // zero padding first
   CK(cudaMemsetAsync(wh, 0, 2ull * y.WR * y.WK, c.s));
   if (wl) CK(cudaMemsetAsync(wl, 0, 2ull * y.WR * y.WK, c.s));
@@ -475,6 +496,7 @@ so2_status chunk_prep(Ctx &c, int64_t e0, int M, const int64_t *ei, const float 
                       so2conv_params prm) {
   const Plan &P = c.P;
   const int smem = 8 * (P.y.dsz + 16) * static_cast<int>(sizeof(float));
+  ProfScope ps(4, c.s);
   if (e0 == 0) {  // the recursion's term table, once per call
     const int ne = ir_table_entries(P.y.L);
     if (ne > 0) {
@@ -503,6 +525,7 @@ so2_status rotate(Ctx &c, int M, const void *X, bool xbf16, int side, int use_sr
   const EdgeRec *rec = at<EdgeRec>(c.ws, P.rec);
   const float *D = at<float>(c.ws, P.D);
   const int dsm = 8 * P.y.dsz * static_cast<int>(sizeof(float));  // staged D per warp
+  ProfScope ps(3, c.s);
   if (xbf16) {
     DISPATCH_LM(P.y.L, P.y.mmax, (k_rotate_gather<__nv_bfloat16, MM, LC><<<warp_grid(M, 8), 256, dsm, c.s>>>(
                                P.y, M, rec, D, static_cast<const __nv_bfloat16 *>(X), side,
@@ -636,6 +659,7 @@ so2_status scatter(Ctx &c, int64_t e0, int M, const ScatterTerms &t, int side,
   const int *off = at<int>(c.ws, P.offsets);
   const float *D = at<float>(c.ws, P.D);
   bool ok = true;
+  ProfScope ps(7, c.s);
   DISPATCH_MM(y.mmax, ok = allow_smem(k_scatter_nodes<MM>, smem);
               if (ok) k_scatter_nodes<MM><<<grid_for(M, 1), threads, smem, c.s>>>(
                   y, e0, M, rec, off, D, t, side, omega, out));
@@ -659,6 +683,7 @@ so2_status rad_grads(Ctx &c, int M, const float *Ag, const float *Bg, const floa
   const int nblk = (M + RAD_TILE - 1) / RAD_TILE;
   const int sm = 2 * RAD_TILE * y.nr * static_cast<int>(sizeof(float));
   if (!allow_smem(k_rad_partial, sm)) return SO2_ERR_CUDA;
+  ProfScope ps(6, c.s);
   k_rad_partial<<<nblk, 128, sm, c.s>>>(y, c.d->rbf_cutoff, M, at<float>(c.ws, P.geo), Ag, Bg,
                                         omega, at<float>(c.ws, P.radp));
   CKL();
@@ -789,6 +814,7 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
       return r;
     if (need_v) {
       {
+        ProfScope ps(5, c.s);
         const int sm = 8 * y.dsz * 4;
         const int g = warp_grid(M, 8);
         EdgeRec *rec = at<EdgeRec>(ws, P.rec);
@@ -797,31 +823,26 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
         if (P.xbf16) {
           const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
           DISPATCH_LM(y.L, y.mmax,
-                      if (LC >= 0 && LC <= 4) {  // lmax 6 unrolled spills
-                        k_edge_terms<__nv_bfloat16, MM, LC, 1><<<g, 256, sm, c.s>>>(
-                            y, M, rec, Dp, gate, grad_out, xb, Vp, Gap, Ggp, hp);
-                        k_edge_terms<__nv_bfloat16, MM, LC, 2><<<g, 256, sm, c.s>>>(
-                            y, M, rec, Dp, gate, grad_out, xb, Vp, Gap, Ggp, hp);
-                      } else {
-                        k_edge_terms<__nv_bfloat16, MM><<<g, 256, sm, c.s>>>(
-                            y, M, rec, Dp, gate, grad_out, xb, Vp, Gap, Ggp, hp);
-                      });
+                      // all levels inlined spills at lmax 6: runtime-degree kernel there
+                      constexpr int LE = (LC >= 0 && LC <= 4) ? LC : -1;
+                      k_edge_terms<__nv_bfloat16, MM, LE, 1><<<g, 256, sm, c.s>>>(
+                          y, M, rec, Dp, gate, grad_out, xb, Vp, Gap, Ggp, hp);
+                      k_edge_terms<__nv_bfloat16, MM, LE, 2><<<g, 256, sm, c.s>>>(
+                          y, M, rec, Dp, gate, grad_out, xb, Vp, Gap, Ggp, hp););
         } else {
           const float *xf = static_cast<const float *>(x);
           DISPATCH_LM(y.L, y.mmax,
-                      if (LC >= 0 && LC <= 4) {  // lmax 6 unrolled spills
-                        k_edge_terms<float, MM, LC, 1><<<g, 256, sm, c.s>>>(
-                            y, M, rec, Dp, gate, grad_out, xf, Vp, Gap, Ggp, hp);
-                        k_edge_terms<float, MM, LC, 2><<<g, 256, sm, c.s>>>(
-                            y, M, rec, Dp, gate, grad_out, xf, Vp, Gap, Ggp, hp);
-                      } else {
-                        k_edge_terms<float, MM><<<g, 256, sm, c.s>>>(
-                            y, M, rec, Dp, gate, grad_out, xf, Vp, Gap, Ggp, hp);
-                      });
+                      // all levels inlined spills at lmax 6: runtime-degree kernel there
+                      constexpr int LE = (LC >= 0 && LC <= 4) ? LC : -1;
+                      k_edge_terms<float, MM, LE, 1><<<g, 256, sm, c.s>>>(
+                          y, M, rec, Dp, gate, grad_out, xf, Vp, Gap, Ggp, hp);
+                      k_edge_terms<float, MM, LE, 2><<<g, 256, sm, c.s>>>(
+                          y, M, rec, Dp, gate, grad_out, xf, Vp, Gap, Ggp, hp););
         }
       }
       CKL();
       if (grad_edge_vec) {
+        ProfScope ps(5, c.s);
         k_edge_final<<<warp_grid(M, 8), 256, 0, c.s>>>(y, desc->rbf_cutoff, M,
                                                         at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo),
                                                         at<float>(ws, P.Gg), at<float>(ws, P.h),
@@ -835,6 +856,7 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
     }
   }
   if (grad_w) {
+    ProfScope ps(7, c.s);
     k_unstack_grad<<<dim3(64, y.ng), 256, 0, c.s>>>(y, block_offsets(y), dws, grad_w);
     CKL();
   }
@@ -898,6 +920,7 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
     for (int64_t e0 = 0; e0 < E; e0 += ch) {
       const int M = static_cast<int>((E - e0) < ch ? (E - e0) : ch);
       if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 0, prm)) != SO2_OK) return r;
+      ProfScope ps(5, c.s);
       k_edge_omega<<<warp_grid(M, 8), 256, 0, c.s>>>(y, desc->rbf_cutoff, M,
                                                      at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo),
                                                      gg_edge_vec, prm.w_rad, at<float>(ws, P.omega),
@@ -924,6 +947,7 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
       const int M = static_cast<int>((E - e0) < ch ? (E - e0) : ch);
       if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 1, prm)) != SO2_OK) return r;
       if (has_r) {
+        ProfScope ps(5, c.s);
         k_edge_omega<<<warp_grid(M, 8), 256, 0, c.s>>>(
             y, desc->rbf_cutoff, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo), gg_edge_vec,
             prm.w_rad, at<float>(ws, P.omega), at<float>(ws, P.dgate));
@@ -956,11 +980,14 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
         if ((r = scatter(c, e0, M, t, 1, has_r ? omega : nullptr, d_grad_out)) != SO2_OK) return r;
       }
       if (d_w_rad || d_b_rad) {
-        DISPATCH_MM(y.mmax, (k_edge_terms2<MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+        {
+          ProfScope ps(5, c.s);
+          DISPATCH_MM(y.mmax, (k_edge_terms2<MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
                                 y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), grad_out,
                                 has_r ? omega : nullptr, V, has_r ? dV : nullptr,
                                 has_x ? Vt : nullptr, at<float>(ws, P.tA), at<float>(ws, P.tB))));
-        CKL();
+          CKL();
+        }
         if ((r = rad_grads(c, M, at<float>(ws, P.tA), has_r ? at<float>(ws, P.tB) : nullptr,
                            omega, d_w_rad, d_b_rad)) != SO2_OK)
           return r;
@@ -984,6 +1011,7 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
     }
   }
   if (d_w) {
+    ProfScope ps(7, c.s);
     k_unstack_grad<<<dim3(64, y.ng), 256, 0, c.s>>>(y, block_offsets(y), dws, d_w);
     CKL();
   }
@@ -1029,7 +1057,7 @@ so2_status so2conv_check(void *ws, so2_stream_t stream) {
 long long so2conv_launch_count(void) { return g_launches; }
 
 void so2conv_profile_enable(int on) {
-  g_prof.on = on != 0;
+  g_prof.on = on < 0 ? 0 : (on > 2 ? 2 : on);
   if (g_prof.on)
     for (int k = 0; k < PROF_KINDS; ++k) g_prof.used[k] = 0;
 }
