@@ -163,49 +163,51 @@ static_assert(sizeof(EdgeRec) == sizeof(int4), "EdgeRec is read as int4 by the f
 // Geometry record: d, r_hat[3], R[9] (row-major), 3 spare.
 constexpr int GEO = 16;
 
-// One warp per edge: lane 0 builds the record and frame, the warp runs the
-// Wigner-D recursion in its shared-memory slice (dsz floats) and copies it
-// out with coalesced stores.
-__global__ void k_edge_prep(Layout y, const int *__restrict__ perm, int64_t e0, int M,
-                            const int64_t *__restrict__ ei, int64_t E, int64_t N, int key_row,
-                            const float *__restrict__ edge_vec, EdgeRec *__restrict__ rec,
-                            float *__restrict__ geo, float *__restrict__ D,
-                            const float *__restrict__ ir_table, DevStatus *st) {
-  extern __shared__ float sDall[];  // [warps][dsz + 16]
-  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
-  float *sD = sDall + (threadIdx.x >> 5) * (y.dsz + 16);
-  float *sR = sD + y.dsz;  // 9 floats of R
-  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
-    __syncwarp();
-    if (lane == 0) {
-      const int e = perm[e0 + i];
-      int64_t s = ei[e], d = ei[E + e];
-      if (s < 0 || s >= N) s = 0;  // already reported by the sort
-      if (d < 0 || d >= N) d = 0;
-      EdgeRec r;
-      r.eid = e;
-      r.src = static_cast<int>(s);
-      r.dst = static_cast<int>(d);
-      r.key = key_row == 0 ? r.src : r.dst;
-      rec[i] = r;
-      Frame f;
-      if (!make_frame(edge_vec[3 * (int64_t)e], edge_vec[3 * (int64_t)e + 1],
-                      edge_vec[3 * (int64_t)e + 2], f))
-        raise_error(st, SO2_ERR_DEGENERATE, e);
-      float *gr = geo + (int64_t)i * GEO;
-      gr[0] = f.d;
-      gr[1] = f.rh[0];
-      gr[2] = f.rh[1];
-      gr[3] = f.rh[2];
-      for (int k = 0; k < 9; ++k) {
-        gr[4 + k] = f.R[k];
-        sR[k] = f.R[k];
-      }
-    }
-    __syncwarp();
-    wigner_blocks_warp(sR, y.L, sD, ir_table);
-    float *dst = D + (int64_t)i * y.dsz;
-    for (int k = lane; k < y.dsz; k += 32) dst[k] = sD[k];
+// One thread per edge: the record, the frame and the Wigner-D blocks, the
+// blocks into this warp's shared tile sD[k][33] (entry-major, so each
+// thread's writes and the copy-out below are free of bank conflicts), then
+// copied out edge by edge with coalesced stores.  Block = one warp.
+template <int L>
+__global__ void __launch_bounds__(32) k_edge_prep(int64_t e0, int M, const int *__restrict__ perm,
+                                                  const int64_t *__restrict__ ei, int64_t E,
+                                                  int64_t N, int key_row,
+                                                  const float *__restrict__ edge_vec,
+                                                  EdgeRec *__restrict__ rec, float *__restrict__ geo,
+                                                  float *__restrict__ D, DevStatus *st) {
+  constexpr int dsz = dsize(L);
+  extern __shared__ float sD[];  // [dsz][33]
+  const int lane = threadIdx.x;
+  const int i0 = blockIdx.x * 32;
+  const int i = i0 + lane;
+  if (i < M) {
+    const int e = perm[e0 + i];
+    int64_t s = ei[e], d = ei[E + e];
+    if (s < 0 || s >= N) s = 0;  // already reported by the sort
+    if (d < 0 || d >= N) d = 0;
+    EdgeRec r;
+    r.eid = e;
+    r.src = static_cast<int>(s);
+    r.dst = static_cast<int>(d);
+    r.key = key_row == 0 ? r.src : r.dst;
+    rec[i] = r;
+    Frame f;
+    if (!make_frame(edge_vec[3 * (int64_t)e], edge_vec[3 * (int64_t)e + 1],
+                    edge_vec[3 * (int64_t)e + 2], f))
+      raise_error(st, SO2_ERR_DEGENERATE, e);
+    float *gr = geo + (int64_t)i * GEO;
+    gr[0] = f.d;
+    gr[1] = f.rh[0];
+    gr[2] = f.rh[1];
+    gr[3] = f.rh[2];
+#pragma unroll
+    for (int k = 0; k < 9; ++k) gr[4 + k] = f.R[k];
+    wigner_blocks_thread<L>(f.R, sD + lane, 33);
+  }
+  __syncwarp();
+  const int nj = (M - i0) < 32 ? (M - i0) : 32;
+  for (int j = 0; j < nj; ++j) {
+    float *dst = D + (int64_t)(i0 + j) * dsz;
+    for (int k = lane; k < dsz; k += 32) dst[k] = sD[k * 33 + j];
   }
 }
 
@@ -1017,27 +1019,29 @@ __global__ void k_edge_terms2(Layout y, int M, const EdgeRec *__restrict__ rec,
   }
 }
 
-// Frames and full Wigner-D for inspection (the same recursion the op uses).
-__global__ void k_frames(int lmax, int64_t E, const float *__restrict__ edge_vec, float *__restrict__ Rout,
-                         float *__restrict__ Dout) {
-  extern __shared__ float sDall[];  // [warps][dsz + 16]
-  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
-  const int dsz = dsize(lmax);
-  float *sD = sDall + (threadIdx.x >> 5) * (dsz + 16);
-  float *sR = sD + dsz;
-  for (int64_t e = blockIdx.x * (int64_t)wpb + (threadIdx.x >> 5); e < E; e += (int64_t)gridDim.x * wpb) {
+// Frames and full Wigner-D for inspection, with the same per-thread code the
+// op uses.  Block = one warp, 32 edges.
+template <int L>
+__global__ void __launch_bounds__(32) k_frames(int64_t E, const float *__restrict__ edge_vec,
+                                               float *__restrict__ Rout, float *__restrict__ Dout) {
+  constexpr int dsz = dsize(L);
+  extern __shared__ float sD[];  // [dsz][33]
+  const int lane = threadIdx.x;
+  for (int64_t e0 = blockIdx.x * 32ll; e0 < E; e0 += gridDim.x * 32ll) {
+    const int64_t e = e0 + lane;
     __syncwarp();
-    if (lane == 0) {
+    if (e < E) {
       Frame f;
       make_frame(edge_vec[3 * e], edge_vec[3 * e + 1], edge_vec[3 * e + 2], f);
-      for (int k = 0; k < 9; ++k) sR[k] = f.R[k];
+      if (Rout)
+        for (int k = 0; k < 9; ++k) Rout[9 * e + k] = f.R[k];
+      wigner_blocks_thread<L>(f.R, sD + lane, 33);
     }
     __syncwarp();
-    if (Rout && lane < 9) Rout[9 * e + lane] = sR[lane];
-    if (Dout) {
-      wigner_blocks_warp(sR, lmax, sD);
-      for (int k = lane; k < dsz; k += 32) Dout[e * dsz + k] = sD[k];
-    }
+    if (!Dout) continue;
+    const int nj = (E - e0) < 32 ? static_cast<int>(E - e0) : 32;
+    for (int j = 0; j < nj; ++j)
+      for (int k = lane; k < dsz; k += 32) Dout[(e0 + j) * dsz + k] = sD[k * 33 + j];
   }
 }
 

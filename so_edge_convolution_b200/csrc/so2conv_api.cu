@@ -101,7 +101,7 @@ struct Plan {
   // byte offsets
   int na = 1, ngv = 1;  // row-stacked operand sets (double backward uses 3 and 2)
   size_t status, counts, cursor, offsets, perm, rec, geo, D, gate, wst_hi, wst_lo, wtr_hi, wtr_lo,
-      a_hi, a_lo, V, gv_hi, gv_lo, Ga, Gg, h, dws, radp, irt, omega,
+      a_hi, a_lo, V, gv_hi, gv_lo, Ga, Gg, h, dws, radp, omega,
       dgate, tA, tB;
 };
 
@@ -151,7 +151,6 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
   p.geo = take(c, sizeof(float) * GEO * p.chunk);
   p.D = take(c, sizeof(float) * (size_t)y.dsz * p.chunk);
   p.gate = take(c, sizeof(float) * (size_t)y.co * p.chunk);
-  p.irt = take(c, sizeof(float) * 2 * IR_TERMS * (ir_table_entries(y.L) + 1));
   p.wst_hi = take(c, 2ull * y.WR * y.WK);
   p.wst_lo = take(c, 2ull * y.WR * y.WK * lo);
   p.wtr_hi = take(c, 2ull * y.WTR * y.WTK);
@@ -495,20 +494,14 @@ so2_status pack_weights(Ctx &c, const void *w, bool transposes) {
 so2_status chunk_prep(Ctx &c, int64_t e0, int M, const int64_t *ei, const float *ev, int key_row,
                       so2conv_params prm) {
   const Plan &P = c.P;
-  const int smem = 8 * (P.y.dsz + 16) * static_cast<int>(sizeof(float));
   ProfScope ps(4, c.s);
-  if (e0 == 0) {  // the recursion's term table, once per call
-    const int ne = ir_table_entries(P.y.L);
-    if (ne > 0) {
-      k_ir_table<<<(ne + 127) / 128, 128, 0, c.s>>>(P.y.L, at<float>(c.ws, P.irt));
-      CKL();
-    }
-  }
-  k_edge_prep<<<warp_grid(M, 8), 256, smem, c.s>>>(P.y, at<int>(c.ws, P.perm), e0, M, ei, P.E, P.N,
-                                                   key_row, ev, at<EdgeRec>(c.ws, P.rec),
-                                                   at<float>(c.ws, P.geo), at<float>(c.ws, P.D),
-                                                   P.y.L >= 2 ? at<float>(c.ws, P.irt) : nullptr,
-                                                   c.st);
+  const int smem = P.y.dsz * 33 * static_cast<int>(sizeof(float));
+  bool ok = true;
+  SO2_DISPATCH_L(P.y.L, ok = allow_smem(k_edge_prep<L>, smem);
+                 if (ok) k_edge_prep<L><<<(M + 31) / 32, 32, smem, c.s>>>(
+                     e0, M, at<int>(c.ws, P.perm), ei, P.E, P.N, key_row, ev,
+                     at<EdgeRec>(c.ws, P.rec), at<float>(c.ws, P.geo), at<float>(c.ws, P.D), c.st));
+  if (!ok) return SO2_ERR_CUDA;
   CKL();
   k_edge_gate<<<(M + GATE_EDGES - 1) / GATE_EDGES, 128, GATE_EDGES * P.y.nr * sizeof(float),
                 c.s>>>(P.y, c.d->rbf_cutoff, M, at<float>(c.ws, P.geo), prm.w_rad, prm.b_rad,
@@ -1097,9 +1090,14 @@ so2_status so2conv_edge_frames(int32_t lmax, int64_t E, const float *edge_vec, f
   if (lmax < 0 || lmax > LMAX_SUPPORTED || E < 0) return SO2_ERR_UNSUPPORTED;
   if (E == 0) return SO2_OK;
   if (!edge_vec) return SO2_ERR_INVALID_ARG;
-  const int smem = 8 * (dsize(lmax) + 16) * static_cast<int>(sizeof(float));
-  k_frames<<<warp_grid(static_cast<int>(E < (1 << 30) ? E : (1 << 30)), 8), 256, smem,
-             reinterpret_cast<cudaStream_t>(stream)>>>(lmax, E, edge_vec, R_out, D_out);
+  const int smem = dsize(lmax) * 33 * static_cast<int>(sizeof(float));
+  const int64_t nb = (E + 31) / 32;
+  const int grid = static_cast<int>(nb < 148 * 64 ? nb : 148 * 64);
+  bool ok = true;
+  SO2_DISPATCH_L(lmax, ok = allow_smem(k_frames<L>, smem);
+                 if (ok) k_frames<L><<<grid, 32, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+                     E, edge_vec, R_out, D_out));
+  if (!ok) return SO2_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? SO2_OK : SO2_ERR_CUDA;
 }
 

@@ -7,7 +7,8 @@
 // Wigner-D: D^1 = P R P^T (P maps (x, y, z) to the l = 1 order (y, z, x)),
 // then D^l for l >= 2 by the Ivanic-Ruedenberg recursion (J. Phys. Chem.
 // 1996, 100, 6342; corrections 1998, 102, 9099), which builds each D^l from
-// D^1 and D^{l-1}.  This is the rotation of real spherical harmonics without
+// D^1 and D^{l-1}.  One thread computes one edge's blocks, with every
+// coefficient of the recursion a compile-time constant.  This is the rotation of real spherical harmonics without
 // the Condon-Shortley phase, with Y(R n) = D(R) Y(n).
 //
 // Generators: J_x, J_y are d/dtheta D(R_{x,y}(theta)) at theta = 0 in the
@@ -16,6 +17,8 @@
 // them, a small turn (I + [w]x) R of the frame changes D by
 // (w_x J_x + w_y J_y + w_z J_z) D.
 #pragma once
+
+#include <utility>
 
 #include "common.cuh"
 
@@ -68,22 +71,46 @@ __device__ __forceinline__ bool make_frame(float rx, float ry, float rz, Frame &
 }
 
 // The Ivanic-Ruedenberg recursion writes entry (m, n) of D^l (l >= 2) as a
-// sum of at most IR_TERMS products coef * D^1[i] * D^{l-1}[j], with D^1
-// row-major 3x3 (index (a+1)*3+(b+1)) and D^{l-1} row-major (2l-1)^2.
-// ir_terms lists them (unused slots have coef 0 and indices 0).
+// sum of at most IR_TERMS products coef * D^1[a] * D^{l-1}[b], with D^1
+// row-major 3x3 (index (i+1)*3+(j+1) for orders i, j in -1..1) and D^{l-1}
+// row-major (2l-1)^2.  ir_terms lists them; it is constexpr, so the kernels
+// below get every coefficient and index as an immediate.
 constexpr int IR_TERMS = 10;
 
-__host__ __device__ inline int ir_terms(int l, int m, int n, float *coef, int *i1, int *i2) {
-  const int wp = 2 * l - 1;
-  int nt = 0;
-  auto put = [&](float c, int i, int j, int a, int b) {
-    coef[nt] = c;
-    i1[nt] = (i + 1) * 3 + (j + 1);
-    i2[nt] = (a + l - 1) * wp + (b + l - 1);
-    ++nt;
-  };
-  // c * P(i, a, b)
-  auto P = [&](float c, int i, int a, int b) {
+struct IRTerm {
+  float c;
+  int a, b;
+};
+struct IREntry {
+  IRTerm t[IR_TERMS];
+  int n;
+};
+
+// Square root by Newton's method in double (compile-time coefficients).
+__host__ __device__ constexpr double cx_sqrt(double v) {
+  if (v <= 0.0) return 0.0;
+  double x = v > 1.0 ? v : 1.0;
+  for (int i = 0; i < 200; ++i) {
+    const double nx = 0.5 * (x + v / x);
+    if (nx == x) break;
+    x = nx;
+  }
+  return x;
+}
+
+struct IRBuilder {
+  IREntry e{};
+  int l;
+  __host__ __device__ constexpr void put(double c, int i, int j, int a, int b) {
+    const int wp = 2 * l - 1;
+    e.t[e.n].c = static_cast<float>(c);
+    e.t[e.n].a = (i + 1) * 3 + (j + 1);
+    e.t[e.n].b = (a + l - 1) * wp + (b + l - 1);
+    ++e.n;
+  }
+  // c * P(i, a, b): the D^1 x D^{l-1} product of the recursion, with the
+  // column of D^{l-1} folded back at the edges b = +-l.
+  __host__ __device__ constexpr void P(double c, int i, int a, int b) {
     if (b == -l) {
       put(c, i, 1, a, -l + 1);
       put(c, i, -1, a, l - 1);
@@ -93,125 +120,104 @@ __host__ __device__ inline int ir_terms(int l, int m, int n, float *coef, int *i
     } else {
       put(c, i, 0, a, b);
     }
-  };
+  }
+};
+
+__host__ __device__ constexpr IREntry ir_terms(int l, int m, int n) {
+  IRBuilder B{};
+  B.l = l;
   const int am = m < 0 ? -m : m;
   const int an = n < 0 ? -n : n;
   const int dm0 = (m == 0);
-  const float den = (an == l) ? static_cast<float>((2 * l) * (2 * l - 1))
-                              : static_cast<float>((l + n) * (l - n));
-  const float u = sqrtf(static_cast<float>((l + m) * (l - m)) / den);
-  const float v = 0.5f * sqrtf(static_cast<float>((1 + dm0) * (l + am - 1) * (l + am)) / den) *
-                  static_cast<float>(1 - 2 * dm0);
-  const float wc = -0.5f * sqrtf(static_cast<float>((l - am - 1) * (l - am)) / den) *
-                   static_cast<float>(1 - dm0);
-  const float r2 = 1.41421356237f;
-  if (u != 0.f) P(u, 0, m, n);
-  if (v != 0.f) {
+  const double den = (an == l) ? static_cast<double>((2 * l) * (2 * l - 1))
+                               : static_cast<double>((l + n) * (l - n));
+  const double u = cx_sqrt(static_cast<double>((l + m) * (l - m)) / den);
+  const double v = 0.5 * cx_sqrt(static_cast<double>((1 + dm0) * (l + am - 1) * (l + am)) / den) *
+                   static_cast<double>(1 - 2 * dm0);
+  const double w = -0.5 * cx_sqrt(static_cast<double>((l - am - 1) * (l - am)) / den) *
+                   static_cast<double>(1 - dm0);
+  const double r2 = cx_sqrt(2.0);
+  if (u != 0.0) B.P(u, 0, m, n);
+  if (v != 0.0) {
     if (m == 0) {
-      P(v, 1, 1, n);
-      P(v, -1, -1, n);
+      B.P(v, 1, 1, n);
+      B.P(v, -1, -1, n);
     } else if (m > 0) {
-      P(v * (m == 1 ? r2 : 1.f), 1, m - 1, n);
-      if (m != 1) P(-v, -1, -m + 1, n);
+      B.P(v * (m == 1 ? r2 : 1.0), 1, m - 1, n);
+      if (m != 1) B.P(-v, -1, -m + 1, n);
     } else {
-      if (m != -1) P(v, 1, m + 1, n);
-      P(v * (m == -1 ? r2 : 1.f), -1, -m - 1, n);
+      if (m != -1) B.P(v, 1, m + 1, n);
+      B.P(v * (m == -1 ? r2 : 1.0), -1, -m - 1, n);
     }
   }
-  if (wc != 0.f) {
+  if (w != 0.0) {
     if (m > 0) {
-      P(wc, 1, m + 1, n);
-      P(wc, -1, -m - 1, n);
+      B.P(w, 1, m + 1, n);
+      B.P(w, -1, -m - 1, n);
     } else {
-      P(wc, 1, m - 1, n);
-      P(-wc, -1, -m + 1, n);
+      B.P(w, 1, m - 1, n);
+      B.P(-w, -1, -m + 1, n);
     }
   }
-  for (int t = nt; t < IR_TERMS; ++t) {
-    coef[t] = 0.f;
-    i1[t] = 0;
-    i2[t] = 0;
-  }
-  return nt;
+  return B.e;
 }
 
-// Entry (m, n) of D^l (l >= 2) evaluated directly from the term list.
-__device__ __forceinline__ float ir_entry(int l, int m, int n, const float *D1, const float *Dp) {
-  float c[IR_TERMS];
-  int a[IR_TERMS], b[IR_TERMS];
-  const int nt = ir_terms(l, m, n, c, a, b);
-  float val = 0.f;
-  for (int t = 0; t < nt; ++t) val += c[t] * D1[a[t]] * Dp[b[t]];
-  return val;
+// Entry E (row-major) of D^l from D^1 (registers) and D^{l-1} (Dp[k * s]).
+template <int l, int E, int... T>
+__device__ __forceinline__ float ir_value(const float (&D1)[9], const float *Dp, int s,
+                                          std::integer_sequence<int, T...>) {
+  constexpr int w = 2 * l + 1;
+  constexpr IREntry en = ir_terms(l, E / w - l, E % w - l);
+  float v = 0.f;
+  ((T < en.n ? (v += en.t[T].c * D1[en.t[T].a] * Dp[en.t[T].b * s]) : 0.f), ...);
+  return v;
 }
 
-// Number of tabulated entries for levels 2..lmax (entry index of (l, m, n)
-// is dblock_off(l) - dblock_off(2) + (m+l)(2l+1) + (n+l)).
-__host__ __device__ constexpr int ir_table_entries(int lmax) {
-  return lmax < 2 ? 0 : dblock_off(lmax + 1) - dblock_off(2);
+template <int l, int... E>
+__device__ __forceinline__ void ir_level(const float (&D1)[9], const float *Dp, float *Dl, int s,
+                                         std::integer_sequence<int, E...>) {
+  ((Dl[E * s] = ir_value<l, E>(D1, Dp, s, std::make_integer_sequence<int, IR_TERMS>{})), ...);
 }
 
-// Table layout (structure of arrays, NE = ir_table_entries(lmax)):
-// coef[t * NE + e] floats, then idx[t * NE + e] ints with i1 | i2 << 8.
-__global__ void k_ir_table(int lmax, float *table) {
-  const int NE = ir_table_entries(lmax);
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= NE) return;
-  int l = 2;
-  while (l < lmax && e >= dblock_off(l + 1) - dblock_off(2)) ++l;
-  const int local = e - (dblock_off(l) - dblock_off(2));
-  const int w = 2 * l + 1;
-  float c[IR_TERMS];
-  int a[IR_TERMS], b[IR_TERMS];
-  ir_terms(l, local / w - l, local % w - l, c, a, b);
-  int *idx = reinterpret_cast<int *>(table + IR_TERMS * NE);
-  for (int t = 0; t < IR_TERMS; ++t) {
-    table[t * NE + e] = c[t];
-    idx[t * NE + e] = a[t] | (b[t] << 8);
+template <int l, int L>
+__device__ __forceinline__ void ir_levels(const float (&D1)[9], float *D, int s) {
+  if constexpr (l <= L) {
+    ir_level<l>(D1, D + dblock_off(l - 1) * s, D + dblock_off(l) * s, s,
+                std::make_integer_sequence<int, (2 * l + 1) * (2 * l + 1)>{});
+    ir_levels<l + 1, L>(D1, D, s);
   }
 }
 
-// Full blocks D^0..D^lmax (each (2l+1)^2 row-major, concatenated) of the
-// rotation R, computed by one warp into D (shared memory): the lanes share
-// the entries of each level, levels one after another.  With a term table
-// (k_ir_table) every entry is the same branch-free 10-term sum; without one
-// the terms are enumerated per entry.
-__device__ inline void wigner_blocks_warp(const float *R, int lmax, float *D,
-                                          const float *table = nullptr) {
-  const int lane = threadIdx.x & 31;
-  if (lane == 0) D[0] = 1.f;
-  if (lmax >= 1 && lane < 9) {
-    // (y, z, x) ordering: sh index 0 <- y(1), 1 <- z(2), 2 <- x(0)
-    const int pm[3] = {1, 2, 0};
-    const int a = lane / 3, b = lane % 3;
-    D[dblock_off(1) + lane] = R[pm[a] * 3 + pm[b]];
-  }
-  __syncwarp();
-  const float *D1 = D + dblock_off(1);
-  for (int l = 2; l <= lmax; ++l) {
-    const float *Dp = D + dblock_off(l - 1);
-    float *Dl = D + dblock_off(l);
-    const int w = 2 * l + 1;
-    if (table) {
-      const int NE = ir_table_entries(lmax);
-      const int *tidx = reinterpret_cast<const int *>(table + IR_TERMS * NE);
-      const int base = dblock_off(l) - dblock_off(2);
-      for (int idx = lane; idx < w * w; idx += 32) {
-        float val = 0.f;
+// Full blocks D^0..D^L of the rotation R (row-major 3x3), each (2l+1)^2
+// row-major, concatenated, computed by one thread into D[k * s]
+// (k < dsize(L)); s is the stride between a thread's consecutive entries.
+template <int L>
+__device__ __forceinline__ void wigner_blocks_thread(const float (&R)[9], float *D, int s) {
+  D[0] = 1.f;
+  if constexpr (L >= 1) {
+    // (y, z, x) ordering of the l = 1 functions: index 0 <- y, 1 <- z, 2 <- x
+    constexpr int pm[3] = {1, 2, 0};
+    float D1[9];
 #pragma unroll
-        for (int t = 0; t < IR_TERMS; ++t) {
-          const int pk = __ldg(tidx + t * NE + base + idx);
-          val += __ldg(table + t * NE + base + idx) * D1[pk & 0xff] * Dp[pk >> 8];
-        }
-        Dl[idx] = val;
-      }
-    } else {
-      for (int idx = lane; idx < w * w; idx += 32)
-        Dl[idx] = ir_entry(l, idx / w - l, idx % w - l, D1, Dp);
+    for (int k = 0; k < 9; ++k) {
+      D1[k] = R[pm[k / 3] * 3 + pm[k % 3]];
+      D[(dblock_off(1) + k) * s] = D1[k];
     }
-    __syncwarp();
+    ir_levels<2, L>(D1, D, s);
   }
 }
+
+// Calls f with the compile-time lmax L (0..LMAX_SUPPORTED).
+#define SO2_DISPATCH_L(lmax, ...)              \
+  switch (lmax) {                              \
+    case 0: { constexpr int L = 0; __VA_ARGS__; } break; \
+    case 1: { constexpr int L = 1; __VA_ARGS__; } break; \
+    case 2: { constexpr int L = 2; __VA_ARGS__; } break; \
+    case 3: { constexpr int L = 3; __VA_ARGS__; } break; \
+    case 4: { constexpr int L = 4; __VA_ARGS__; } break; \
+    case 5: { constexpr int L = 5; __VA_ARGS__; } break; \
+    default: { constexpr int L = 6; __VA_ARGS__; } break; \
+  }
 
 __device__ __forceinline__ float gen_s(int l, int k) {
   return 0.5f * sqrtf(static_cast<float>((l - k) * (l + k + 1)));
