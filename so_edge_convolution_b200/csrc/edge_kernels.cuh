@@ -833,7 +833,7 @@ __global__ void k_edge_final(Layout y, float cutoff, int M, const EdgeRec *__res
 // omega[i][2]) is optional.  One thread per channel keeps all nr + 1 sums
 // in registers and reads each product once.  Stage 2 adds the blocks in
 // order.
-constexpr int RAD_TILE = 256;
+constexpr int RAD_TILE = 64;
 constexpr int RAD_MAX_NR = 64;
 __global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__restrict__ geo,
                               const float *__restrict__ Ag, const float *__restrict__ Bg,

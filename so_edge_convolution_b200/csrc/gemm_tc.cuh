@@ -410,7 +410,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (p.store && row < G.M) {
           float *crow = Cg + static_cast<long long>(row) * G.ldc + col0;
           const bool vec = (col0 + 32 <= G.N) && ((reinterpret_cast<uintptr_t>(crow) & 15) == 0);
-          if (atomic_c) {
+          if (atomic_c && vec) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              atomicAdd(reinterpret_cast<float4 *>(crow + j),
+                        make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                    __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])));
+          } else if (atomic_c) {
             for (int j = 0; j < 32 && col0 + j < G.N; ++j) atomicAdd(crow + j, __uint_as_float(r[j]));
           } else if (vec) {
 #pragma unroll

@@ -477,7 +477,7 @@ so2_status pack_weights(Ctx &c, const void *w, bool transposes) {
     CK(cudaMemsetAsync(th, 0, 2ull * y.WTR * y.WTK, c.s));
     if (tl) CK(cudaMemsetAsync(tl, 0, 2ull * y.WTR * y.WTK, c.s));
   }
-  dim3 grid(64, y.ng);
+  dim3 grid(256, y.ng);
   BlockOffsets bo = block_offsets(y);
   for (int t = 0; t < (transposes ? 2 : 1); ++t) {
     __nv_bfloat16 *h = t ? th : wh, *l = t ? tl : wl;
@@ -582,13 +582,25 @@ so2_status gemm_dw(Ctx &c, int M, int seg_g, int seg_a) {
   const Plan &P = c.P;
   const Layout &y = P.y;
   const int Kp = round_up(M, 64);
-  // the output is small (a few hundred tiles at most) and K long: split K
-  // until the launch covers about two waves of SMs
+  // The output is small (a few hundred tiles at most) and K long: split K.
+  // Pick the split count that wastes least of the last wave (the time is
+  // waves x K per split), keeping at least 2,048 edges per split so that the
+  // atomic epilogue of a split stays hidden behind the next one's main loop.
   int tiles = 0;
   for (int g = 0; g < y.ng; ++g)
     tiles += ((y.Kout[g] + GEMM_BM - 1) / GEMM_BM) * ((y.Kin[g] + GEMM_BN - 1) / GEMM_BN);
-  int ksplit = (2 * num_sms() + tiles - 1) / tiles;
-  if (ksplit > Kp / 512) ksplit = Kp / 512 > 0 ? Kp / 512 : 1;  // keep >= 512 edges per split
+  const int sms = num_sms();
+  const int max_split = Kp / 2048 > 1 ? Kp / 2048 : 1;
+  int ksplit = 1;
+  long long best = -1;
+  for (int ks = 1; ks <= max_split; ++ks) {
+    const long long waves = (static_cast<long long>(tiles) * ks + sms - 1) / sms;
+    const long long cost = waves * round_up((Kp + ks - 1) / ks, 64);
+    if (best < 0 || cost < best) {
+      best = cost;
+      ksplit = ks;
+    }
+  }
   GemmLauncher L;
   for (int g = 0; g < y.ng; ++g)
     L.add(y.Kout[g], y.Kin[g], Kp, y.kout_off[g], seg_g * P.chunk, y.kin_off[g], seg_a * P.chunk,
