@@ -13,20 +13,40 @@
 
 namespace so2 {
 
-// Resident 256-thread blocks per SM that the generic-degree (runtime lmax)
-// gather kernels are compiled for: caps their registers, since they are
-// latency bound and every level is instantiated in one function.
-#ifndef SO2_GATHER_MINB
+// Occupancy and load-batching of the per-edge gather kernels (rotation on
+// gather, edge terms).  They are latency bound, so each is compiled for a
+// number of resident 256-thread blocks per SM (which caps its registers),
+// and the edge-term kernels may fence every few rows so that the compiler
+// does not hoist a whole level's loads into registers.  Defaults are the
+// fastest measured on B200 for lmax 4 and 6, mmax 2, C 128.
+#ifndef SO2_GATHER_MINB  // runtime-degree kernels
 #define SO2_GATHER_MINB 2
 #endif
-// Rows of x / G whose loads may be in flight at once in the generic-degree
-// edge-term kernels (0: no limit).
-#ifndef SO2_ET_BATCH
+#ifndef SO2_ET_BATCH  // rows per load batch, runtime-degree edge terms (0: no fence)
 #define SO2_ET_BATCH 2
+#endif
+#ifndef SO2_ET_MINB_LC  // compile-time-degree edge terms
+#define SO2_ET_MINB_LC 2
+#endif
+#ifndef SO2_ET_BATCH_LC
+#define SO2_ET_BATCH_LC 2
+#endif
+#ifndef SO2_ROT_MINB  // compile-time-degree rotation, lmax < 6
+#define SO2_ROT_MINB 2
+#endif
+#ifndef SO2_ROT_MINB_L6  // compile-time-degree rotation, lmax 6
+#define SO2_ROT_MINB_L6 3
 #endif
 
 // Keeps the compiler from moving loads across this point.
 __device__ __forceinline__ void load_fence() { asm volatile("" ::: "memory"); }
+
+// Whether the edge-term kernels fence before row mp of degree l.
+template <int LC>
+__device__ __forceinline__ constexpr bool et_fence(int l, int mp) {
+  constexpr int b = LC < 0 ? SO2_ET_BATCH : SO2_ET_BATCH_LC;
+  return b > 0 && mp > -l && (mp + l) % b == 0;
+}
 
 // Degree l as a compile-time value.
 template <int N>
@@ -322,7 +342,7 @@ __device__ __forceinline__ void stage_d(const float *De, int dsz, float *sD) {
 // LC >= 0 fixes lmax at compile time (loops fully unrolled); -1 reads it
 // from the layout.
 template <typename TX, int MM, int LC = -1>
-__global__ void __launch_bounds__(256, LC >= 0 ? 2 : SO2_GATHER_MINB) k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec,
+__global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO2_ROT_MINB : SO2_GATHER_MINB)) k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec,
                                 const float *__restrict__ D, const TX *__restrict__ X, int side,
                                 int use_src, Coef A, Coef B, const float *__restrict__ omega,
                                 __nv_bfloat16 *__restrict__ out_hi, __nv_bfloat16 *__restrict__ out_lo,
@@ -658,7 +678,7 @@ __global__ void k_unstack_grad(Layout y, BlockOffsets bo, const float *__restric
 // PART: 3 = both sides in one pass; 1 = output side only (writes Gg and h);
 // 2 = input side only (adds its share to h).
 template <typename TX, int MM, int LC = -1, int PART = 3>
-__global__ void __launch_bounds__(256, LC >= 0 ? 1 : SO2_GATHER_MINB) k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
+__global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MINB) k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
                              const float *__restrict__ D, const float *__restrict__ gate,
                              const float *__restrict__ G, const TX *__restrict__ X,
                              const float *__restrict__ V, const float *__restrict__ Ga,
@@ -688,7 +708,7 @@ __global__ void __launch_bounds__(256, LC >= 0 ? 1 : SO2_GATHER_MINB) k_edge_ter
         const float *Dl = sD + dblock_off(l);
 #pragma unroll
         for (int mp = -l; mp <= l; ++mp) {
-          if (LC < 0 && SO2_ET_BATCH > 0 && mp > -l && (mp + l) % SO2_ET_BATCH == 0) load_fence();
+          if (et_fence<LC>(l, mp)) load_fence();
           const float4 gx = load4(Gn + (l * l + l + mp) * y.co + c);
 #pragma unroll
           for (int m = -mw; m <= mw; ++m) {
@@ -739,7 +759,7 @@ __global__ void __launch_bounds__(256, LC >= 0 ? 1 : SO2_GATHER_MINB) k_edge_ter
         const float *Dl = sD + dblock_off(l);
 #pragma unroll
         for (int mp = -l; mp <= l; ++mp) {
-          if (LC < 0 && SO2_ET_BATCH > 0 && mp > -l && (mp + l) % SO2_ET_BATCH == 0) load_fence();
+          if (et_fence<LC>(l, mp)) load_fence();
           const float4 xv = load4(Xn + (l * l + l + mp) * y.ci + c);
 #pragma unroll
           for (int m = -mw; m <= mw; ++m) {
