@@ -200,10 +200,14 @@ __device__ __forceinline__ void epi_scatter_chunk(const GemmParams &p, int row_b
 
 // BK = 32 uses the 64-byte swizzle (4 stages of 48 KB with hi/lo planes),
 // BK = 64 the 128-byte swizzle.
-template <int BK, int STAGES, bool SPLIT, bool SCATTER>
+// With PAIR, two CTAs (a cluster) share each 256 x 256 tile: each holds 128
+// rows of A and of the output, and half (128 rows) of B.
+template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool PAIR = false>
 struct GemmCfg {
+  static constexpr int NB = PAIR ? GEMM_BN / 2 : GEMM_BN;  // B rows held by this CTA
+  static constexpr int TBM = PAIR ? 2 * GEMM_BM : GEMM_BM;  // output rows per tile
   static constexpr int A_BYTES = GEMM_BM * BK * 2;
-  static constexpr int B_BYTES = GEMM_BN * BK * 2;
+  static constexpr int B_BYTES = NB * BK * 2;
   static constexpr int PLANES = SPLIT ? 2 : 1;
   static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES) * PLANES;
   static constexpr int SMEM =
@@ -218,6 +222,8 @@ __device__ __forceinline__ uint64_t sdesc_k(uint32_t saddr, int bk) {
 
 // Tile -> group, output origin and K range [k0, k0 + klen_t).  K splits are
 // outermost inside a group so that concurrent tiles share operand rows in L2.
+// TBM: output rows per tile.
+template <int TBM>
 __device__ __forceinline__ void tile_coords(const GemmParams &p, int tile, int &gi, int &m0,
                                             int &n0, int &k0, int &kl) {
   gi = 0;
@@ -225,18 +231,21 @@ __device__ __forceinline__ void tile_coords(const GemmParams &p, int tile, int &
   const GemmGroup &G = p.g[gi];
   const int local = tile - G.tile_begin;
   const int ks = local / G.tiles_mn, mn = local % G.tiles_mn;
-  m0 = (mn / G.tiles_n) * GEMM_BM;
+  m0 = (mn / G.tiles_n) * TBM;
   n0 = (mn % G.tiles_n) * GEMM_BN;
   k0 = ks * G.klen;
   kl = (G.K - k0) < G.klen ? (G.K - k0) : G.klen;
 }
 
-template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool MN>
+// PAIR: launched in clusters of two CTAs; the even CTA issues the pair's
+// MMAs, both load their operand halves and drain their own accumulator lanes.
+template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool MN, bool PAIR = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
               const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
               const __grid_constant__ GemmParams p) {
-  using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER>;
+  using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER, PAIR>;
+  constexpr int NB = Cfg::NB, TBM = Cfg::TBM;
   static_assert(!MN || BK % 16 == 0, "MN-major K block");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -251,6 +260,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA pair: rank in the cluster, the cluster's index and count; the even
+  // CTA's full[] and tempty[] barriers serve both CTAs
+  const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const int unit0 = PAIR ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
+  const uint32_t full_c = PAIR ? mapa_shared(smem_u32(full), 0) : 0;
+  const uint32_t tempty_c = PAIR ? mapa_shared(smem_u32(tempty), 0) : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -259,17 +275,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], EPI_WARPS);  // one arrive per epilogue warp
+      mbar_init(&tempty[a], (PAIR ? 2 : 1) * EPI_WARPS);  // one arrive per epilogue warp
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -277,11 +299,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ---------------- TMA producer ----------------
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+    for (int tile = unit0; ok && tile < p.total_tiles; tile += units) {
       int gi, m0, n0, k0, kl;
-      tile_coords(p, tile, gi, m0, n0, k0, kl);
+      tile_coords<TBM>(p, tile, gi, m0, n0, k0, kl);
       const GemmGroup &G = p.g[gi];
       const int nk = kl / BK;
+      const int am = G.a_row + m0 + rank * GEMM_BM;  // this CTA's A rows
+      const int bn = G.b_row + n0 + rank * NB;       // this CTA's B rows
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
@@ -290,46 +314,48 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           break;
         }
         uint8_t *st = smem + s * Cfg::STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[s], Cfg::STAGE_BYTES);
+        // the even CTA expects the bytes of both CTAs' loads
+        if (rank == 0) mbar_arrive_expect_tx(&full[s], (PAIR ? 2 : 1) * Cfg::STAGE_BYTES);
+        auto load = [&](void *dst, const CUtensorMap *map, int c0, int c1) {
+          if (PAIR)
+            tma_load_2d_pair(dst, map, full_c + 8u * s, c0, c1);
+          else
+            tma_load_2d(dst, map, &full[s], c0, c1);
+        };
         const int kc = k0 + kb * BK;
         if (!MN) {
-          tma_load_2d(st, &tA_hi, &full[s], G.a_col + kc, G.a_row + m0);
-          tma_load_2d(st + Cfg::A_BYTES, &tB_hi, &full[s], G.b_col + kc, G.b_row + n0);
+          load(st, &tA_hi, G.a_col + kc, am);
+          load(st + Cfg::A_BYTES, &tB_hi, G.b_col + kc, bn);
           if (SPLIT) {
-            tma_load_2d(st + Cfg::A_BYTES + Cfg::B_BYTES, &tA_lo, &full[s], G.a_col + kc,
-                        G.a_row + m0);
-            tma_load_2d(st + 2 * Cfg::A_BYTES + Cfg::B_BYTES, &tB_lo, &full[s], G.b_col + kc,
-                        G.b_row + n0);
+            load(st + Cfg::A_BYTES + Cfg::B_BYTES, &tA_lo, G.a_col + kc, am);
+            load(st + 2 * Cfg::A_BYTES + Cfg::B_BYTES, &tB_lo, G.b_col + kc, bn);
           }
         } else {
           // MN-major operands: the inner TMA coordinate is the M / N index, the
           // outer one the K index; one box per 64 M / N elements
           constexpr int BOX = 64 * BK * 2;
-          for (int h = 0; h < GEMM_BM / 64; ++h)
-            tma_load_2d(st + h * BOX, &tA_hi, &full[s], G.a_row + m0 + 64 * h, G.a_col + kc);
-          for (int h = 0; h < GEMM_BN / 64; ++h)
-            tma_load_2d(st + Cfg::A_BYTES + h * BOX, &tB_hi, &full[s], G.b_row + n0 + 64 * h,
-                        G.b_col + kc);
+          for (int h = 0; h < GEMM_BM / 64; ++h) load(st + h * BOX, &tA_hi, am + 64 * h, G.a_col + kc);
+          for (int h = 0; h < NB / 64; ++h)
+            load(st + Cfg::A_BYTES + h * BOX, &tB_hi, bn + 64 * h, G.b_col + kc);
           if (SPLIT) {
             for (int h = 0; h < GEMM_BM / 64; ++h)
-              tma_load_2d(st + Cfg::A_BYTES + Cfg::B_BYTES + h * BOX, &tA_lo, &full[s],
-                          G.a_row + m0 + 64 * h, G.a_col + kc);
-            for (int h = 0; h < GEMM_BN / 64; ++h)
-              tma_load_2d(st + 2 * Cfg::A_BYTES + Cfg::B_BYTES + h * BOX, &tB_lo, &full[s],
-                          G.b_row + n0 + 64 * h, G.b_col + kc);
+              load(st + Cfg::A_BYTES + Cfg::B_BYTES + h * BOX, &tA_lo, am + 64 * h, G.a_col + kc);
+            for (int h = 0; h < NB / 64; ++h)
+              load(st + 2 * Cfg::A_BYTES + Cfg::B_BYTES + h * BOX, &tB_lo, bn + 64 * h,
+                   G.b_col + kc);
           }
         }
       }
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer ----------------
-    constexpr uint32_t idesc = idesc_bf16_f32(GEMM_BM, GEMM_BN, MN);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ---------------- MMA issuer (the even CTA of a pair) ----------------
+    constexpr uint32_t idesc = idesc_bf16_f32(TBM, GEMM_BN, MN);
     constexpr uint32_t LBO = 64 * BK * 2;  // MN-major: bytes between 64-element MN chunks
     int it = 0, tcount = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tcount) {
+    for (int tile = unit0; ok && tile < p.total_tiles; tile += units, ++tcount) {
       int gi, m0, n0, k0, kl;
-      tile_coords(p, tile, gi, m0, n0, k0, kl);
+      tile_coords<TBM>(p, tile, gi, m0, n0, k0, kl);
       const int nk = kl / BK;
       const int acc = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
@@ -357,15 +383,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           // next 16 K: 32 bytes along a K-major row, or two 1024-byte atoms of
           // an MN-major tile (in 16-byte units)
           const uint64_t step = static_cast<uint64_t>(MN ? kk * 128 : kk * 2);
-          umma_bf16(d_tmem, a_hi + step, b_hi + step, idesc, (kb | kk) != 0);
-          if (SPLIT) {
-            umma_bf16(d_tmem, a_hi + step, b_lo + step, idesc, 1);
-            umma_bf16(d_tmem, a_lo + step, b_hi + step, idesc, 1);
+          if (PAIR) {
+            umma_bf16_pair(d_tmem, a_hi + step, b_hi + step, idesc, (kb | kk) != 0);
+            if (SPLIT) {
+              umma_bf16_pair(d_tmem, a_hi + step, b_lo + step, idesc, 1);
+              umma_bf16_pair(d_tmem, a_lo + step, b_hi + step, idesc, 1);
+            }
+          } else {
+            umma_bf16(d_tmem, a_hi + step, b_hi + step, idesc, (kb | kk) != 0);
+            if (SPLIT) {
+              umma_bf16(d_tmem, a_hi + step, b_lo + step, idesc, 1);
+              umma_bf16(d_tmem, a_lo + step, b_hi + step, idesc, 1);
+            }
           }
         }
-        umma_commit(&empty[s]);
+        if (PAIR)
+          umma_commit_pair(&empty[s]);  // frees stage s in both CTAs
+        else
+          umma_commit(&empty[s]);
       }
-      if (ok) umma_commit(&tfull[acc]);
+      if (ok) {
+        if (PAIR)
+          umma_commit_pair(&tfull[acc]);
+        else
+          umma_commit(&tfull[acc]);
+      }
     }
   } else if (warp >= 2) {
     // ---------------- epilogue: TMEM -> registers -> C and/or node sums ----------------
@@ -373,14 +415,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int half = (warp - 2) >> 2;  // which share of the tile's column chunks
     const EpiScratch xs = epi_scratch(epi_smem + (warp - 2) * (EPI_SMEM_PER_WARP / 4));
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tcount) {
+    for (int tile = unit0; tile < p.total_tiles; tile += units, ++tcount) {
       int gi, m0, n0, k0, kl;
-      tile_coords(p, tile, gi, m0, n0, k0, kl);
+      tile_coords<TBM>(p, tile, gi, m0, n0, k0, kl);
       const GemmGroup &G = p.g[gi];
       const bool atomic_c = G.klen < G.K;  // split K: partial sums meet in C
       const int acc = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
-      const int row_base = m0 + q * 32;
+      const int row_base = m0 + rank * GEMM_BM + q * 32;  // this CTA's accumulator lanes
       if (SCATTER && p.scatter) {
         const int e = row_base + lane;
         xs.keys[lane] = (e < G.M) ? p.sc.rec[e].w : -1;
@@ -443,14 +485,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if (PAIR)
+          mbar_arrive_cluster(tempty_c + 8u * acc);  // the even CTA's barrier
+        else
+          mbar_arrive(&tempty[acc]);
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
+  // a pair's MMAs read both CTAs' shared memory and write both CTAs' tensor
+  // memory: neither CTA frees or leaves before the other is done
+  if (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, Cfg::TMEM_COLS);
+    if (PAIR)
+      tmem_dealloc_pair(tmem, Cfg::TMEM_COLS);
+    else
+      tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
 }
 

@@ -299,6 +299,11 @@ bool allow_smem(K kernel, int bytes) {
          cudaSuccess;
 }
 
+// Plain products on CTA pairs (cta_group::2).
+#ifndef SO2_PAIR_PLAIN
+#define SO2_PAIR_PLAIN 1
+#endif
+
 int warp_grid(int M, int warps_per_block) {
   int g = (M + warps_per_block - 1) / warps_per_block;
   if (g < 1) g = 1;
@@ -311,6 +316,7 @@ int warp_grid(int M, int warps_per_block) {
 // --------------------------------------------------------------------------
 struct GemmLauncher {
   GemmParams p{};
+  int bm = GEMM_BM;  // output rows per tile: 2 * GEMM_BM for CTA-pair launches
   // ksplit > 1 splits K into that many ranges (multiples of 64) whose
   // partial products are added into C atomically (C must hold the base).
   void add(int M, int N, int K, int a_row, int a_col, int b_row, int b_col, long long c_off,
@@ -328,7 +334,7 @@ struct GemmLauncher {
     g.ldc = ldc;
     g.mgroup = p.n_groups - 1;
     g.tiles_n = (N + GEMM_BN - 1) / GEMM_BN;
-    g.tiles_mn = ((M + GEMM_BM - 1) / GEMM_BM) * g.tiles_n;
+    g.tiles_mn = ((M + bm - 1) / bm) * g.tiles_n;
     if (ksplit < 1) ksplit = 1;
     g.klen = round_up((K + ksplit - 1) / ksplit, 64);
     if (g.klen > K) g.klen = K;
@@ -338,28 +344,64 @@ struct GemmLauncher {
   }
 };
 
-template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool MN>
+template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool MN, bool PAIR = false>
 cudaError_t launch_gemm_t(const CUtensorMap &a_hi, const CUtensorMap &a_lo, const CUtensorMap &b_hi,
                           const CUtensorMap &b_lo, const GemmParams &p, cudaStream_t s) {
-  using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER>;
+  using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER, PAIR>;
+  auto kernel = k_gemm_tc<BK, STAGES, SPLIT, SCATTER, MN, PAIR>;
   static bool configured = false;
+  static int max_units = 0;  // persistent CTAs (non-pair) or clusters (pair)
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BK, STAGES, SPLIT, SCATTER, MN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM);
     if (e != cudaSuccess) return e;
+    max_units = num_sms();
+    if (PAIR) {
+      // clusters of two CTAs that can be resident at once (both SMs of a TPC)
+      cudaLaunchConfig_t cfg{};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * max_units, 1, 1);
+      cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+      cfg.dynamicSmemBytes = Cfg::SMEM;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+      if (e != cudaSuccess) return e;
+      if (n < 1) return cudaErrorInvalidConfiguration;
+      max_units = n;
+    }
     configured = true;
   }
-  static int sms = num_sms();
-  const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-  k_gemm_tc<BK, STAGES, SPLIT, SCATTER, MN><<<grid, GEMM_THREADS, Cfg::SMEM, s>>>(a_hi, a_lo,
-                                                                               b_hi, b_lo, p);
-  return cudaPeekAtLastError();
+  const int units = p.total_tiles < max_units ? p.total_tiles : max_units;
+  if (!PAIR) {
+    kernel<<<units, GEMM_THREADS, Cfg::SMEM, s>>>(a_hi, a_lo, b_hi, b_lo, p);
+    return cudaPeekAtLastError();
+  }
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * units, 1, 1);
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a_hi, a_lo, b_hi, b_lo, p);
 }
 
 cudaError_t launch_gemm(int kind, bool split, const CUtensorMap &a_hi, const CUtensorMap &a_lo,
                         const CUtensorMap &b_hi, const CUtensorMap &b_lo, GemmParams p,
                         float *C, int beta, DevStatus *st, cudaStream_t s,
-                        const GemmScatter *sc = nullptr, bool store = true, bool mn = false) {
+                        const GemmScatter *sc = nullptr, bool store = true, bool mn = false,
+                        bool pair = false) {
   if (p.total_tiles == 0) return cudaSuccess;
   p.C = C;
   p.beta = beta;
@@ -384,6 +426,9 @@ cudaError_t launch_gemm(int kind, bool split, const CUtensorMap &a_hi, const CUt
   else if (mn)
     r = split ? launch_gemm_t<32, 4, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, 4, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
+  else if (pair)
+    r = split ? launch_gemm_t<32, 6, true, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
+              : launch_gemm_t<64, 6, false, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
   else
     r = split ? launch_gemm_t<32, 4, true, false, false>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, 4, false, false, false>(a_hi, a_lo, b_hi, b_lo, p, s);
@@ -401,6 +446,7 @@ struct Ctx {
   cudaStream_t s;
   DevStatus *st;
   CUtensorMap m_a_hi, m_a_lo, m_v_hi, m_v_lo, m_wst_hi, m_wst_lo, m_wtr_hi, m_wtr_lo;
+  CUtensorMap m_wst2_hi, m_wst2_lo;  // stacked weights, half-height boxes (CTA pairs)
   CUtensorMap m_amn_hi, m_amn_lo, m_vmn_hi, m_vmn_lo;  // the same planes, MN-major boxes
 };
 
@@ -430,6 +476,8 @@ so2_status build_maps(Ctx &c, bool bwd) {
   ok &= make_map(&c.m_a_lo, at<void>(ws, P.split ? P.a_lo : P.a_hi), ra, y.KA, y.KA, GEMM_BM, bk);
   ok &= make_map(&c.m_wst_hi, at<void>(ws, P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN, bk);
   ok &= make_map(&c.m_wst_lo, at<void>(ws, P.split ? P.wst_lo : P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN, bk);
+  ok &= make_map(&c.m_wst2_hi, at<void>(ws, P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN / 2, bk);
+  ok &= make_map(&c.m_wst2_lo, at<void>(ws, P.split ? P.wst_lo : P.wst_hi), y.WR, y.WK, y.WK, GEMM_BN / 2, bk);
   if (bwd) {
     ok &= make_map(&c.m_v_hi, at<void>(ws, P.gv_hi), rg, y.KG, y.KG, GEMM_BM, bk);
     ok &= make_map(&c.m_v_lo, at<void>(ws, P.split ? P.gv_lo : P.gv_hi), rg, y.KG, y.KG, GEMM_BM, bk);
@@ -622,15 +670,19 @@ so2_status gemm_ga(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store
   return SO2_OK;
 }
 
-// V = rotated features times stacked weights (one group per m).
+// V = rotated features times stacked weights (one group per m).  The plain
+// product runs on CTA pairs (256 x 256 tiles, half of B per CTA).
 so2_status gemm_v(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store = true) {
   const Plan &P = c.P;
   const Layout &y = P.y;
+  const bool pair = SO2_PAIR_PLAIN && !sc;
   GemmLauncher L;
+  L.bm = pair ? 2 * GEMM_BM : GEMM_BM;
   for (int g = 0; g < y.ng; ++g)
     L.add(rows, y.Kout[g], y.Kin_pad[g], 0, y.kin_off[g], y.wr_off[g], 0, y.kout_off[g], y.KG);
-  CK(launch_gemm(0, P.split, c.m_a_hi, c.m_a_lo, c.m_wst_hi, c.m_wst_lo, L.p, at<float>(c.ws, P.V), 0,
-                 c.st, c.s, sc, store));
+  CK(launch_gemm(0, P.split, c.m_a_hi, c.m_a_lo, pair ? c.m_wst2_hi : c.m_wst_hi,
+                 pair ? c.m_wst2_lo : c.m_wst_lo, L.p, at<float>(c.ws, P.V), 0, c.st, c.s, sc,
+                 store, false, pair));
   return SO2_OK;
 }
 
