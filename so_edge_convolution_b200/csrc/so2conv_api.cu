@@ -299,9 +299,16 @@ bool allow_smem(K kernel, int bytes) {
          cudaSuccess;
 }
 
-// Plain products on CTA pairs (cta_group::2).
+// Which products run on CTA pairs (cta_group::2): plain, with the fused
+// reduction epilogue, weight gradients (MN-major operands).
 #ifndef SO2_PAIR_PLAIN
 #define SO2_PAIR_PLAIN 1
+#endif
+#ifndef SO2_PAIR_SCATTER
+#define SO2_PAIR_SCATTER 1
+#endif
+#ifndef SO2_PAIR_MN
+#define SO2_PAIR_MN 1
 #endif
 
 int warp_grid(int M, int warps_per_block) {
@@ -420,9 +427,15 @@ cudaError_t launch_gemm(int kind, bool split, const CUtensorMap &a_hi, const CUt
   // the fused reduction epilogue's scratch (6.4 KB per epilogue warp) can cost
   // a pipeline stage
   cudaError_t r;
-  if (sc)
+  if (sc && pair)
+    r = split ? launch_gemm_t<32, 4, true, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
+              : launch_gemm_t<64, 4, false, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
+  else if (sc)
     r = split ? launch_gemm_t<32, SO2_SCATTER_STAGES, true, true, false>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, SO2_SCATTER_STAGES, false, true, false>(a_hi, a_lo, b_hi, b_lo, p, s);
+  else if (mn && pair)
+    r = split ? launch_gemm_t<32, 6, true, false, true, true>(a_hi, a_lo, b_hi, b_lo, p, s)
+              : launch_gemm_t<64, 6, false, false, true, true>(a_hi, a_lo, b_hi, b_lo, p, s);
   else if (mn)
     r = split ? launch_gemm_t<32, 4, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, 4, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
@@ -447,6 +460,7 @@ struct Ctx {
   DevStatus *st;
   CUtensorMap m_a_hi, m_a_lo, m_v_hi, m_v_lo, m_wst_hi, m_wst_lo, m_wtr_hi, m_wtr_lo;
   CUtensorMap m_wst2_hi, m_wst2_lo;  // stacked weights, half-height boxes (CTA pairs)
+  CUtensorMap m_wtr2_hi, m_wtr2_lo;  // their transposes, likewise
   CUtensorMap m_amn_hi, m_amn_lo, m_vmn_hi, m_vmn_lo;  // the same planes, MN-major boxes
 };
 
@@ -483,6 +497,8 @@ so2_status build_maps(Ctx &c, bool bwd) {
     ok &= make_map(&c.m_v_lo, at<void>(ws, P.split ? P.gv_lo : P.gv_hi), rg, y.KG, y.KG, GEMM_BM, bk);
     ok &= make_map(&c.m_wtr_hi, at<void>(ws, P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN, bk);
     ok &= make_map(&c.m_wtr_lo, at<void>(ws, P.split ? P.wtr_lo : P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN, bk);
+    ok &= make_map(&c.m_wtr2_hi, at<void>(ws, P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN / 2, bk);
+    ok &= make_map(&c.m_wtr2_lo, at<void>(ws, P.split ? P.wtr_lo : P.wtr_hi), y.WTR, y.WTK, y.WTK, GEMM_BN / 2, bk);
     ok &= make_map_mn(&c.m_amn_hi, at<void>(ws, P.a_hi), ra, y.KA, y.KA, bk);
     ok &= make_map_mn(&c.m_amn_lo, at<void>(ws, P.split ? P.a_lo : P.a_hi), ra, y.KA, y.KA, bk);
     ok &= make_map_mn(&c.m_vmn_hi, at<void>(ws, P.gv_hi), rg, y.KG, y.KG, bk);
@@ -634,10 +650,12 @@ so2_status gemm_dw(Ctx &c, int M, int seg_g, int seg_a) {
   // Pick the split count that wastes least of the last wave (the time is
   // waves x K per split), keeping at least 2,048 edges per split so that the
   // atomic epilogue of a split stays hidden behind the next one's main loop.
+  const bool pair = SO2_PAIR_MN;
+  const int bm = pair ? 2 * GEMM_BM : GEMM_BM;
   int tiles = 0;
   for (int g = 0; g < y.ng; ++g)
-    tiles += ((y.Kout[g] + GEMM_BM - 1) / GEMM_BM) * ((y.Kin[g] + GEMM_BN - 1) / GEMM_BN);
-  const int sms = num_sms();
+    tiles += ((y.Kout[g] + bm - 1) / bm) * ((y.Kin[g] + GEMM_BN - 1) / GEMM_BN);
+  const int sms = pair ? num_sms() / 2 : num_sms();  // concurrent tiles
   const int max_split = Kp / 2048 > 1 ? Kp / 2048 : 1;
   int ksplit = 1;
   long long best = -1;
@@ -650,11 +668,12 @@ so2_status gemm_dw(Ctx &c, int M, int seg_g, int seg_a) {
     }
   }
   GemmLauncher L;
+  L.bm = bm;
   for (int g = 0; g < y.ng; ++g)
     L.add(y.Kout[g], y.Kin[g], Kp, y.kout_off[g], seg_g * P.chunk, y.kin_off[g], seg_a * P.chunk,
           static_cast<long long>(y.wr_off[g]) * y.WK, y.WK, ksplit);
   CK(launch_gemm(2, P.split, c.m_vmn_hi, c.m_vmn_lo, c.m_amn_hi, c.m_amn_lo, L.p,
-                 at<float>(c.ws, P.dws), 1, c.st, c.s, nullptr, true, true));
+                 at<float>(c.ws, P.dws), 1, c.st, c.s, nullptr, true, true, pair));
   return SO2_OK;
 }
 
@@ -662,11 +681,14 @@ so2_status gemm_dw(Ctx &c, int M, int seg_g, int seg_a) {
 so2_status gemm_ga(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store = true) {
   const Plan &P = c.P;
   const Layout &y = P.y;
+  const bool pair = sc ? SO2_PAIR_SCATTER : SO2_PAIR_PLAIN;
   GemmLauncher L;
+  L.bm = pair ? 2 * GEMM_BM : GEMM_BM;
   for (int g = 0; g < y.ng; ++g)
     L.add(rows, y.Kin[g], y.Kout_pad[g], 0, y.kout_off[g], y.wt_off[g], 0, y.kin_off[g], y.KA);
-  CK(launch_gemm(1, P.split, c.m_v_hi, c.m_v_lo, c.m_wtr_hi, c.m_wtr_lo, L.p,
-                 at<float>(c.ws, P.Ga), 0, c.st, c.s, sc, store));
+  CK(launch_gemm(1, P.split, c.m_v_hi, c.m_v_lo, pair ? c.m_wtr2_hi : c.m_wtr_hi,
+                 pair ? c.m_wtr2_lo : c.m_wtr_lo, L.p, at<float>(c.ws, P.Ga), 0, c.st, c.s, sc,
+                 store, false, pair));
   return SO2_OK;
 }
 
@@ -675,7 +697,7 @@ so2_status gemm_ga(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store
 so2_status gemm_v(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store = true) {
   const Plan &P = c.P;
   const Layout &y = P.y;
-  const bool pair = SO2_PAIR_PLAIN && !sc;
+  const bool pair = sc ? SO2_PAIR_SCATTER : SO2_PAIR_PLAIN;
   GemmLauncher L;
   L.bm = pair ? 2 * GEMM_BM : GEMM_BM;
   for (int g = 0; g < y.ng; ++g)
