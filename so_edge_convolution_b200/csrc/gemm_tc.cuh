@@ -110,42 +110,70 @@ __device__ __forceinline__ EpiScratch epi_scratch(float *base) {
   return e;
 }
 
-// Stage D^l[m][:] for the warp's 32 edges (rows row_base..) into Dw.
-__device__ __forceinline__ void epi_stage_d(const GemmParams &p, const GemmGroup &G, int row_base,
-                                            int l, int m, const EpiScratch &x) {
+// Stage D^l[m][:] (W = 2l + 1 floats, row stride 16) of the warp's 32 edges
+// (rows row_base..) into Dw; zero past the end of the chunk.
+template <int W>
+__device__ __forceinline__ void epi_stage_d(const GemmScatter &S, int M, int row_base, int doff,
+                                            const EpiScratch &x) {
   const int lane = threadIdx.x & 31;
-  const int w = 2 * l + 1;
-  const int doff = l * (4 * l * l - 1) / 3 + (m + l) * w;
-  for (int idx = lane; idx < 32 * w; idx += 32) {
-    const int el = idx / w, k = idx % w;
+#pragma unroll
+  for (int it = 0; it < W; ++it) {
+    const int idx = lane + 32 * it;
+    const int el = idx / W, k = idx - el * W;
     const int ee = row_base + el;
-    x.Dw[el * 16 + k] = (ee < G.M) ? p.sc.D[(int64_t)ee * p.sc.dsz + doff + k] : 0.f;
+    x.Dw[el * 16 + k] = (ee < M) ? S.D[(int64_t)ee * S.dsz + doff + k] : 0.f;
   }
 }
 
-// The sums of one warp-chunk for a fixed width W = 2l + 1 (see below).  The
-// warp's 32 edges split into runs of equal node (a ballot finds the run
-// starts); each run is summed branch-free and flushed with W coalesced
-// atomics.
+// One warp, one 32-column chunk (channels c0.. of edge-frame row (l, m)) of
+// its 32 edges: adds sum_e D_e^l[m][m'] g_e[c] v_e[c] onto
+// out[key_e][(l, m')][c], one coalesced atomic per (node run, m', c).
+// r holds one edge's 32 values per lane (lane = edge); keys must be staged;
+// with `stage` the edges' D rows are staged into Dw first.  Each lane scales
+// its edge's values by the gate (8 vector loads of its gate row) on the way
+// into shared memory, read back with lane = channel; the warp's 32 edges split into
+// runs of equal node (a ballot finds the run starts), each summed in
+// registers and flushed with W coalesced atomics.
 template <int W>
-__device__ __forceinline__ void epi_rotate_reduce(const GemmScatter &S, int row_base, int l, int c,
-                                                  const EpiScratch &x) {
+__device__ __forceinline__ void epi_scatter_w(const GemmScatter &S, int M, int row_base, int l,
+                                              int m, int c0, const uint32_t (&r)[32],
+                                              bool stage, const EpiScratch &x) {
   const int lane = threadIdx.x & 31;
-  const int S_ = (S.L + 1) * (S.L + 1);
   const int my_key = x.keys[lane];
+  __syncwarp();  // the previous chunk's reads of T and Dw are done
+  if (S.gate && my_key >= 0) {
+    const float4 *gp =
+        reinterpret_cast<const float4 *>(S.gate + (int64_t)(row_base + lane) * S.C + c0);
+#pragma unroll
+    for (int k4 = 0; k4 < 8; ++k4) {
+      const float4 g = __ldg(gp + k4);
+      x.T[lane * 33 + 4 * k4 + 0] = __uint_as_float(r[4 * k4 + 0]) * g.x;
+      x.T[lane * 33 + 4 * k4 + 1] = __uint_as_float(r[4 * k4 + 1]) * g.y;
+      x.T[lane * 33 + 4 * k4 + 2] = __uint_as_float(r[4 * k4 + 2]) * g.z;
+      x.T[lane * 33 + 4 * k4 + 3] = __uint_as_float(r[4 * k4 + 3]) * g.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) x.T[lane * 33 + k] = __uint_as_float(r[k]);
+  }
+  if (stage) epi_stage_d<W>(S, M, row_base, l * (4 * l * l - 1) / 3 + (m + l) * W, x);
+  __syncwarp();
+  // lane = channel from here on
+  const int c = c0 + lane;
+  const int S_ = (S.L + 1) * (S.L + 1);
   const int prev_key = lane ? x.keys[lane - 1] : -2;
+  const int nvalid = __popc(__ballot_sync(0xffffffffu, my_key >= 0));  // a prefix of the warp
   unsigned starts = __ballot_sync(0xffffffffu, my_key != prev_key && my_key >= 0);
   while (starts) {
     const int s0 = __ffs(starts) - 1;
     starts &= starts - 1;
-    const int s1 = starts ? __ffs(starts) - 1 : 32;
+    const int s1 = starts ? __ffs(starts) - 1 : nvalid;
     const int key = x.keys[s0];
     float acc[W];
 #pragma unroll
     for (int k = 0; k < W; ++k) acc[k] = 0.f;
 #pragma unroll 4
     for (int el = s0; el < s1; ++el) {
-      if (x.keys[el] < 0) break;  // past the end of the chunk (uniform)
       const float v = x.T[el * 33 + lane];
       const float4 *d4 = reinterpret_cast<const float4 *>(x.Dw + el * 16);
 #pragma unroll
@@ -163,39 +191,18 @@ __device__ __forceinline__ void epi_rotate_reduce(const GemmScatter &S, int row_
   }
 }
 
-// One warp, one 32-column chunk (channels c0.. of edge-frame row (l, m)) of
-// its 32 edges: adds sum_e D_e^l[m][m'] g_e[c] v_e[c] onto
-// out[key_e][(l, m')][c], one coalesced atomic per (node run, m', c).
-// keys and Dw must be staged; r holds one edge's 32 values per lane.
-__device__ __forceinline__ void epi_scatter_chunk(const GemmParams &p, int row_base, int l, int c0,
-                                                  const uint32_t (&r)[32], const EpiScratch &x) {
-  const GemmScatter &S = p.sc;
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int k = 0; k < 32; ++k) x.T[lane * 33 + k] = __uint_as_float(r[k]);
-  __syncwarp();
-  // lane = channel from here on
-  const int c = c0 + lane;
-  if (S.gate) {
-    // all 32 gate loads in flight at once (coalesced per edge), then scale
-    float g[32];
-#pragma unroll
-    for (int el = 0; el < 32; ++el)
-      g[el] = (x.keys[el] >= 0) ? S.gate[(int64_t)(row_base + el) * S.C + c] : 0.f;
-#pragma unroll
-    for (int el = 0; el < 32; ++el) x.T[el * 33 + lane] *= g[el];
-    __syncwarp();
-  }
+__device__ __forceinline__ void epi_scatter_chunk(const GemmScatter &S, int M, int row_base, int l,
+                                                  int m, int c0, const uint32_t (&r)[32],
+                                                  bool stage, const EpiScratch &x) {
   switch (2 * l + 1) {
-    case 1: epi_rotate_reduce<1>(S, row_base, l, c, x); break;
-    case 3: epi_rotate_reduce<3>(S, row_base, l, c, x); break;
-    case 5: epi_rotate_reduce<5>(S, row_base, l, c, x); break;
-    case 7: epi_rotate_reduce<7>(S, row_base, l, c, x); break;
-    case 9: epi_rotate_reduce<9>(S, row_base, l, c, x); break;
-    case 11: epi_rotate_reduce<11>(S, row_base, l, c, x); break;
-    default: epi_rotate_reduce<13>(S, row_base, l, c, x); break;
+    case 1: epi_scatter_w<1>(S, M, row_base, l, m, c0, r, stage, x); break;
+    case 3: epi_scatter_w<3>(S, M, row_base, l, m, c0, r, stage, x); break;
+    case 5: epi_scatter_w<5>(S, M, row_base, l, m, c0, r, stage, x); break;
+    case 7: epi_scatter_w<7>(S, M, row_base, l, m, c0, r, stage, x); break;
+    case 9: epi_scatter_w<9>(S, M, row_base, l, m, c0, r, stage, x); break;
+    case 11: epi_scatter_w<11>(S, M, row_base, l, m, c0, r, stage, x); break;
+    default: epi_scatter_w<13>(S, M, row_base, l, m, c0, r, stage, x); break;
   }
-  __syncwarp();
 }
 
 // BK = 32 uses the 64-byte swizzle (4 stages of 48 KB with hi/lo planes),
@@ -437,18 +444,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (col0 >= G.N) break;  // warp-uniform
         uint32_t r[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * GEMM_BN + cc * 32, r);
-        if (SCATTER && p.scatter) {
-          const int j = col0 / p.sc.C, c0 = col0 % p.sc.C;
-          int l, m;
-          gemm_row_lm(p.sc.L, G.mgroup, j, l, m);
-          if (j != staged) {
-            __syncwarp();
-            epi_stage_d(p, G, row_base, l, m, xs);
-            staged = j;
-          }
-          __syncwarp();
-          epi_scatter_chunk(p, row_base, l, c0, r, xs);
-        }
+        // store first (when asked), so that r is dead before the reduction
         if (p.store && row < G.M) {
           float *crow = Cg + static_cast<long long>(row) * G.ldc + col0;
           const bool vec = (col0 + 32 <= G.N) && ((reinterpret_cast<uintptr_t>(crow) & 15) == 0);
@@ -481,6 +477,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               crow[j] = p.beta ? crow[j] + v : v;
             }
           }
+        }
+        if (SCATTER && p.scatter) {
+          const int j = col0 / p.sc.C, c0 = col0 % p.sc.C;
+          int l, m;
+          gemm_row_lm(p.sc.L, G.mgroup, j, l, m);
+          epi_scatter_chunk(p.sc, G.M, row_base, l, m, c0, r, j != staged, xs);
+          staged = j;
         }
       }
       tc_fence_before();
