@@ -676,13 +676,16 @@ __global__ void k_unstack_grad(Layout y, BlockOffsets bo, const float *__restric
 // the two products.  h_x, h_y give the frame part of dL/dr.
 // ---------------------------------------------------------------------------
 // PART: 3 = both sides in one pass; 1 = output side only (writes Gg and h);
-// 2 = input side only (adds its share to h).
+// 2 = input side only (adds its share to h).  With gv_hi, the output side
+// also writes g * (D G[dst]) on the kept rows as the transposed product's
+// operand planes (what rotation on gather of G would write).
 template <typename TX, int MM, int LC = -1, int PART = 3>
 __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MINB) k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
                              const float *__restrict__ D, const float *__restrict__ gate,
                              const float *__restrict__ G, const TX *__restrict__ X,
                              const float *__restrict__ V, const float *__restrict__ Ga,
-                             float *__restrict__ Gg, float *__restrict__ h) {
+                             float *__restrict__ Gg, float *__restrict__ h,
+                             __nv_bfloat16 *__restrict__ gv_hi, __nv_bfloat16 *__restrict__ gv_lo) {
   constexpr int W = MM + 1;  // widest |m| needed by the generators
   extern __shared__ float sDall[];  // [warps][dsz]
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
@@ -723,6 +726,12 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
         for (int m = -mm; m <= mm; ++m) {
           int g, j;
           lm_group_row(y, l, m, g, j);
+          if (gv_hi) {  // the output-side operand g * (D G[dst]) of the transposed product
+            const int64_t col = (int64_t)i * y.KG + y.kout_off[g] + j * y.co + c;
+            store_split4(gv_hi + col, gv_lo ? gv_lo + col : nullptr,
+                         make_float4(gv.x * b[m + W].x, gv.y * b[m + W].y, gv.z * b[m + W].z,
+                                     gv.w * b[m + W].w));
+          }
           const float4 v = load4(Vi + y.kout_off[g] + j * y.co + c);
           gg.x += b[m + W].x * v.x;
           gg.y += b[m + W].y * v.y;
@@ -744,6 +753,13 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
         }
       });
       *reinterpret_cast<float4 *>(Gg + (int64_t)i * y.co + c) = gg;
+    }
+    if ((PART & 1) && gv_hi) {
+      for (int g = 0; g < y.ng; ++g)
+        for (int k = y.rows[g] * y.co + 4 * lane; k < y.Kout_pad[g]; k += 128) {
+          const int64_t col = (int64_t)i * y.KG + y.kout_off[g] + k;
+          store_split4(gv_hi + col, gv_lo ? gv_lo + col : nullptr, make_float4(0.f, 0.f, 0.f, 0.f));
+        }
     }
     // input side
     const TX *Xn = X + (int64_t)r.src * y.S * y.ci;

@@ -773,6 +773,42 @@ so2_status rad_grads(Ctx &c, int M, const float *Ag, const float *Bg, const floa
   return SO2_OK;
 }
 
+// Per-edge gradient terms of the backward (see k_edge_terms): part 1 the
+// output side (Gg, h; with write_gv also the transposed product's operand
+// planes), part 2 the input side (adds to h).
+so2_status edge_terms(Ctx &c, int M, int part, const void *x, const float *grad_out,
+                      bool write_gv) {
+  const Plan &P = c.P;
+  const Layout &y = P.y;
+  ProfScope ps(5, c.s);
+  const int sm = 8 * y.dsz * 4;
+  const int g = warp_grid(M, 8);
+  const EdgeRec *rec = at<EdgeRec>(c.ws, P.rec);
+  const float *Dp = at<float>(c.ws, P.D), *gate = at<float>(c.ws, P.gate);
+  const float *Vp = at<float>(c.ws, P.V), *Gap = at<float>(c.ws, P.Ga);
+  float *Ggp = at<float>(c.ws, P.Gg), *hp = at<float>(c.ws, P.h);
+  __nv_bfloat16 *gh = write_gv ? at<__nv_bfloat16>(c.ws, P.gv_hi) : nullptr;
+  __nv_bfloat16 *gl = write_gv && P.split ? at<__nv_bfloat16>(c.ws, P.gv_lo) : nullptr;
+#define SO2_ET_LAUNCH(TX)                                                                    \
+  DISPATCH_LM(y.L, y.mmax,                                                                   \
+              /* all levels inlined spills at lmax 6: runtime-degree kernel there */          \
+              constexpr int LE = (LC >= 0 && LC <= 4) ? LC : -1;                              \
+              if (part == 1) k_edge_terms<TX, MM, LE, 1><<<g, 256, sm, c.s>>>(                 \
+                  y, M, rec, Dp, gate, grad_out, static_cast<const TX *>(x), Vp, Gap, Ggp, hp, \
+                  gh, gl);                                                                    \
+              else k_edge_terms<TX, MM, LE, 2><<<g, 256, sm, c.s>>>(                           \
+                  y, M, rec, Dp, gate, grad_out, static_cast<const TX *>(x), Vp, Gap, Ggp, hp, \
+                  nullptr, nullptr);)
+  if (P.xbf16) {
+    SO2_ET_LAUNCH(__nv_bfloat16)
+  } else {
+    SO2_ET_LAUNCH(float)
+  }
+#undef SO2_ET_LAUNCH
+  CKL();
+  return SO2_OK;
+}
+
 // Library-owned scratch for so2conv_forward_noalloc (see its declaration).
 static __device__ __align__(256) unsigned char g_noalloc_ws[SO2_NOALLOC_WORKSPACE_BYTES];
 constexpr int NOALLOC_MAX_DEVICES = 64;
@@ -872,9 +908,14 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
     const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
     if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 0, prm)) != SO2_OK) return r;
     if ((r = rotate_x(c, M, x, P.xbf16)) != SO2_OK) return r;
-    // Gv = g * (D G[dst]) on the kept rows
-    if ((r = rotate_g(c, M, grad_out, 0, arr(at<float>(ws, P.gate)))) != SO2_OK) return r;
-    if (need_v && (r = gemm_v(c, M)) != SO2_OK) return r;
+    // Gv = g * (D G[dst]) on the kept rows: written by the output-side edge
+    // terms when they run (they rotate G[dst] anyway), else by rotation on gather
+    if (need_v) {
+      if ((r = gemm_v(c, M)) != SO2_OK) return r;
+      if ((r = edge_terms(c, M, 1, x, grad_out, true)) != SO2_OK) return r;
+    } else if ((r = rotate_g(c, M, grad_out, 0, arr(at<float>(ws, P.gate)))) != SO2_OK) {
+      return r;
+    }
     const bool fuse_gx = grad_x && fusable(y.ci);
     if (need_ga) {
       const GemmScatter sc = make_scatter(c, nullptr, grad_x, y.ci);
@@ -892,34 +933,7 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
             SO2_OK)
       return r;
     if (need_v) {
-      {
-        ProfScope ps(5, c.s);
-        const int sm = 8 * y.dsz * 4;
-        const int g = warp_grid(M, 8);
-        EdgeRec *rec = at<EdgeRec>(ws, P.rec);
-        float *Dp = at<float>(ws, P.D), *gate = at<float>(ws, P.gate), *Vp = at<float>(ws, P.V);
-        float *Gap = at<float>(ws, P.Ga), *Ggp = at<float>(ws, P.Gg), *hp = at<float>(ws, P.h);
-        if (P.xbf16) {
-          const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
-          DISPATCH_LM(y.L, y.mmax,
-                      // all levels inlined spills at lmax 6: runtime-degree kernel there
-                      constexpr int LE = (LC >= 0 && LC <= 4) ? LC : -1;
-                      k_edge_terms<__nv_bfloat16, MM, LE, 1><<<g, 256, sm, c.s>>>(
-                          y, M, rec, Dp, gate, grad_out, xb, Vp, Gap, Ggp, hp);
-                      k_edge_terms<__nv_bfloat16, MM, LE, 2><<<g, 256, sm, c.s>>>(
-                          y, M, rec, Dp, gate, grad_out, xb, Vp, Gap, Ggp, hp););
-        } else {
-          const float *xf = static_cast<const float *>(x);
-          DISPATCH_LM(y.L, y.mmax,
-                      // all levels inlined spills at lmax 6: runtime-degree kernel there
-                      constexpr int LE = (LC >= 0 && LC <= 4) ? LC : -1;
-                      k_edge_terms<float, MM, LE, 1><<<g, 256, sm, c.s>>>(
-                          y, M, rec, Dp, gate, grad_out, xf, Vp, Gap, Ggp, hp);
-                      k_edge_terms<float, MM, LE, 2><<<g, 256, sm, c.s>>>(
-                          y, M, rec, Dp, gate, grad_out, xf, Vp, Gap, Ggp, hp););
-        }
-      }
-      CKL();
+      if (grad_edge_vec && (r = edge_terms(c, M, 2, x, grad_out, false)) != SO2_OK) return r;
       if (grad_edge_vec) {
         ProfScope ps(5, c.s);
         k_edge_final<<<warp_grid(M, 8), 256, 0, c.s>>>(y, desc->rbf_cutoff, M,
