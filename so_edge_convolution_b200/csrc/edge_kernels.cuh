@@ -239,27 +239,42 @@ __device__ __forceinline__ float rbf_val(float d, int k, const Layout &y, float 
 }
 
 // g[i][c'] = b[c'] + sum_k w_rad[k][c'] phi_k(d_i).  A block takes
-// GATE_EDGES edges: the basis values are computed once per edge into shared
-// memory, then threads over channels form the gates.
-constexpr int GATE_EDGES = 16;
+// GATE_EDGES edges: the basis values go to shared memory basis-major
+// (phi[k][i]), then each thread keeps one channel's GATE_EDGES sums in
+// registers, reading each w_rad[k][c'] once and four basis values per
+// shared-memory load.
+constexpr int GATE_EDGES = 32;
 __global__ void k_edge_gate(Layout y, float cutoff, int M, const float *__restrict__ geo,
                             const float *__restrict__ w_rad, const float *__restrict__ b_rad,
                             float *__restrict__ gate) {
-  extern __shared__ float phi[];  // [GATE_EDGES][nr]
+  extern __shared__ float4 phi4[];  // [nr][GATE_EDGES / 4]
+  float *phi = reinterpret_cast<float *>(phi4);
   const int i0 = blockIdx.x * GATE_EDGES;
   const int n = (M - i0) < GATE_EDGES ? (M - i0) : GATE_EDGES;
-  for (int t = threadIdx.x; t < n * y.nr; t += blockDim.x) {
-    const int i = t / y.nr, k = t % y.nr;
-    phi[t] = rbf_val(geo[(int64_t)(i0 + i) * GEO], k, y, cutoff);
+  for (int t = threadIdx.x; t < y.nr * GATE_EDGES; t += blockDim.x) {
+    const int k = t / GATE_EDGES, i = t % GATE_EDGES;
+    phi[t] = (i < n) ? rbf_val(geo[(int64_t)(i0 + i) * GEO], k, y, cutoff) : 0.f;
   }
   __syncthreads();
   for (int c = threadIdx.x; c < y.co; c += blockDim.x) {
+    float acc[GATE_EDGES];
     const float b = b_rad[c];
-    for (int i = 0; i < n; ++i) {
-      float acc = b;
-      for (int k = 0; k < y.nr; ++k) acc += w_rad[k * y.co + c] * phi[i * y.nr + k];
-      gate[(int64_t)(i0 + i) * y.co + c] = acc;
+#pragma unroll
+    for (int i = 0; i < GATE_EDGES; ++i) acc[i] = b;
+    for (int k = 0; k < y.nr; ++k) {
+      const float w = w_rad[k * y.co + c];
+#pragma unroll
+      for (int q = 0; q < GATE_EDGES / 4; ++q) {
+        const float4 f = phi4[k * (GATE_EDGES / 4) + q];
+        acc[4 * q + 0] += f.x * w;
+        acc[4 * q + 1] += f.y * w;
+        acc[4 * q + 2] += f.z * w;
+        acc[4 * q + 3] += f.w * w;
+      }
     }
+#pragma unroll
+    for (int i = 0; i < GATE_EDGES; ++i)
+      if (i < n) gate[(int64_t)(i0 + i) * y.co + c] = acc[i];
   }
 }
 
@@ -471,6 +486,116 @@ __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO
       for (int k = width + 4 * lane; k < col_pad[g]; k += 128)
         store_split4(oh + col_off[g] + k, ol ? ol + col_off[g] + k : nullptr,
                      make_float4(0.f, 0.f, 0.f, 0.f));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Inverse rotation on reduction, node-centric, one term: for every node n
+// whose sorted segment meets this chunk and every degree l,
+//   out[n][(l, m')][c] += sum_{chunk edges i of n} sum_m D_i^l[m][m'] k_i[c] F[i][(l, m)][c]
+// with k the optional per-edge channel coefficient (the gate) and F the
+// product rows (grouped layout, row stride ld).  One warp per (node, l),
+// four channels per lane, the node's sums in registers; each output element
+// has one writer per launch and the chunks run in stream order, so the sum
+// order is fixed and no atomics are needed.
+// ---------------------------------------------------------------------------
+template <int MM, int l>
+__device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int C,
+                                             const int *col_off, const float *__restrict__ D,
+                                             const float *__restrict__ F, int ld,
+                                             const float *__restrict__ coef, float *o, int c,
+                                             bool act) {
+  constexpr int w = 2 * l + 1;
+  constexpr int mm = MM < l ? MM : l;  // kept rows |m| <= mm
+  const int lane = threadIdx.x & 31;
+  float4 acc[w];
+#pragma unroll
+  for (int k = 0; k < w; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  int cols[2 * mm + 1];
+#pragma unroll
+  for (int m = -mm; m <= mm; ++m) {
+    int g, j;
+    lm_group_row(y, l, m, g, j);
+    cols[m + mm] = col_off[g] + j * C + c;
+  }
+  for (int i = b; i < e; ++i) {
+    // the rows m of D^l this edge needs, one entry per lane, then broadcast
+    constexpr int nd = (2 * mm + 1) * w;
+    const float *Dl = D + (int64_t)i * y.dsz + dblock_off(l) + (l - mm) * w;
+    float dreg[(nd + 31) / 32];
+#pragma unroll
+    for (int u = 0; u < (nd + 31) / 32; ++u)
+      dreg[u] = (lane + 32 * u < nd) ? __ldg(Dl + lane + 32 * u) : 0.f;
+    float4 kc = make_float4(1.f, 1.f, 1.f, 1.f);
+    if (coef && act) kc = __ldg(reinterpret_cast<const float4 *>(coef + (int64_t)i * C + c));
+    float4 z[2 * mm + 1];
+#pragma unroll
+    for (int m = 0; m < 2 * mm + 1; ++m) {
+      const float4 f = act ? __ldg(reinterpret_cast<const float4 *>(F + (int64_t)i * ld + cols[m]))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      z[m] = make_float4(kc.x * f.x, kc.y * f.y, kc.z * f.z, kc.w * f.w);
+    }
+#pragma unroll
+    for (int m = 0; m < 2 * mm + 1; ++m) {
+#pragma unroll
+      for (int mp = 0; mp < w; ++mp) {
+        const int q = m * w + mp;  // entry (m - mm + l, mp) of the kept rows
+        const float dv = __shfl_sync(0xffffffffu, dreg[q >> 5], q & 31);
+        acc[mp].x += dv * z[m].x;
+        acc[mp].y += dv * z[m].y;
+        acc[mp].z += dv * z[m].z;
+        acc[mp].w += dv * z[m].w;
+      }
+    }
+  }
+  if (!act) return;
+#pragma unroll
+  for (int mp = 0; mp < w; ++mp) {
+    float4 *dst = reinterpret_cast<float4 *>(o + (l * l + mp) * C + c);
+    float4 v = *dst;
+    v.x += acc[mp].x;
+    v.y += acc[mp].y;
+    v.z += acc[mp].z;
+    v.w += acc[mp].w;
+    *dst = v;
+  }
+}
+
+template <int MM>
+__global__ void __launch_bounds__(256, 2) k_reduce_nodes(Layout y, int64_t e0, int M,
+                                                      const EdgeRec *__restrict__ rec,
+                                                      const int *__restrict__ offsets,
+                                                      const float *__restrict__ D,
+                                                      const float *__restrict__ F, int ld,
+                                                      const float *__restrict__ coef, int side,
+                                                      float *__restrict__ out) {
+  if (M <= 0) return;
+  const int C = side ? y.co : y.ci;
+  const int *col_off = side ? y.kout_off : y.kin_off;
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  const int n_first = rec[0].key, n_last = rec[M - 1].key;
+  const int items = (n_last - n_first + 1) * (y.L + 1);
+  for (int it = blockIdx.x * wpb + (threadIdx.x >> 5); it < items; it += gridDim.x * wpb) {
+    const int n = n_first + it / (y.L + 1), l = it % (y.L + 1);
+    int b = offsets[n] - static_cast<int>(e0), e = offsets[n + 1] - static_cast<int>(e0);
+    b = b < 0 ? 0 : b;
+    e = e > M ? M : e;
+    if (b >= e) continue;
+    float *o = out + (int64_t)n * y.S * C;
+    // warp-uniform channel loop (the level bodies shuffle across the warp)
+    for (int c0 = 0; c0 < C; c0 += 128) {
+      const int c = c0 + 4 * lane;
+      const bool act = c < C;  // C is a multiple of 16, so c + 3 < C too
+      switch (l) {
+        case 0: reduce_level<MM, 0>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
+        case 1: reduce_level<MM, 1>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
+        case 2: reduce_level<MM, 2>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
+        case 3: reduce_level<MM, 3>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
+        case 4: reduce_level<MM, 4>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
+        case 5: reduce_level<MM, 5>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
+        default: reduce_level<MM, 6>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
+      }
     }
   }
 }

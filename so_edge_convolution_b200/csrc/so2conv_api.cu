@@ -710,7 +710,10 @@ so2_status gemm_v(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store 
 
 // The fused gate + inverse rotation + reduction epilogue needs whole 32-wide
 // channel chunks inside one edge-frame row.
-bool fusable(int C) { return C % 32 == 0; }
+#ifndef SO2_FUSE_BF16
+#define SO2_FUSE_BF16 1
+#endif
+bool fusable(int C, bool split) { return C % 32 == 0 && (split || SO2_FUSE_BF16); }
 
 GemmScatter make_scatter(Ctx &c, const float *gate, float *out, int C) {
   GemmScatter sc;
@@ -743,6 +746,27 @@ so2_status scatter(Ctx &c, int64_t e0, int M, const ScatterTerms &t, int side,
               if (ok) k_scatter_nodes<MM><<<grid_for(M, 1), threads, smem, c.s>>>(
                   y, e0, M, rec, off, D, t, side, omega, out));
   if (!ok) return SO2_ERR_CUDA;
+  CKL();
+  return SO2_OK;
+}
+
+// One-term node-centric reduction (see k_reduce_nodes): out += D^T (k * F)
+// per node; falls back to the general kernel when out is not 16-byte aligned.
+so2_status reduce_nodes(Ctx &c, int64_t e0, int M, const float *F, int ld, const float *coef,
+                        int side, float *out) {
+  const Plan &P = c.P;
+  const Layout &y = P.y;
+  if (reinterpret_cast<uintptr_t>(out) & 15) {
+    ScatterTerms t{};
+    t.F[0] = F;
+    t.ld[0] = ld;
+    t.A[0] = coef ? Coef{coef, 2} : Coef{nullptr, 1};
+    return scatter(c, e0, M, t, side, nullptr, out);
+  }
+  ProfScope ps(7, c.s);
+  DISPATCH_MM(y.mmax, k_reduce_nodes<MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                          y, e0, M, at<EdgeRec>(c.ws, P.rec), at<int>(c.ws, P.offsets),
+                          at<float>(c.ws, P.D), F, ld, coef, side, out));
   CKL();
   return SO2_OK;
 }
@@ -858,14 +882,14 @@ so2_status so2conv_forward(const so2conv_desc *desc, int64_t N, int64_t E, const
     const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
     if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 1, prm)) != SO2_OK) return r;
     if ((r = rotate_x(c, M, x, P.xbf16)) != SO2_OK) return r;
-    if (fusable(y.co)) {
+    if (fusable(y.co, P.split)) {
       // product, gate, inverse rotation and reduction in one kernel
       const GemmScatter sc = make_scatter(c, at<float>(ws, P.gate), out, y.co);
       if ((r = gemm_v(c, M, &sc, false)) != SO2_OK) return r;
     } else {
       if ((r = gemm_v(c, M)) != SO2_OK) return r;
-      if ((r = scatter(c, e0, M, one_term(at<float>(ws, P.V), y.KG, arr(at<float>(ws, P.gate))),
-                       1, nullptr, out)) != SO2_OK)
+      if ((r = reduce_nodes(c, e0, M, at<float>(ws, P.V), y.KG, at<float>(ws, P.gate), 1, out)) !=
+          SO2_OK)
         return r;
     }
   }
@@ -916,7 +940,7 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
     } else if ((r = rotate_g(c, M, grad_out, 0, arr(at<float>(ws, P.gate)))) != SO2_OK) {
       return r;
     }
-    const bool fuse_gx = grad_x && fusable(y.ci);
+    const bool fuse_gx = grad_x && fusable(y.ci, P.split);
     if (need_ga) {
       const GemmScatter sc = make_scatter(c, nullptr, grad_x, y.ci);
       if ((r = gemm_ga(c, M, fuse_gx ? &sc : nullptr, grad_edge_vec != nullptr || !fuse_gx)) !=
@@ -929,8 +953,7 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
       if ((r = gemm_dw(c, M, 0, 0)) != SO2_OK) return r;
     }
     if (grad_x && !fuse_gx &&
-        (r = scatter(c, e0, M, one_term(at<float>(ws, P.Ga), y.KA, ONE), 0, nullptr, grad_x)) !=
-            SO2_OK)
+        (r = reduce_nodes(c, e0, M, at<float>(ws, P.Ga), y.KA, nullptr, 0, grad_x)) != SO2_OK)
       return r;
     if (need_v) {
       if (grad_edge_vec && (r = edge_terms(c, M, 2, x, grad_out, false)) != SO2_OK) return r;
