@@ -181,6 +181,17 @@ so2_status so2conv_forward_noalloc(const so2conv_desc *desc, int64_t n_nodes,
  * points, all devices).  A plain counter, not thread safe. */
 long long so2conv_launch_count(void);
 
+/* Edges per chunk of per-edge intermediates (records, frames, Wigner-D,
+ * operands and products live in the workspace for one chunk at a time; the
+ * double backward uses half).  Larger chunks mean fewer, fuller launches and
+ * a larger workspace.  n = 0 restores the default (65,536); otherwise n is
+ * rounded up to a multiple of 256 (at least 256).  Returns
+ * SO2_ERR_INVALID_ARG for n < 0 or n > 2^22.  Process-wide and not thread
+ * safe: query so2conv_workspace_size after changing it, and do not change it
+ * while a call is being issued. */
+so2_status so2conv_set_max_chunk_edges(int64_t n);
+int64_t so2conv_max_chunk_edges(void);
+
 /* Live timing of the library's launches.  so2conv_profile_enable(1) clears
  * the record and starts recording a pair of CUDA events around every
  * tensor-core launch, on the stream it is launched on; (2) does the same and

@@ -75,6 +75,10 @@ def load():
     lib.so2conv_forward_noalloc.restype = ctypes.c_int
     lib.so2conv_launch_count.argtypes = []
     lib.so2conv_launch_count.restype = ctypes.c_longlong
+    lib.so2conv_set_max_chunk_edges.argtypes = [ctypes.c_int64]
+    lib.so2conv_set_max_chunk_edges.restype = ctypes.c_int
+    lib.so2conv_max_chunk_edges.argtypes = []
+    lib.so2conv_max_chunk_edges.restype = ctypes.c_int64
     lib.so2conv_profile_enable.argtypes = [ctypes.c_int]
     lib.so2conv_profile_enable.restype = None
     lib.so2conv_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
@@ -238,6 +242,14 @@ def edge_frames(lmax, edge_vec):
                                       _stream(edge_vec.device))
     _check_call(code, "so2conv_edge_frames")
     return R.view(E, 3, 3), D
+
+
+def set_max_chunk_edges(n):
+    """so2conv_set_max_chunk_edges: edges per chunk of per-edge intermediates
+    (0 restores the default); returns the value now in force."""
+    lib = load()
+    _check_call(lib.so2conv_set_max_chunk_edges(int(n)), "so2conv_set_max_chunk_edges")
+    return int(lib.so2conv_max_chunk_edges())
 
 
 def launch_count():

@@ -500,6 +500,13 @@ __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO
 // has one writer per launch and the chunks run in stream order, so the sum
 // order is fixed and no atomics are needed.
 // ---------------------------------------------------------------------------
+#ifndef SO2_RN_MINB  // resident 256-thread blocks per SM for k_reduce_nodes
+#define SO2_RN_MINB 2
+#endif
+#ifndef SO2_RN_UNROLL  // edges per unrolled step of its edge loop
+#define SO2_RN_UNROLL 1
+#endif
+constexpr int kReduceUnroll = SO2_RN_UNROLL;
 template <int MM, int l>
 __device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int C,
                                              const int *col_off, const float *__restrict__ D,
@@ -519,6 +526,7 @@ __device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int 
     lm_group_row(y, l, m, g, j);
     cols[m + mm] = col_off[g] + j * C + c;
   }
+#pragma unroll kReduceUnroll
   for (int i = b; i < e; ++i) {
     // the rows m of D^l this edge needs, one entry per lane, then broadcast
     constexpr int nd = (2 * mm + 1) * w;
@@ -563,7 +571,7 @@ __device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int 
 }
 
 template <int MM>
-__global__ void __launch_bounds__(256, 2) k_reduce_nodes(Layout y, int64_t e0, int M,
+__global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes(Layout y, int64_t e0, int M,
                                                       const EdgeRec *__restrict__ rec,
                                                       const int *__restrict__ offsets,
                                                       const float *__restrict__ D,

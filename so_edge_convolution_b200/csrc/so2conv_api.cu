@@ -18,7 +18,12 @@ using namespace so2;
 
 namespace {
 
-constexpr int CHUNK_MAX = 32768;  // edges per chunk of per-edge intermediates
+// Edges per chunk of per-edge intermediates (the workspace grows with it);
+// so2conv_set_max_chunk_edges changes it for the process.
+#ifndef SO2_CHUNK_MAX
+#define SO2_CHUNK_MAX 65536
+#endif
+int g_chunk_max = SO2_CHUNK_MAX;
 
 // --------------------------------------------------------------------------
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -131,7 +136,7 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
   p.E = E;
   p.split = d->dtype == SO2_F32;
   p.xbf16 = d->dtype == SO2_BF16;
-  const int64_t cap = which == SO2_WS_DOUBLE_BACKWARD ? CHUNK_MAX / 2 : CHUNK_MAX;
+  const int64_t cap = which == SO2_WS_DOUBLE_BACKWARD ? g_chunk_max / 2 : g_chunk_max;
   const int64_t ch = E < cap ? E : cap;
   p.chunk = static_cast<int>(round_up(static_cast<int>(ch > 0 ? ch : 1), 128));
   const Layout &y = p.y;
@@ -1171,6 +1176,14 @@ so2_status so2conv_check(void *ws, so2_stream_t stream) {
 }
 
 long long so2conv_launch_count(void) { return g_launches; }
+
+so2_status so2conv_set_max_chunk_edges(int64_t n) {
+  if (n < 0 || n > (1 << 22)) return SO2_ERR_INVALID_ARG;
+  g_chunk_max = n == 0 ? SO2_CHUNK_MAX : round_up(static_cast<int>(n) < 256 ? 256 : static_cast<int>(n), 256);
+  return SO2_OK;
+}
+
+int64_t so2conv_max_chunk_edges(void) { return g_chunk_max; }
 
 void so2conv_profile_enable(int on) {
   g_prof.on = on < 0 ? 0 : (on > 2 ? 2 : on);

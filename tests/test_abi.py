@@ -53,6 +53,22 @@ def test_workspace_sizes(lib):
     assert B.workspace_size(bad, 10, 10, B.WS_FORWARD) == 0
 
 
+def test_chunk_size_knob(lib):
+    d = B.make_desc(4, 2, 128, 128, 16, 6.0, B.SO2_F32)
+    assert B.set_max_chunk_edges(0) == 65536
+    big = B.workspace_size(d, 2000, 200000, B.WS_BACKWARD)
+    try:
+        assert B.set_max_chunk_edges(1000) == 1024
+        small = B.workspace_size(d, 2000, 200000, B.WS_BACKWARD)
+        assert 0 < small < big
+        assert lib.so2conv_set_max_chunk_edges(-1) == 1  # SO2_ERR_INVALID_ARG
+        assert lib.so2conv_set_max_chunk_edges(1 << 23) == 1
+        assert lib.so2conv_max_chunk_edges() == 1024
+    finally:
+        B.set_max_chunk_edges(0)
+    assert B.workspace_size(d, 2000, 200000, B.WS_BACKWARD) == big
+
+
 def _fwd(lib, desc, N=4, E=3, x=1, ei=1, ev=1, w=1, ws=1, nbytes=None):
     P = lambda f: ctypes.c_void_p(0x1000 if f else 0)  # noqa: E731 (never dereferenced)
     prm = B.Params(0x1000 if w else 0, 0x1000, 0x1000)

@@ -117,9 +117,23 @@ def _small(L=3, M=2, C=32, n=300, nb=30, seed=0, bf16=False):
     return p
 
 
+@pytest.fixture(autouse=True)
+def _small_chunks_for_chunked_cases(request):
+    # cases named *_chunks run with 2,048-edge chunks (1,024 in the double
+    # backward), so that small graphs cross several chunk boundaries
+    params = getattr(getattr(request.node, "callspec", None), "params", {})
+    chunked = "chunks" in str(params.get("name", ""))
+    if chunked:
+        B.set_max_chunk_edges(2048)
+    yield
+    if chunked:
+        B.set_max_chunk_edges(0)
+
+
 CASES = [
     ("tiny", lambda: synth.make_problem("tiny")),
-    ("L3M2C32_two_chunks", lambda: _small(L=3, M=2, C=32, n=300, nb=30)),  # 9000 edges
+    ("L3M2C32_chunks", lambda: _small(L=3, M=2, C=32, n=300, nb=30)),  # 9,000 edges, 5 chunks
+    ("L4M2C128_bf16_chunks", lambda: _small(L=4, M=2, C=128, n=180, nb=25, seed=6, bf16=True)),
     ("L4M2C128_ragged", lambda: _small(L=4, M=2, C=128, n=150, nb=23, seed=1)),
     ("L2M0C16", lambda: _small(L=2, M=0, C=16, n=100, nb=11, seed=2)),
     ("L6M2C48_bf16", lambda: _small(L=6, M=2, C=48, n=120, nb=17, seed=3, bf16=True)),
@@ -237,7 +251,7 @@ def test_device_reports_bad_index_and_zero_length_edge():
 DB_CASES = [
     ("tiny", lambda: synth.make_problem("tiny")),
     ("L3M2C32", lambda: _small(L=3, M=2, C=32, n=150, nb=20, seed=12)),
-    ("L2M1C16_two_chunks", lambda: _small(L=2, M=1, C=16, n=600, nb=30, seed=13)),  # 18000 edges
+    ("L2M1C16_chunks", lambda: _small(L=2, M=1, C=16, n=600, nb=30, seed=13)),  # 18,000 edges
     ("L4M2C128_bf16", lambda: _small(L=4, M=2, C=128, n=60, nb=20, seed=14, bf16=True)),
 ]
 
@@ -280,3 +294,20 @@ def test_force_training_step_parity():
     want = oracle_double_backward(p, gg_edge_vec=gg_r)
     for k in ["d_w", "d_w_rad", "d_b_rad", "d_x"]:
         assert rel_err(got[k], want[k]) < 1e-4, k
+
+
+def test_chunk_size_does_not_change_results():
+    # the same problem in one chunk and in 1,024-edge chunks
+    p = _small(L=4, M=2, C=64, n=160, nb=24, seed=31)
+    out1, g1 = _gpu_forward(p).cpu(), {k: v.cpu() for k, v in _gpu_backward(p).items()}
+    try:
+        assert B.set_max_chunk_edges(1000) == 1024
+        out2, g2 = _gpu_forward(p).cpu(), {k: v.cpu() for k, v in _gpu_backward(p).items()}
+    finally:
+        B.set_max_chunk_edges(0)
+    # only the summation order differs (reductions onto nodes, the K split of
+    # the weight gradient); each order carries the split product's ~1e-5
+    # relative error
+    assert rel_err(out2, out1) < 5e-5
+    for k in g1:
+        assert rel_err(g2[k], g1[k]) < 5e-5, k
