@@ -503,57 +503,79 @@ __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO
 #ifndef SO2_RN_MINB  // resident 256-thread blocks per SM for k_reduce_nodes
 #define SO2_RN_MINB 2
 #endif
-#ifndef SO2_RN_UNROLL  // edges per unrolled step of its edge loop
-#define SO2_RN_UNROLL 1
-#endif
-constexpr int kReduceUnroll = SO2_RN_UNROLL;
+// Shared memory per warp of k_reduce_nodes: two buffers of the kept D rows
+// of one edge, rows padded to a multiple of 4 floats (at most 13 x 16).
+constexpr int RN_DBUF = 13 * 16;
+
 template <int MM, int l>
 __device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int C,
                                              const int *col_off, const float *__restrict__ D,
                                              const float *__restrict__ F, int ld,
                                              const float *__restrict__ coef, float *o, int c,
-                                             bool act) {
+                                             bool act, float *dsm) {
   constexpr int w = 2 * l + 1;
+  constexpr int wpad = (w + 3) / 4 * 4;
   constexpr int mm = MM < l ? MM : l;  // kept rows |m| <= mm
+  constexpr int nm = 2 * mm + 1;
+  constexpr int nd = nm * w;  // kept D entries of one edge
+  constexpr int nu = (nd + 31) / 32;
+  static_assert(nm * wpad <= RN_DBUF, "D staging buffer");
   const int lane = threadIdx.x & 31;
   float4 acc[w];
 #pragma unroll
   for (int k = 0; k < w; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  int cols[2 * mm + 1];
+  int cols[nm];
 #pragma unroll
   for (int m = -mm; m <= mm; ++m) {
     int g, j;
     lm_group_row(y, l, m, g, j);
     cols[m + mm] = col_off[g] + j * C + c;
   }
-#pragma unroll kReduceUnroll
-  for (int i = b; i < e; ++i) {
-    // the rows m of D^l this edge needs, one entry per lane, then broadcast
-    constexpr int nd = (2 * mm + 1) * w;
+  // one edge's inputs: its kept D entries (one per lane), coefficient, rows
+  float dreg[nu];
+  float4 kc, fz[nm];
+  auto load_edge = [&](int i) {
     const float *Dl = D + (int64_t)i * y.dsz + dblock_off(l) + (l - mm) * w;
-    float dreg[(nd + 31) / 32];
 #pragma unroll
-    for (int u = 0; u < (nd + 31) / 32; ++u)
-      dreg[u] = (lane + 32 * u < nd) ? __ldg(Dl + lane + 32 * u) : 0.f;
-    float4 kc = make_float4(1.f, 1.f, 1.f, 1.f);
+    for (int u = 0; u < nu; ++u) dreg[u] = (lane + 32 * u < nd) ? __ldg(Dl + lane + 32 * u) : 0.f;
+    kc = make_float4(1.f, 1.f, 1.f, 1.f);
     if (coef && act) kc = __ldg(reinterpret_cast<const float4 *>(coef + (int64_t)i * C + c));
-    float4 z[2 * mm + 1];
 #pragma unroll
-    for (int m = 0; m < 2 * mm + 1; ++m) {
-      const float4 f = act ? __ldg(reinterpret_cast<const float4 *>(F + (int64_t)i * ld + cols[m]))
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-      z[m] = make_float4(kc.x * f.x, kc.y * f.y, kc.z * f.z, kc.w * f.w);
+    for (int m = 0; m < nm; ++m)
+      fz[m] = act ? __ldg(reinterpret_cast<const float4 *>(F + (int64_t)i * ld + cols[m]))
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  if (b < e) load_edge(b);
+  for (int i = b; i < e; ++i) {
+    // stage this edge's D rows (buffer i & 1), scale its rows, fetch the next edge
+    float *Ds = dsm + (i & 1) * RN_DBUF;
+#pragma unroll
+    for (int u = 0; u < nu; ++u) {
+      const int k = lane + 32 * u;
+      if (k < nd) Ds[(k / w) * wpad + k % w] = dreg[u];
     }
+    float4 z[nm];
 #pragma unroll
-    for (int m = 0; m < 2 * mm + 1; ++m) {
+    for (int m = 0; m < nm; ++m)
+      z[m] = make_float4(kc.x * fz[m].x, kc.y * fz[m].y, kc.z * fz[m].z, kc.w * fz[m].w);
+    __syncwarp();
+    if (i + 1 < e) load_edge(i + 1);
 #pragma unroll
-      for (int mp = 0; mp < w; ++mp) {
-        const int q = m * w + mp;  // entry (m - mm + l, mp) of the kept rows
-        const float dv = __shfl_sync(0xffffffffu, dreg[q >> 5], q & 31);
-        acc[mp].x += dv * z[m].x;
-        acc[mp].y += dv * z[m].y;
-        acc[mp].z += dv * z[m].z;
-        acc[mp].w += dv * z[m].w;
+    for (int m = 0; m < nm; ++m) {
+#pragma unroll
+      for (int q = 0; q < wpad / 4; ++q) {
+        const float4 d = *reinterpret_cast<const float4 *>(Ds + m * wpad + 4 * q);
+        const float dv[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int mp = 4 * q + t;
+          if (mp < w) {
+            acc[mp].x += dv[t] * z[m].x;
+            acc[mp].y += dv[t] * z[m].y;
+            acc[mp].z += dv[t] * z[m].z;
+            acc[mp].w += dv[t] * z[m].w;
+          }
+        }
       }
     }
   }
@@ -578,10 +600,12 @@ __global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes(Layout y, int
                                                       const float *__restrict__ F, int ld,
                                                       const float *__restrict__ coef, int side,
                                                       float *__restrict__ out) {
+  __shared__ __align__(16) float dbuf[8][2 * RN_DBUF];
   if (M <= 0) return;
   const int C = side ? y.co : y.ci;
   const int *col_off = side ? y.kout_off : y.kin_off;
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  float *dsm = dbuf[threadIdx.x >> 5];
   const int n_first = rec[0].key, n_last = rec[M - 1].key;
   const int items = (n_last - n_first + 1) * (y.L + 1);
   for (int it = blockIdx.x * wpb + (threadIdx.x >> 5); it < items; it += gridDim.x * wpb) {
@@ -596,13 +620,13 @@ __global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes(Layout y, int
       const int c = c0 + 4 * lane;
       const bool act = c < C;  // C is a multiple of 16, so c + 3 < C too
       switch (l) {
-        case 0: reduce_level<MM, 0>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
-        case 1: reduce_level<MM, 1>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
-        case 2: reduce_level<MM, 2>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
-        case 3: reduce_level<MM, 3>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
-        case 4: reduce_level<MM, 4>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
-        case 5: reduce_level<MM, 5>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
-        default: reduce_level<MM, 6>(y, b, e, C, col_off, D, F, ld, coef, o, c, act); break;
+        case 0: reduce_level<MM, 0>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 1: reduce_level<MM, 1>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 2: reduce_level<MM, 2>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 3: reduce_level<MM, 3>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 4: reduce_level<MM, 4>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 5: reduce_level<MM, 5>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        default: reduce_level<MM, 6>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
       }
     }
   }

@@ -715,8 +715,13 @@ so2_status gemm_v(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store 
 
 // The fused gate + inverse rotation + reduction epilogue needs whole 32-wide
 // channel chunks inside one edge-frame row.
+// Whether the reduction onto nodes runs in the product's epilogue.  The
+// epilogue costs the same per tile on both paths, but the bf16 product's main
+// loop is three times shorter, so there the epilogue would set the pace:
+// bf16 products store their rows and k_reduce_nodes reduces them
+// (measured 2-4 % faster per step); the split f32 path keeps the fusion.
 #ifndef SO2_FUSE_BF16
-#define SO2_FUSE_BF16 1
+#define SO2_FUSE_BF16 0
 #endif
 bool fusable(int C, bool split) { return C % 32 == 0 && (split || SO2_FUSE_BF16); }
 
