@@ -607,9 +607,13 @@ __global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes(Layout y, int
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
   float *dsm = dbuf[threadIdx.x >> 5];
   const int n_first = rec[0].key, n_last = rec[M - 1].key;
-  const int items = (n_last - n_first + 1) * (y.L + 1);
+  const int nn = n_last - n_first + 1;
+  const int items = nn * (y.L + 1);
+  // degree-major item order, highest degree first: warps that run at the
+  // same time mostly run the same degree's code (instruction cache), and the
+  // heaviest items start first
   for (int it = blockIdx.x * wpb + (threadIdx.x >> 5); it < items; it += gridDim.x * wpb) {
-    const int n = n_first + it / (y.L + 1), l = it % (y.L + 1);
+    const int n = n_first + it % nn, l = y.L - it / nn;
     int b = offsets[n] - static_cast<int>(e0), e = offsets[n + 1] - static_cast<int>(e0);
     b = b < 0 ? 0 : b;
     e = e > M ? M : e;

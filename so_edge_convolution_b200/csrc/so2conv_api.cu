@@ -723,7 +723,12 @@ so2_status gemm_v(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store 
 #ifndef SO2_FUSE_BF16
 #define SO2_FUSE_BF16 0
 #endif
-bool fusable(int C, bool split) { return C % 32 == 0 && (split || SO2_FUSE_BF16); }
+#ifndef SO2_FUSE_F32
+#define SO2_FUSE_F32 1
+#endif
+bool fusable(int C, bool split) {
+  return C % 32 == 0 && (split ? SO2_FUSE_F32 : SO2_FUSE_BF16);
+}
 
 GemmScatter make_scatter(Ctx &c, const float *gate, float *out, int C) {
   GemmScatter sc;
