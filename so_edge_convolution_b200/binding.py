@@ -170,9 +170,28 @@ def forward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, out=None, ws=None):
     return out
 
 
+def _outputs(names, need, shapes, out, f32):
+    """The output tensors: caller-given ones (checked) or new ones."""
+    res = {}
+    for n in names:
+        if n not in need:
+            res[n] = None
+        elif out is not None and out.get(n) is not None:
+            t = out[n]
+            if (tuple(t.shape) != tuple(shapes[n]) or t.dtype != torch.float32
+                    or t.device != f32["device"] or not t.is_contiguous()):
+                raise ValueError(f"out[{n!r}] must be a contiguous float32 tensor of shape "
+                                 f"{tuple(shapes[n])} on {f32['device']}")
+            res[n] = t
+        else:
+            res[n] = torch.empty(shapes[n], **f32)
+    return res
+
+
 def backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, need=None,
-             ws=None):
-    """Returns a dict of gradients; `need` limits which ones are computed."""
+             ws=None, out=None):
+    """Returns a dict of gradients; `need` limits which ones are computed and
+    `out` (a dict) may give preallocated tensors for some of them."""
     lib = load()
     x, edge_index, edge_vec, w, w_rad, b_rad, grad_out = map(
         _c, (x, edge_index, edge_vec, w, w_rad, b_rad, grad_out))
@@ -185,7 +204,7 @@ def backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, need=None
     shapes = {"grad_x": (N, S, desc.c_in), "grad_w": (num_weights(desc),),
               "grad_w_rad": (desc.n_rbf, desc.c_out), "grad_b_rad": (desc.c_out,),
               "grad_edge_vec": (E, 3)}
-    outs = {n: (torch.empty(shapes[n], **f32) if n in need else None) for n in names}
+    outs = _outputs(names, need, shapes, out, f32)
     p, nb = _wsarg(desc, N, E, WS_BACKWARD, dev, ws)
     code = lib.so2conv_backward(ctypes.byref(desc), N, E, _ptr(x), _ptr(edge_index),
                                 _ptr(edge_vec), Params(w.data_ptr(), w_rad.data_ptr(),
@@ -197,7 +216,7 @@ def backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, need=None
 
 
 def double_backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg_x=None,
-                    gg_edge_vec=None, need=None, ws=None):
+                    gg_edge_vec=None, need=None, ws=None, out=None):
     lib = load()
     x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg_x, gg_edge_vec = map(
         _c, (x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg_x, gg_edge_vec))
@@ -210,7 +229,7 @@ def double_backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg
     shapes = {"d_x": (N, S, desc.c_in), "d_w": (num_weights(desc),),
               "d_w_rad": (desc.n_rbf, desc.c_out), "d_b_rad": (desc.c_out,),
               "d_grad_out": (N, S, desc.c_out)}
-    outs = {n: (torch.empty(shapes[n], **f32) if n in need else None) for n in names}
+    outs = _outputs(names, need, shapes, out, f32)
     p, nb = _wsarg(desc, N, E, WS_DOUBLE_BACKWARD, dev, ws)
     code = lib.so2conv_double_backward(
         ctypes.byref(desc), N, E, _ptr(x), _ptr(edge_index), _ptr(edge_vec),

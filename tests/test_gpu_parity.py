@@ -311,3 +311,21 @@ def test_chunk_size_does_not_change_results():
     assert rel_err(out2, out1) < 5e-5
     for k in g1:
         assert rel_err(g2[k], g1[k]) < 5e-5, k
+
+
+def test_preallocated_outputs():
+    # results written into caller-given tensors equal freshly allocated ones
+    p = _small(L=3, M=2, C=32, n=80, nb=12, seed=33)
+    d = _dev(p)
+    desc = _desc(p)
+    ref = B.backward(desc, d["x"], d["edge_index"], d["edge_vec"], d["w"], d["w_rad"],
+                     d["b_rad"], d["grad_out"])
+    given = {k: torch.full_like(v, float("nan")) for k, v in ref.items()}
+    got = B.backward(desc, d["x"], d["edge_index"], d["edge_vec"], d["w"], d["w_rad"],
+                     d["b_rad"], d["grad_out"], out=given)
+    for k in ref:
+        assert got[k].data_ptr() == given[k].data_ptr()
+        assert rel_err(got[k], ref[k]) < 1e-6, k
+    with pytest.raises(ValueError):
+        B.backward(desc, d["x"], d["edge_index"], d["edge_vec"], d["w"], d["w_rad"],
+                   d["b_rad"], d["grad_out"], out={"grad_x": torch.empty(3, device=DEV)})
