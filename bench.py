@@ -40,6 +40,8 @@ CONFIGS = {
              "forward+backward", 4),
     "force": ("force", "force-training step on the eSEN-like graph: forward, backward to the "
               "edge vectors, force assembly and loss, double backward to the weights, f32", 7),
+    "md": ("force", "molecular-dynamics step on the eSEN-like graph: forward, backward to the "
+           "edge vectors only and force assembly (no weight gradients), f32", 3),
     "uma": ("uma", "UMA-like: N=5000 atoms, 30 nearest within 6 A (E=150000), lmax=6, mmax=2, "
             "C=128, bf16 features and weights, f32 accumulation, forward+backward", 4),
     "large": ("large", "Large periodic: N=20000 atoms, 50 nearest within 6 A (E=1000000), "
@@ -291,7 +293,21 @@ def run_ours(args, world, rank, local):
                               out=o["g"] if o else None)
         return out, g
 
-    step = step_force if args.config == "force" else step_fwd_bwd
+    def step_md(t, o=None):
+        # energy and forces: the forward, the edge-vector gradient of the
+        # energy (cotangent grad_out) and F_i = sum of the edge gradients
+        out = B.forward(desc, t["x"], t["edge_index"], t["edge_vec"], t["w"], t["w_rad"],
+                        t["b_rad"], ws=ws, out=o["out"] if o else None)
+        g = B.backward(desc, t["x"], t["edge_index"], t["edge_vec"], t["w"], t["w_rad"],
+                       t["b_rad"], t["grad_out"], need=["grad_edge_vec"], ws=ws,
+                       out=o["g"] if o else None)
+        gr = g["grad_edge_vec"]
+        src, dst = t["edge_index"][0], t["edge_index"][1]
+        F = o["g"]["forces"].zero_() if o else torch.zeros_like(t["f_ref"])
+        F.index_add_(0, src, -gr).index_add_(0, dst, gr)
+        return out, {"grad_edge_vec": gr, "forces": F}
+
+    step = {"force": step_force, "md": step_md}.get(args.config, step_fwd_bwd)
 
     for _ in range(max(args.warmup, 3)):
         step(d)

@@ -48,6 +48,10 @@
  *
  * Supported: 0 <= mmax <= lmax <= 6, c_in and c_out multiples of 16 in
  * [16, 512], 2 <= n_rbf <= 64.  Anything else is SO2_ERR_UNSUPPORTED.
+ *
+ * Alignment: the node feature arrays read with vector loads (x, grad_out,
+ * gg_x) must be 16-byte aligned, as cudaMalloc and PyTorch allocations are;
+ * otherwise SO2_ERR_INVALID_ARG.  Other arrays need their element alignment.
  */
 #ifndef SO2CONV_H
 #define SO2CONV_H

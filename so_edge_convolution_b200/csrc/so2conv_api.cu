@@ -469,6 +469,8 @@ struct Ctx {
   CUtensorMap m_amn_hi, m_amn_lo, m_vmn_hi, m_vmn_lo;  // the same planes, MN-major boxes
 };
 
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 so2_status common_checks(const so2conv_desc *d, int64_t N, int64_t E, const void *x,
                          const int64_t *ei, const float *ev, so2conv_params prm, void *ws,
                          size_t ws_bytes, int which, Plan &P) {
@@ -477,6 +479,7 @@ so2_status common_checks(const so2conv_desc *d, int64_t N, int64_t E, const void
   if (N == 0 && E > 0) return SO2_ERR_INVALID_ARG;
   if ((N > 0 && !x) || (E > 0 && (!ei || !ev)) || !prm.w || !prm.w_rad || !prm.b_rad)
     return SO2_ERR_INVALID_ARG;
+  if (!aligned16(x)) return SO2_ERR_INVALID_ARG;  // read with 16-byte vector loads
   if (!ws) return SO2_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) & 255) return SO2_ERR_WORKSPACE;
   P = make_plan(d, N, E, which);
@@ -921,7 +924,7 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
   so2_status r = common_checks(desc, N, E, x, edge_index, edge_vec, prm, ws, ws_bytes,
                                SO2_WS_BACKWARD, P);
   if (r != SO2_OK) return r;
-  if (N > 0 && !grad_out) return SO2_ERR_INVALID_ARG;
+  if ((N > 0 && !grad_out) || !aligned16(grad_out)) return SO2_ERR_INVALID_ARG;
   Ctx c;
   c.d = desc;
   c.P = P;
@@ -1019,7 +1022,7 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
   so2_status r = common_checks(desc, N, E, x, edge_index, edge_vec, prm, ws, ws_bytes,
                                SO2_WS_DOUBLE_BACKWARD, P);
   if (r != SO2_OK) return r;
-  if (N > 0 && !grad_out) return SO2_ERR_INVALID_ARG;
+  if ((N > 0 && !grad_out) || !aligned16(grad_out)) return SO2_ERR_INVALID_ARG;
   Ctx c;
   c.d = desc;
   c.P = P;
@@ -1034,6 +1037,7 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
   if (d_w) CK(cudaMemsetAsync(d_w, 0, sizeof(float) * nw, c.s));
   if (d_w_rad) CK(cudaMemsetAsync(d_w_rad, 0, sizeof(float) * y.nr * y.co, c.s));
   if (d_b_rad) CK(cudaMemsetAsync(d_b_rad, 0, sizeof(float) * y.co, c.s));
+  if (!aligned16(gg_x)) return SO2_ERR_INVALID_ARG;
   const bool has_r = gg_edge_vec != nullptr, has_x = gg_x != nullptr;
   if (E == 0 || (!has_r && !has_x)) return SO2_OK;
   if ((r = build_maps(c, true)) != SO2_OK) return r;

@@ -70,7 +70,8 @@ def test_chunk_size_knob(lib):
 
 
 def _fwd(lib, desc, N=4, E=3, x=1, ei=1, ev=1, w=1, ws=1, nbytes=None):
-    P = lambda f: ctypes.c_void_p(0x1000 if f else 0)  # noqa: E731 (never dereferenced)
+    # (never dereferenced) f = 2: a pointer that is not 16-byte aligned
+    P = lambda f: ctypes.c_void_p({0: 0, 1: 0x1000, 2: 0x1008}[f])  # noqa: E731
     prm = B.Params(0x1000 if w else 0, 0x1000, 0x1000)
     nb = nbytes if nbytes is not None else (1 << 40)
     return lib.so2conv_forward(ctypes.byref(desc), N, E, P(x), P(ei), P(ev), prm,
@@ -85,6 +86,7 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert _fwd(lib, B.make_desc(2, 2, 24, 16, 8, 5.0)) == 2       # c_in % 16
     assert _fwd(lib, B.make_desc(2, 2, 16, 16, 1, 5.0)) == 2       # n_rbf < 2
     assert _fwd(lib, good, x=0) == 1
+    assert _fwd(lib, good, x=2) == 1                                 # x not 16-byte aligned
     assert _fwd(lib, good, ei=0) == 1
     assert _fwd(lib, good, w=0) == 1
     assert _fwd(lib, good, ws=0) == 3
