@@ -181,6 +181,16 @@ so2_status so2conv_forward_noalloc(const so2conv_desc *desc, int64_t n_nodes,
                                    const float *edge_vec, so2conv_params params,
                                    float *out, so2_stream_t stream);
 
+/* Self-test of failure detection without a fault: enqueues one kernel whose
+ * thread waits, with the bounded wait every tensor-core kernel uses, on an
+ * mbarrier phase that nothing completes.  The wait gives up after limit_us
+ * microseconds (1 .. 10^7) and records SO2_ERR_TIMEOUT in the status word at
+ * the head of ws (>= 256-byte aligned device memory of at least 8 bytes), so
+ * so2conv_check(ws, stream) then returns SO2_ERR_TIMEOUT and the context stays
+ * usable. */
+so2_status so2conv_wait_selftest(void *ws, size_t ws_bytes, int64_t limit_us,
+                                 so2_stream_t stream);
+
 /* Number of kernels this library has launched in this process (all entry
  * points, all devices).  A plain counter, not thread safe. */
 long long so2conv_launch_count(void);

@@ -75,6 +75,9 @@ def load():
     lib.so2conv_forward_noalloc.restype = ctypes.c_int
     lib.so2conv_launch_count.argtypes = []
     lib.so2conv_launch_count.restype = ctypes.c_longlong
+    lib.so2conv_wait_selftest.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64,
+                                          ctypes.c_void_p]
+    lib.so2conv_wait_selftest.restype = ctypes.c_int
     lib.so2conv_set_max_chunk_edges.argtypes = [ctypes.c_int64]
     lib.so2conv_set_max_chunk_edges.restype = ctypes.c_int
     lib.so2conv_max_chunk_edges.argtypes = []
@@ -261,6 +264,17 @@ def edge_frames(lmax, edge_vec):
                                       _stream(edge_vec.device))
     _check_call(code, "so2conv_edge_frames")
     return R.view(E, 3, 3), D
+
+
+def wait_selftest(device, limit_us=1000):
+    """so2conv_wait_selftest, then so2conv_check: returns the recorded status
+    (SO2_ERR_TIMEOUT = 6 when the bounded wait gave up as it should)."""
+    lib = load()
+    w = workspace(device)
+    p, nb = w.get(256)
+    _check_call(lib.so2conv_wait_selftest(p, nb, int(limit_us), _stream(device)),
+                "so2conv_wait_selftest")
+    return int(lib.so2conv_check(p, _stream(device)))
 
 
 def set_max_chunk_edges(n):

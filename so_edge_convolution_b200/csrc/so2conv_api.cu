@@ -851,6 +851,18 @@ so2_status edge_terms(Ctx &c, int M, int part, const void *x, const float *grad_
   return SO2_OK;
 }
 
+// One thread waits, with the library's bounded wait, on an mbarrier phase
+// that nothing completes; the wait gives up after limit_ns and records
+// SO2_ERR_TIMEOUT (the path every tensor-core wait takes when a partner
+// never arrives).
+__global__ void k_wait_selftest(DevStatus *st, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait(&bar, 0, st, nullptr, limit_ns);
+}
+
 // Library-owned scratch for so2conv_forward_noalloc (see its declaration).
 static __device__ __align__(256) unsigned char g_noalloc_ws[SO2_NOALLOC_WORKSPACE_BYTES];
 constexpr int NOALLOC_MAX_DEVICES = 64;
@@ -1190,6 +1202,19 @@ so2_status so2conv_check(void *ws, so2_stream_t stream) {
 }
 
 long long so2conv_launch_count(void) { return g_launches; }
+
+so2_status so2conv_wait_selftest(void *ws, size_t ws_bytes, int64_t limit_us,
+                                 so2_stream_t stream) {
+  if (!ws || ws_bytes < sizeof(DevStatus) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return SO2_ERR_WORKSPACE;
+  if (limit_us < 1 || limit_us > 10000000) return SO2_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(DevStatus), s) != cudaSuccess) return SO2_ERR_CUDA;
+  k_wait_selftest<<<1, 32, 0, s>>>(static_cast<DevStatus *>(ws),
+                                    static_cast<uint64_t>(limit_us) * 1000ull);
+  ++g_launches;
+  return cudaPeekAtLastError() == cudaSuccess ? SO2_OK : SO2_ERR_CUDA;
+}
 
 so2_status so2conv_set_max_chunk_edges(int64_t n) {
   if (n < 0 || n > (1 << 22)) return SO2_ERR_INVALID_ARG;

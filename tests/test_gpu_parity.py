@@ -329,3 +329,11 @@ def test_preallocated_outputs():
     with pytest.raises(ValueError):
         B.backward(desc, d["x"], d["edge_index"], d["edge_vec"], d["w"], d["w_rad"],
                    d["b_rad"], d["grad_out"], out={"grad_x": torch.empty(3, device=DEV)})
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    # a wait that nothing completes gives up and reports SO2_ERR_TIMEOUT
+    assert B.wait_selftest(DEV, limit_us=2000) == 6
+    # the context is still usable: a small forward afterwards is correct
+    p = synth.make_problem("tiny")
+    assert rel_err(_gpu_forward(p), oracle_forward(p)) < 1e-4
