@@ -70,8 +70,8 @@ struct GemmParams {
   DevStatus *status;
 };
 
-constexpr int EPI_WARPS = SO2_EPI_WARPS;  // 4, 8 or 12: one to three per TMEM lane quadrant
-static_assert(EPI_WARPS % 4 == 0 && EPI_WARPS <= 12, "epilogue warps per TMEM quadrant");
+constexpr int EPI_WARPS = SO2_EPI_WARPS;  // 4 to 16: one to four per TMEM lane quadrant
+static_assert(EPI_WARPS % 4 == 0 && EPI_WARPS <= 16, "epilogue warps per TMEM quadrant");
 constexpr int EPI_SMEM_PER_WARP = (32 * 33 + 32 * 16 + 32) * 4;  // multiple of 16 B
 constexpr int EPI_SMEM = EPI_WARPS * EPI_SMEM_PER_WARP;
 

@@ -12,6 +12,9 @@
 
 using namespace so2;
 
+#ifndef SO2_SCATTER_PAIR_STAGES  // pipeline stages of the CTA-pair product with the fused epilogue
+#define SO2_SCATTER_PAIR_STAGES 4
+#endif
 #ifndef SO2_SCATTER_STAGES
 #define SO2_SCATTER_STAGES 3
 #endif
@@ -433,8 +436,8 @@ cudaError_t launch_gemm(int kind, bool split, const CUtensorMap &a_hi, const CUt
   // a pipeline stage
   cudaError_t r;
   if (sc && pair)
-    r = split ? launch_gemm_t<32, 4, true, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
-              : launch_gemm_t<64, 4, false, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
+    r = split ? launch_gemm_t<32, SO2_SCATTER_PAIR_STAGES, true, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
+              : launch_gemm_t<64, SO2_SCATTER_PAIR_STAGES, false, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
   else if (sc)
     r = split ? launch_gemm_t<32, SO2_SCATTER_STAGES, true, true, false>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, SO2_SCATTER_STAGES, false, true, false>(a_hi, a_lo, b_hi, b_lo, p, s);
