@@ -309,7 +309,8 @@ __device__ __forceinline__ float2 coef2(const Coef &k, int64_t i, int C, int c) 
 
 // out[row (l,m)] = A * b[m] + B * (Omega b)[m],  b = D^l X[node][l, :],
 // Omega = w_x J_x + w_y J_y with (w_x, w_y) = omega[i][0..1].  With B absent
-// this is plain rotation on gather (A = 1) or gated rotation (A = g).
+// this is plain rotation on gather (A = 1) or gated rotation (A = g).  With
+// out2 the same rotation also gives out2 = A2 * b + B2 * (Omega b).
 __device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 // Read-only (non-coherent) loads, free to move across the kernel's stores.
 __device__ __forceinline__ float4 load4_ro(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
@@ -356,12 +357,13 @@ __device__ __forceinline__ void stage_d(const float *De, int dsz, float *sD) {
 
 // LC >= 0 fixes lmax at compile time (loops fully unrolled); -1 reads it
 // from the layout.
-template <typename TX, int MM, int LC = -1>
+template <typename TX, int MM, int LC = -1, bool DUAL = false>
 __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO2_ROT_MINB : SO2_GATHER_MINB)) k_rotate_gather(Layout y, int M, const EdgeRec *__restrict__ rec,
                                 const float *__restrict__ D, const TX *__restrict__ X, int side,
                                 int use_src, Coef A, Coef B, const float *__restrict__ omega,
                                 __nv_bfloat16 *__restrict__ out_hi, __nv_bfloat16 *__restrict__ out_lo,
-                                int ld) {
+                                int ld, Coef A2, Coef B2, __nv_bfloat16 *__restrict__ out2_hi,
+                                __nv_bfloat16 *__restrict__ out2_lo) {
   constexpr int W = MM + 1;
   extern __shared__ float sDall[];  // [warps][dsz]
   const int C = side ? y.co : y.ci;
@@ -369,7 +371,8 @@ __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO
   const int *col_pad = side ? y.Kout_pad : y.Kin_pad;
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
   float *sD = sDall + (threadIdx.x >> 5) * y.dsz;
-  const bool wide = B.mode != 0;
+  constexpr bool dual = DUAL;  // a second output from the same rotation
+  const bool wide = B.mode != 0 || (dual && B2.mode != 0);
   for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
     const EdgeRec r = rec[i];
     const int node = use_src ? r.src : r.dst;
@@ -378,6 +381,8 @@ __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO
     const TX *Xn = X + (int64_t)node * y.S * C;
     __nv_bfloat16 *oh = out_hi + (int64_t)i * ld;
     __nv_bfloat16 *ol = out_lo ? out_lo + (int64_t)i * ld : nullptr;
+    __nv_bfloat16 *o2h = dual ? out2_hi + (int64_t)i * ld : nullptr;
+    __nv_bfloat16 *o2l = dual && out2_lo ? out2_lo + (int64_t)i * ld : nullptr;
     float wx = 0.f, wy = 0.f;
     if (wide) {
       wx = omega[4 * (int64_t)i];
@@ -389,6 +394,8 @@ __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO
     if constexpr (LC == 6) {
       for (int c = 4 * lane; c < C; c += 128) {
         const float4 ca = coef4(A, i, C, c), cb = coef4(B, i, C, c);
+        const float4 ca2 = dual ? coef4(A2, i, C, c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 cb2 = dual ? coef4(B2, i, C, c) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int l = 0; l <= LC; ++l) {
           float4 a[2 * W + 1];
@@ -416,26 +423,34 @@ __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO
             int g, j;
             lm_group_row(y, l, m, g, j);
             const int col = col_off[g] + j * C + c;
-            float4 o = make_float4(ca.x * a[m + W].x, ca.y * a[m + W].y, ca.z * a[m + W].z,
-                                   ca.w * a[m + W].w);
+            float4 om = make_float4(0.f, 0.f, 0.f, 0.f);  // (Omega a)[m]
             if (wide) {
               float jx, jy;
               gen_xy(l, m, [&](int q) { return a[q + W].x; }, jx, jy);
-              o.x += cb.x * (wx * jx + wy * jy);
+              om.x = wx * jx + wy * jy;
               gen_xy(l, m, [&](int q) { return a[q + W].y; }, jx, jy);
-              o.y += cb.y * (wx * jx + wy * jy);
+              om.y = wx * jx + wy * jy;
               gen_xy(l, m, [&](int q) { return a[q + W].z; }, jx, jy);
-              o.z += cb.z * (wx * jx + wy * jy);
+              om.z = wx * jx + wy * jy;
               gen_xy(l, m, [&](int q) { return a[q + W].w; }, jx, jy);
-              o.w += cb.w * (wx * jx + wy * jy);
+              om.w = wx * jx + wy * jy;
             }
-            store_split4(oh + col, ol ? ol + col : nullptr, o);
+            const float4 av = a[m + W];
+            store_split4(oh + col, ol ? ol + col : nullptr,
+                         make_float4(ca.x * av.x + cb.x * om.x, ca.y * av.y + cb.y * om.y,
+                                     ca.z * av.z + cb.z * om.z, ca.w * av.w + cb.w * om.w));
+            if (dual)
+              store_split4(o2h + col, o2l ? o2l + col : nullptr,
+                           make_float4(ca2.x * av.x + cb2.x * om.x, ca2.y * av.y + cb2.y * om.y,
+                                       ca2.z * av.z + cb2.z * om.z, ca2.w * av.w + cb2.w * om.w));
           }
         }
       }
     } else {
       for (int c = 4 * lane; c < C; c += 128) {
         const float4 ca = coef4(A, i, C, c), cb = coef4(B, i, C, c);
+        const float4 ca2 = dual ? coef4(A2, i, C, c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 cb2 = dual ? coef4(B2, i, C, c) : make_float4(0.f, 0.f, 0.f, 0.f);
         each_level<LC>(y.L, [&](auto lv) {
           constexpr int l = decltype(lv)::value;
           constexpr int w = 2 * l + 1;
@@ -463,29 +478,39 @@ __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO
             int g, j;
             lm_group_row(y, l, m, g, j);
             const int col = col_off[g] + j * C + c;
-            float4 o = make_float4(ca.x * a[m + W].x, ca.y * a[m + W].y, ca.z * a[m + W].z,
-                                   ca.w * a[m + W].w);
+            float4 om = make_float4(0.f, 0.f, 0.f, 0.f);  // (Omega a)[m]
             if (wide) {
               float jx, jy;
               gen_xy(l, m, [&](int q) { return a[q + W].x; }, jx, jy);
-              o.x += cb.x * (wx * jx + wy * jy);
+              om.x = wx * jx + wy * jy;
               gen_xy(l, m, [&](int q) { return a[q + W].y; }, jx, jy);
-              o.y += cb.y * (wx * jx + wy * jy);
+              om.y = wx * jx + wy * jy;
               gen_xy(l, m, [&](int q) { return a[q + W].z; }, jx, jy);
-              o.z += cb.z * (wx * jx + wy * jy);
+              om.z = wx * jx + wy * jy;
               gen_xy(l, m, [&](int q) { return a[q + W].w; }, jx, jy);
-              o.w += cb.w * (wx * jx + wy * jy);
+              om.w = wx * jx + wy * jy;
             }
-            store_split4(oh + col, ol ? ol + col : nullptr, o);
+            const float4 av = a[m + W];
+            store_split4(oh + col, ol ? ol + col : nullptr,
+                         make_float4(ca.x * av.x + cb.x * om.x, ca.y * av.y + cb.y * om.y,
+                                     ca.z * av.z + cb.z * om.z, ca.w * av.w + cb.w * om.w));
+            if (dual)
+              store_split4(o2h + col, o2l ? o2l + col : nullptr,
+                           make_float4(ca2.x * av.x + cb2.x * om.x, ca2.y * av.y + cb2.y * om.y,
+                                       ca2.z * av.z + cb2.z * om.z, ca2.w * av.w + cb2.w * om.w));
           }
         });
       }
     }
     for (int g = 0; g < y.ng; ++g) {
       const int width = y.rows[g] * C;
-      for (int k = width + 4 * lane; k < col_pad[g]; k += 128)
+      for (int k = width + 4 * lane; k < col_pad[g]; k += 128) {
         store_split4(oh + col_off[g] + k, ol ? ol + col_off[g] + k : nullptr,
                      make_float4(0.f, 0.f, 0.f, 0.f));
+        if (dual)
+          store_split4(o2h + col_off[g] + k, o2l ? o2l + col_off[g] + k : nullptr,
+                       make_float4(0.f, 0.f, 0.f, 0.f));
+      }
     }
   }
 }

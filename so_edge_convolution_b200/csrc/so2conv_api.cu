@@ -588,21 +588,33 @@ so2_status chunk_prep(Ctx &c, int64_t e0, int M, const int64_t *ei, const float 
 // Rotation on gather into the grouped layout (rows of `out_*`, stride ld):
 // out = A * D X + B * Omega D X  (see k_rotate_gather).
 so2_status rotate(Ctx &c, int M, const void *X, bool xbf16, int side, int use_src, Coef A, Coef B,
-                  const float *omega, __nv_bfloat16 *hi, __nv_bfloat16 *lo, int ld) {
+                  const float *omega, __nv_bfloat16 *hi, __nv_bfloat16 *lo, int ld,
+                  Coef A2 = Coef{nullptr, 0}, Coef B2 = Coef{nullptr, 0},
+                  __nv_bfloat16 *hi2 = nullptr, __nv_bfloat16 *lo2 = nullptr) {
   const Plan &P = c.P;
   const EdgeRec *rec = at<EdgeRec>(c.ws, P.rec);
   const float *D = at<float>(c.ws, P.D);
   const int dsm = 8 * P.y.dsz * static_cast<int>(sizeof(float));  // staged D per warp
   ProfScope ps(3, c.s);
+#define SO2_ROT_LAUNCH(TX, DU)                                                                 \
+  DISPATCH_LM(P.y.L, P.y.mmax,                                                                 \
+              (k_rotate_gather<TX, MM, LC, DU><<<warp_grid(M, 8), 256, dsm, c.s>>>(             \
+                  P.y, M, rec, D, static_cast<const TX *>(X), side, use_src, A, B, omega, hi, lo, \
+                  ld, A2, B2, hi2, lo2)))
   if (xbf16) {
-    DISPATCH_LM(P.y.L, P.y.mmax, (k_rotate_gather<__nv_bfloat16, MM, LC><<<warp_grid(M, 8), 256, dsm, c.s>>>(
-                               P.y, M, rec, D, static_cast<const __nv_bfloat16 *>(X), side,
-                               use_src, A, B, omega, hi, lo, ld)));
+    if (hi2) {
+      SO2_ROT_LAUNCH(__nv_bfloat16, true);
+    } else {
+      SO2_ROT_LAUNCH(__nv_bfloat16, false);
+    }
   } else {
-    DISPATCH_LM(P.y.L, P.y.mmax, (k_rotate_gather<float, MM, LC><<<warp_grid(M, 8), 256, dsm, c.s>>>(
-                               P.y, M, rec, D, static_cast<const float *>(X), side, use_src, A,
-                               B, omega, hi, lo, ld)));
+    if (hi2) {
+      SO2_ROT_LAUNCH(float, true);
+    } else {
+      SO2_ROT_LAUNCH(float, false);
+    }
   }
+#undef SO2_ROT_LAUNCH
   CKL();
   return SO2_OK;
 }
@@ -619,6 +631,29 @@ so2_status rotate_x(Ctx &c, int M, const void *x, bool xbf16, int row0 = 0, Coef
   __nv_bfloat16 *hi = at<__nv_bfloat16>(c.ws, P.a_hi) + off;
   __nv_bfloat16 *lo = P.split ? at<__nv_bfloat16>(c.ws, P.a_lo) + off : nullptr;
   return rotate(c, M, x, xbf16, 0, 1, A, B, omega, hi, lo, P.y.KA);
+}
+
+// x[src] rotated once into two row sets of the a-operand planes:
+// rows [row0, row0 + M) get A * D x + B * Omega D x, rows [row1, ...) A2, B2.
+so2_status rotate_x2(Ctx &c, int M, const void *x, bool xbf16, int row0, Coef A, Coef B,
+                     int row1, Coef A2, Coef B2, const float *omega) {
+  const Plan &P = c.P;
+  __nv_bfloat16 *hi = at<__nv_bfloat16>(c.ws, P.a_hi);
+  __nv_bfloat16 *lo = P.split ? at<__nv_bfloat16>(c.ws, P.a_lo) : nullptr;
+  const size_t o0 = (size_t)row0 * P.y.KA, o1 = (size_t)row1 * P.y.KA;
+  return rotate(c, M, x, xbf16, 0, 1, A, B, omega, hi + o0, lo ? lo + o0 : nullptr, P.y.KA, A2,
+                B2, hi + o1, lo ? lo + o1 : nullptr);
+}
+
+// G[dst] rotated once into two row sets of the output-side operand planes.
+so2_status rotate_g2(Ctx &c, int M, const float *G, int row0, Coef A, Coef B, int row1, Coef A2,
+                     Coef B2, const float *omega) {
+  const Plan &P = c.P;
+  __nv_bfloat16 *hi = at<__nv_bfloat16>(c.ws, P.gv_hi);
+  __nv_bfloat16 *lo = P.split ? at<__nv_bfloat16>(c.ws, P.gv_lo) : nullptr;
+  const size_t o0 = (size_t)row0 * P.y.KG, o1 = (size_t)row1 * P.y.KG;
+  return rotate(c, M, G, false, 1, 0, A, B, omega, hi + o0, lo ? lo + o0 : nullptr, P.y.KG, A2,
+                B2, hi + o1, lo ? lo + o1 : nullptr);
 }
 
 // G[dst] rotated (with coefficients) into rows [row0, row0 + M) of the
@@ -1076,8 +1111,9 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
                                                      gg_edge_vec, prm.w_rad, at<float>(ws, P.omega),
                                                      at<float>(ws, P.dgate));
       CKL();
-      if ((r = rotate_g(c, M, grad_out, 0, dgate, gate, omega)) != SO2_OK) return r;  // P
-      if ((r = rotate_g(c, M, grad_out, ch, gate)) != SO2_OK) return r;              // Gv
+      // P = dg * b + g * Omega b and Gv = g * b from one rotation b = D G[dst]
+      if ((r = rotate_g2(c, M, grad_out, 0, dgate, gate, ch, gate, ZERO, omega)) != SO2_OK)
+        return r;
       if ((r = gemm_ga(c, ch + M)) != SO2_OK) return r;  // [M^T P; M^T Gv]
       ScatterTerms t{};
       t.F[0] = at<float>(ws, P.Ga);
@@ -1104,8 +1140,12 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
         CKL();
       }
       // a-operand rows: [a; da; a~]
-      if ((r = rotate_x(c, M, x, P.xbf16, 0)) != SO2_OK) return r;
-      if (has_r && (r = rotate_x(c, M, x, P.xbf16, ch, ZERO, ONE, omega)) != SO2_OK) return r;
+      if (has_r) {  // a = D x and da = Omega D x from one rotation
+        if ((r = rotate_x2(c, M, x, P.xbf16, 0, ONE, ZERO, ch, ZERO, ONE, omega)) != SO2_OK)
+          return r;
+      } else if ((r = rotate_x(c, M, x, P.xbf16, 0)) != SO2_OK) {
+        return r;
+      }
       if (has_x && (r = rotate_x(c, M, gg_x, false, 2 * ch)) != SO2_OK) return r;
       if ((r = gemm_v(c, has_x ? 2 * ch + M : (has_r ? ch + M : M))) != SO2_OK) return r;
       const float *V = at<float>(ws, P.V);
@@ -1143,8 +1183,12 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
           return r;
       }
       if (d_w) {
-        if (has_r && (r = rotate_g(c, M, grad_out, 0, dgate, gate, omega)) != SO2_OK) return r;
-        if ((r = rotate_g(c, M, grad_out, ch, gate)) != SO2_OK) return r;
+        if (has_r) {
+          if ((r = rotate_g2(c, M, grad_out, 0, dgate, gate, ch, gate, ZERO, omega)) != SO2_OK)
+            return r;
+        } else if ((r = rotate_g(c, M, grad_out, ch, gate)) != SO2_OK) {
+          return r;
+        }
         if (has_r) {
           if ((r = zero_tail(c, M, true, 0)) != SO2_OK) return r;
           if ((r = zero_tail(c, M, false, 0)) != SO2_OK) return r;
