@@ -1178,65 +1178,81 @@ __global__ void k_edge_omega(Layout y, float cutoff, int M, const EdgeRec *__res
 //   A[c'] = sum_{kept rows} (Omega Gy~)(V) + Gy~ dV + Gy~ V~    (d Q / d g)
 //   B[c'] = sum_{kept rows} Gy~ V                              (d Q / d dg)
 // with Gy~ = D G[dst] (rows up to mmax + 1 for Omega), V = M a, dV = M(Omega a),
-// V~ = M(D gg_x[src]) (optional).  One warp per edge, lanes over channels.
-template <int MM>
-__global__ void k_edge_terms2(Layout y, int M, const EdgeRec *__restrict__ rec,
-                              const float *__restrict__ D, const float *__restrict__ G,
-                              const float *__restrict__ omega, const float *__restrict__ V,
-                              const float *__restrict__ dV, const float *__restrict__ Vt,
-                              float *__restrict__ Aout, float *__restrict__ Bout) {
+// V~ = M(D gg_x[src]) (optional).  One warp per edge, four channels per lane,
+// D staged in shared memory, degrees compile-time as in k_edge_terms.
+template <int MM, int LC = -1>
+__global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MINB)
+    k_edge_terms2(Layout y, int M, const EdgeRec *__restrict__ rec, const float *__restrict__ D,
+                  const float *__restrict__ G, const float *__restrict__ omega,
+                  const float *__restrict__ V, const float *__restrict__ dV,
+                  const float *__restrict__ Vt, float *__restrict__ Aout,
+                  float *__restrict__ Bout) {
   constexpr int W = MM + 1;
+  extern __shared__ float sDall[];  // [warps][dsz]
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  float *sD = sDall + (threadIdx.x >> 5) * y.dsz;
   for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
     const EdgeRec r = rec[i];
-    const float *De = D + (int64_t)i * y.dsz;
+    __syncwarp();
+    stage_d(D + (int64_t)i * y.dsz, y.dsz, sD);
     const float *Gn = G + (int64_t)r.dst * y.S * y.co;
     const float wx = omega ? omega[4 * (int64_t)i] : 0.f;
     const float wy = omega ? omega[4 * (int64_t)i + 1] : 0.f;
     const int64_t ro = (int64_t)i * y.KG;
-    for (int c = 2 * lane; c < y.co; c += 64) {
-      float A0 = 0.f, A1 = 0.f, B0 = 0.f, B1 = 0.f;
-      for (int l = 0; l <= y.L; ++l) {
-        float b0[2 * W + 1], b1[2 * W + 1];
+    for (int c = 4 * lane; c < y.co; c += 128) {
+      float4 Aa = make_float4(0.f, 0.f, 0.f, 0.f), Bb = make_float4(0.f, 0.f, 0.f, 0.f);
+      each_level<LC>(y.L, [&](auto lv) {
+        constexpr int l = decltype(lv)::value;
+        constexpr int w = 2 * l + 1;
+        constexpr int mw = W < l ? W : l, mm = MM < l ? MM : l;
+        float4 b[2 * W + 1];
 #pragma unroll
-        for (int k = 0; k < 2 * W + 1; ++k) b0[k] = b1[k] = 0.f;
-        const float *Dl = De + dblock_off(l);
-        const int w = 2 * l + 1;
+        for (int k = 0; k < 2 * W + 1; ++k) b[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *Dl = sD + dblock_off(l);
+#pragma unroll
         for (int mp = -l; mp <= l; ++mp) {
-          const float2 gx = load2(Gn + (l * l + l + mp) * y.co + c);
+          if (et_fence<LC>(l, mp)) load_fence();
+          const float4 gx = load4(Gn + (l * l + l + mp) * y.co + c);
 #pragma unroll
-          for (int m = -W; m <= W; ++m) {
-            if (m < -l || m > l) continue;
+          for (int m = -mw; m <= mw; ++m) {
             const float dv = Dl[(m + l) * w + mp + l];
-            b0[m + W] += dv * gx.x;
-            b1[m + W] += dv * gx.y;
+            b[m + W].x += dv * gx.x;
+            b[m + W].y += dv * gx.y;
+            b[m + W].z += dv * gx.z;
+            b[m + W].w += dv * gx.w;
           }
         }
 #pragma unroll
-        for (int m = -MM; m <= MM; ++m) {
-          if (m < -l || m > l) continue;
+        for (int m = -mm; m <= mm; ++m) {
           int g, j;
           lm_group_row(y, l, m, g, j);
           const int64_t col = ro + y.kout_off[g] + j * y.co + c;
-          const float2 v = load2(V + col);
-          const float2 dv = dV ? load2(dV + col) : make_float2(0.f, 0.f);
-          float jx0, jy0, jx1, jy1;
-          gen_xy(l, m, [&](int q) { return b0[q + W]; }, jx0, jy0);
-          gen_xy(l, m, [&](int q) { return b1[q + W]; }, jx1, jy1);
-          const float og0 = wx * jx0 + wy * jy0, og1 = wx * jx1 + wy * jy1;
-          A0 += og0 * v.x + b0[m + W] * dv.x;
-          A1 += og1 * v.y + b1[m + W] * dv.y;
-          if (Vt) {
-            const float2 vt = load2(Vt + col);
-            A0 += b0[m + W] * vt.x;
-            A1 += b1[m + W] * vt.y;
-          }
-          B0 += b0[m + W] * v.x;
-          B1 += b1[m + W] * v.y;
+          const float4 v = load4(V + col);
+          const float4 dv = dV ? load4(dV + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 vt = Vt ? load4(Vt + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+          float4 og;  // (Omega Gy~)[m]
+          float jx, jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].x; }, jx, jy);
+          og.x = wx * jx + wy * jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].y; }, jx, jy);
+          og.y = wx * jx + wy * jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].z; }, jx, jy);
+          og.z = wx * jx + wy * jy;
+          gen_xy(l, m, [&](int q) { return b[q + W].w; }, jx, jy);
+          og.w = wx * jx + wy * jy;
+          const float4 bm = b[m + W];
+          Aa.x += og.x * v.x + bm.x * (dv.x + vt.x);
+          Aa.y += og.y * v.y + bm.y * (dv.y + vt.y);
+          Aa.z += og.z * v.z + bm.z * (dv.z + vt.z);
+          Aa.w += og.w * v.w + bm.w * (dv.w + vt.w);
+          Bb.x += bm.x * v.x;
+          Bb.y += bm.y * v.y;
+          Bb.z += bm.z * v.z;
+          Bb.w += bm.w * v.w;
         }
-      }
-      *reinterpret_cast<float2 *>(Aout + (int64_t)i * y.co + c) = make_float2(A0, A1);
-      *reinterpret_cast<float2 *>(Bout + (int64_t)i * y.co + c) = make_float2(B0, B1);
+      });
+      *reinterpret_cast<float4 *>(Aout + (int64_t)i * y.co + c) = Aa;
+      *reinterpret_cast<float4 *>(Bout + (int64_t)i * y.co + c) = Bb;
     }
   }
 }

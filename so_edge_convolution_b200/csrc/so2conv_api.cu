@@ -1172,7 +1172,7 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
       if (d_w_rad || d_b_rad) {
         {
           ProfScope ps(5, c.s);
-          DISPATCH_MM(y.mmax, (k_edge_terms2<MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+          DISPATCH_LM(y.L, y.mmax, (k_edge_terms2<MM, ((LC >= 0 && LC <= 4) ? LC : -1)><<<warp_grid(M, 8), 256, 8 * y.dsz * 4, c.s>>>(
                                 y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), grad_out,
                                 has_r ? omega : nullptr, V, has_r ? dV : nullptr,
                                 has_x ? Vt : nullptr, at<float>(ws, P.tA), at<float>(ws, P.tB))));
