@@ -515,6 +515,16 @@ __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO
   }
 }
 
+// Up to three per-edge row sets F_u (grouped layout, row stride ld[u]) and
+// their per-channel coefficients: the reduced rows are
+//   Z = sum_u A_u F_u - Omega (sum_{u<2} B_u F_u)      (|m| up to mmax + 1)
+struct ScatterTerms {
+  const float *F[3];
+  int ld[3];
+  Coef A[3];
+  Coef B[2];
+};
+
 // ---------------------------------------------------------------------------
 // Inverse rotation on reduction, node-centric, one term: for every node n
 // whose sorted segment meets this chunk and every degree l,
@@ -617,6 +627,164 @@ __device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int 
   }
 }
 
+// The general form of the node reduction (several product row sets and the
+// frame-turn term of the double backward, see ScatterTerms):
+//   Z = sum_u A_u F_u - Omega (sum_{u<2} B_u F_u),  rows |m| <= mmax + 1,
+//   out[n][(l, m')][c] += sum_{chunk edges i of n} sum_m D_i^l[m][m'] Z_i[(l, m)][c].
+// One warp per (node, l), four channels per lane, D rows staged per edge.
+template <int MM, int l>
+__device__ __forceinline__ void reduce_level_terms(const Layout &y, int b, int e, int C,
+                                                   const int *col_off, const float *__restrict__ D,
+                                                   const ScatterTerms &t,
+                                                   const float *__restrict__ omega, bool wide,
+                                                   float *o, int c, bool act, float *dsm) {
+  constexpr int W = MM + 1;
+  constexpr int w = 2 * l + 1;
+  constexpr int wpad = (w + 3) / 4 * 4;
+  constexpr int mm = MM < l ? MM : l;  // rows of the products
+  constexpr int mz = W < l ? W : l;    // rows of Z (the frame turn reaches one further)
+  constexpr int nz = 2 * mz + 1;
+  constexpr int nd = nz * w;
+  constexpr int nu = (nd + 31) / 32;
+  static_assert(nz * wpad <= RN_DBUF, "D staging buffer");
+  const int lane = threadIdx.x & 31;
+  float4 acc[w];
+#pragma unroll
+  for (int k = 0; k < w; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  int cols[2 * mm + 1];
+#pragma unroll
+  for (int m = -mm; m <= mm; ++m) {
+    int g, j;
+    lm_group_row(y, l, m, g, j);
+    cols[m + mm] = col_off[g] + j * C + c;
+  }
+  for (int i = b; i < e; ++i) {
+    const float *Dl = D + (int64_t)i * y.dsz + dblock_off(l) + (l - mz) * w;
+    float dreg[nu];
+#pragma unroll
+    for (int u = 0; u < nu; ++u) dreg[u] = (lane + 32 * u < nd) ? __ldg(Dl + lane + 32 * u) : 0.f;
+    float4 z[nz], q[2 * mm + 1];
+#pragma unroll
+    for (int m = 0; m < nz; ++m) z[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m = 0; m < 2 * mm + 1; ++m) q[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+      if (!t.F[u]) continue;
+      const float4 ka = act ? coef4(t.A[u], i, C, c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 kb =
+          (u < 2 && act) ? coef4(t.B[u < 2 ? u : 0], i, C, c) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int m = 0; m < 2 * mm + 1; ++m) {
+        const float4 f = act ? load4(t.F[u] + (int64_t)i * t.ld[u] + cols[m])
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        z[m - mm + mz].x += ka.x * f.x;
+        z[m - mm + mz].y += ka.y * f.y;
+        z[m - mm + mz].z += ka.z * f.z;
+        z[m - mm + mz].w += ka.w * f.w;
+        q[m].x += kb.x * f.x;
+        q[m].y += kb.y * f.y;
+        q[m].z += kb.z * f.z;
+        q[m].w += kb.w * f.w;
+      }
+    }
+    if (wide) {
+      const float wx = omega[4 * (int64_t)i], wy = omega[4 * (int64_t)i + 1];
+#pragma unroll
+      for (int m = -mz; m <= mz; ++m) {
+        auto qx = [&](int r) { return (r < -mm || r > mm) ? 0.f : q[r + mm].x; };
+        auto qy = [&](int r) { return (r < -mm || r > mm) ? 0.f : q[r + mm].y; };
+        auto qz = [&](int r) { return (r < -mm || r > mm) ? 0.f : q[r + mm].z; };
+        auto qw = [&](int r) { return (r < -mm || r > mm) ? 0.f : q[r + mm].w; };
+        float jx, jy;
+        gen_xy(l, m, qx, jx, jy);
+        z[m + mz].x -= wx * jx + wy * jy;
+        gen_xy(l, m, qy, jx, jy);
+        z[m + mz].y -= wx * jx + wy * jy;
+        gen_xy(l, m, qz, jx, jy);
+        z[m + mz].z -= wx * jx + wy * jy;
+        gen_xy(l, m, qw, jx, jy);
+        z[m + mz].w -= wx * jx + wy * jy;
+      }
+    }
+    __syncwarp();  // every lane is done reading the previous edge's D rows
+#pragma unroll
+    for (int u = 0; u < nu; ++u) {
+      const int k = lane + 32 * u;
+      if (k < nd) dsm[(k / w) * wpad + k % w] = dreg[u];
+    }
+    __syncwarp();
+#pragma unroll
+    for (int m = 0; m < nz; ++m) {
+#pragma unroll
+      for (int q4 = 0; q4 < wpad / 4; ++q4) {
+        const float4 d = *reinterpret_cast<const float4 *>(dsm + m * wpad + 4 * q4);
+        const float dv[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) {
+          const int mp = 4 * q4 + tt;
+          if (mp < w) {
+            acc[mp].x += dv[tt] * z[m].x;
+            acc[mp].y += dv[tt] * z[m].y;
+            acc[mp].z += dv[tt] * z[m].z;
+            acc[mp].w += dv[tt] * z[m].w;
+          }
+        }
+      }
+    }
+  }
+  if (!act) return;
+#pragma unroll
+  for (int mp = 0; mp < w; ++mp) {
+    float4 *dst = reinterpret_cast<float4 *>(o + (l * l + mp) * C + c);
+    float4 v = *dst;
+    v.x += acc[mp].x;
+    v.y += acc[mp].y;
+    v.z += acc[mp].z;
+    v.w += acc[mp].w;
+    *dst = v;
+  }
+}
+
+template <int MM>
+__global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes_terms(
+    Layout y, int64_t e0, int M, const EdgeRec *__restrict__ rec, const int *__restrict__ offsets,
+    const float *__restrict__ D, ScatterTerms t, int side, const float *__restrict__ omega,
+    float *__restrict__ out) {
+  __shared__ __align__(16) float dbuf[8][RN_DBUF];
+  if (M <= 0) return;
+  const int C = side ? y.co : y.ci;
+  const int *col_off = side ? y.kout_off : y.kin_off;
+  const bool wide = t.B[0].mode != 0 || t.B[1].mode != 0;
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  float *dsm = dbuf[threadIdx.x >> 5];
+  const int n_first = rec[0].key, n_last = rec[M - 1].key;
+  const int nn = n_last - n_first + 1;
+  const int items = nn * (y.L + 1);
+  // degree-major item order, highest degree first (as in k_reduce_nodes)
+  for (int it = blockIdx.x * wpb + (threadIdx.x >> 5); it < items; it += gridDim.x * wpb) {
+    const int n = n_first + it % nn, l = y.L - it / nn;
+    int b = offsets[n] - static_cast<int>(e0), e = offsets[n + 1] - static_cast<int>(e0);
+    b = b < 0 ? 0 : b;
+    e = e > M ? M : e;
+    if (b >= e) continue;
+    float *o = out + (int64_t)n * y.S * C;
+    for (int c0 = 0; c0 < C; c0 += 128) {
+      const int c = c0 + 4 * lane;
+      const bool act = c < C;
+      switch (l) {
+        case 0: reduce_level_terms<MM, 0>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 1: reduce_level_terms<MM, 1>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 2: reduce_level_terms<MM, 2>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 3: reduce_level_terms<MM, 3>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 4: reduce_level_terms<MM, 4>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 5: reduce_level_terms<MM, 5>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        default: reduce_level_terms<MM, 6>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+      }
+    }
+  }
+}
+
 template <int MM>
 __global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes(Layout y, int64_t e0, int M,
                                                       const EdgeRec *__restrict__ rec,
@@ -661,15 +829,6 @@ __global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes(Layout y, int
   }
 }
 
-// Up to three per-edge row sets F_u (grouped layout, row stride ld[u]) and
-// their per-channel coefficients: the reduced rows are
-//   Z = sum_u A_u F_u - Omega (sum_{u<2} B_u F_u)      (|m| up to mmax + 1)
-struct ScatterTerms {
-  const float *F[3];
-  int ld[3];
-  Coef A[3];
-  Coef B[2];
-};
 
 // ---------------------------------------------------------------------------
 // Inverse rotation on reduction, node-centric.  For every node whose sorted

@@ -796,8 +796,14 @@ so2_status scatter(Ctx &c, int64_t e0, int M, const ScatterTerms &t, int side,
   const EdgeRec *rec = at<EdgeRec>(c.ws, P.rec);
   const int *off = at<int>(c.ws, P.offsets);
   const float *D = at<float>(c.ws, P.D);
-  bool ok = true;
   ProfScope ps(7, c.s);
+  if (!(reinterpret_cast<uintptr_t>(out) & 15)) {  // node-centric kernel with vector RMW
+    DISPATCH_MM(y.mmax, k_reduce_nodes_terms<MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                            y, e0, M, rec, off, D, t, side, omega, out));
+    CKL();
+    return SO2_OK;
+  }
+  bool ok = true;
   DISPATCH_MM(y.mmax, ok = allow_smem(k_scatter_nodes<MM>, smem);
               if (ok) k_scatter_nodes<MM><<<grid_for(M, 1), threads, smem, c.s>>>(
                   y, e0, M, rec, off, D, t, side, omega, out));
@@ -1105,12 +1111,13 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
     for (int64_t e0 = 0; e0 < E; e0 += ch) {
       const int M = static_cast<int>((E - e0) < ch ? (E - e0) : ch);
       if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 0, prm)) != SO2_OK) return r;
-      ProfScope ps(5, c.s);
-      k_edge_omega<<<warp_grid(M, 8), 256, 0, c.s>>>(y, desc->rbf_cutoff, M,
-                                                     at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo),
-                                                     gg_edge_vec, prm.w_rad, at<float>(ws, P.omega),
-                                                     at<float>(ws, P.dgate));
-      CKL();
+      {
+        ProfScope ps(5, c.s);
+        k_edge_omega<<<warp_grid(M, 8), 256, 0, c.s>>>(
+            y, desc->rbf_cutoff, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo), gg_edge_vec,
+            prm.w_rad, at<float>(ws, P.omega), at<float>(ws, P.dgate));
+        CKL();
+      }
       // P = dg * b + g * Omega b and Gv = g * b from one rotation b = D G[dst]
       if ((r = rotate_g2(c, M, grad_out, 0, dgate, gate, ch, gate, ZERO, omega)) != SO2_OK)
         return r;
