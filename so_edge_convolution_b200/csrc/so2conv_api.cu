@@ -833,14 +833,6 @@ so2_status reduce_nodes(Ctx &c, int64_t e0, int M, const float *F, int ld, const
   return SO2_OK;
 }
 
-ScatterTerms one_term(const float *F, int ld, Coef A) {
-  ScatterTerms t{};
-  t.F[0] = F;
-  t.ld[0] = ld;
-  t.A[0] = A;
-  return t;
-}
-
 so2_status rad_grads(Ctx &c, int M, const float *Ag, const float *Bg, const float *omega,
                      float *grad_w_rad, float *grad_b) {
   const Plan &P = c.P;
