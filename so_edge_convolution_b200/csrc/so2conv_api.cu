@@ -364,8 +364,15 @@ cudaError_t launch_gemm_t(const CUtensorMap &a_hi, const CUtensorMap &a_lo, cons
                           const CUtensorMap &b_lo, const GemmParams &p, cudaStream_t s) {
   using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER, PAIR>;
   auto kernel = k_gemm_tc<BK, STAGES, SPLIT, SCATTER, MN, PAIR>;
-  static bool configured = false;
-  static int max_units = 0;  // persistent CTAs (non-pair) or clusters (pair)
+  // per device: the shared-memory attribute and the persistent grid size
+  // (CTAs, or clusters for pairs)
+  constexpr int MAX_DEV = 64;
+  static bool configured_dev[MAX_DEV] = {};
+  static int max_units_dev[MAX_DEV] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEV) return cudaErrorInvalidDevice;
+  bool &configured = configured_dev[dev];
+  int &max_units = max_units_dev[dev];
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg::SMEM);
