@@ -205,8 +205,8 @@ __device__ __forceinline__ void epi_scatter_chunk(const GemmScatter &S, int M, i
   }
 }
 
-// BK = 32 uses the 64-byte swizzle (4 stages of 48 KB with hi/lo planes),
-// BK = 64 the 128-byte swizzle.
+// BK = 32 uses the 64-byte swizzle, BK = 64 the 128-byte swizzle; a pair's
+// stage with hi/lo planes is 64 KB per CTA at BK = 64.
 // With PAIR, two CTAs (a cluster) share each 256 x 256 tile: each holds 128
 // rows of A and of the output, and half (128 rows) of B.
 template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool PAIR = false>

@@ -18,6 +18,25 @@ using namespace so2;
 #ifndef SO2_SCATTER_STAGES
 #define SO2_SCATTER_STAGES 3
 #endif
+// K block of the split (hi/lo) products: 64 (128-byte rows, 128-byte swizzle;
+// by measurement the operands arrive faster in 128-byte rows, even with half as
+// many, twice as large stages) or 32 (64-byte rows and swizzle)
+#ifndef SO2_SPLIT_BK
+#define SO2_SPLIT_BK 64
+#endif
+#if SO2_SPLIT_BK == 64
+#define SO2_SPLIT_PLAIN_PAIR_STAGES 3
+#define SO2_SPLIT_MN_PAIR_STAGES 3
+#define SO2_SPLIT_SCATTER_PAIR_STAGES 2
+#define SO2_SPLIT_SCATTER_STAGES 1
+#define SO2_SPLIT_PLAIN_STAGES 2
+#else
+#define SO2_SPLIT_PLAIN_PAIR_STAGES 6
+#define SO2_SPLIT_MN_PAIR_STAGES 6
+#define SO2_SPLIT_SCATTER_PAIR_STAGES SO2_SCATTER_PAIR_STAGES
+#define SO2_SPLIT_SCATTER_STAGES SO2_SCATTER_STAGES
+#define SO2_SPLIT_PLAIN_STAGES 4
+#endif
 
 namespace {
 
@@ -85,9 +104,9 @@ bool make_map_mn(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, i
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// K block of the product kernel: 32 (64-byte swizzle) for the split path so
-// that four stages of hi/lo planes fit in shared memory, 64 otherwise.
-inline int gemm_bk(bool split) { return split ? 32 : 64; }
+// K block of the product kernel (64 elements = 128-byte rows unless the split
+// path is built with 32).
+inline int gemm_bk(bool split) { return split ? SO2_SPLIT_BK : 64; }
 
 int num_sms() {
   int dev = 0, n = 148;
@@ -443,22 +462,22 @@ cudaError_t launch_gemm(int kind, bool split, const CUtensorMap &a_hi, const CUt
   // a pipeline stage
   cudaError_t r;
   if (sc && pair)
-    r = split ? launch_gemm_t<32, SO2_SCATTER_PAIR_STAGES, true, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
+    r = split ? launch_gemm_t<SO2_SPLIT_BK, SO2_SPLIT_SCATTER_PAIR_STAGES, true, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, SO2_SCATTER_PAIR_STAGES, false, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
   else if (sc)
-    r = split ? launch_gemm_t<32, SO2_SCATTER_STAGES, true, true, false>(a_hi, a_lo, b_hi, b_lo, p, s)
+    r = split ? launch_gemm_t<SO2_SPLIT_BK, SO2_SPLIT_SCATTER_STAGES, true, true, false>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, SO2_SCATTER_STAGES, false, true, false>(a_hi, a_lo, b_hi, b_lo, p, s);
   else if (mn && pair)
-    r = split ? launch_gemm_t<32, 6, true, false, true, true>(a_hi, a_lo, b_hi, b_lo, p, s)
+    r = split ? launch_gemm_t<SO2_SPLIT_BK, SO2_SPLIT_MN_PAIR_STAGES, true, false, true, true>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, 6, false, false, true, true>(a_hi, a_lo, b_hi, b_lo, p, s);
   else if (mn)
-    r = split ? launch_gemm_t<32, 4, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
+    r = split ? launch_gemm_t<SO2_SPLIT_BK, SO2_SPLIT_PLAIN_STAGES, true, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, 4, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
   else if (pair)
-    r = split ? launch_gemm_t<32, 6, true, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
+    r = split ? launch_gemm_t<SO2_SPLIT_BK, SO2_SPLIT_PLAIN_PAIR_STAGES, true, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, 6, false, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
   else
-    r = split ? launch_gemm_t<32, 4, true, false, false>(a_hi, a_lo, b_hi, b_lo, p, s)
+    r = split ? launch_gemm_t<SO2_SPLIT_BK, SO2_SPLIT_PLAIN_STAGES, true, false, false>(a_hi, a_lo, b_hi, b_lo, p, s)
               : launch_gemm_t<64, 4, false, false, false>(a_hi, a_lo, b_hi, b_lo, p, s);
   if (e1) cudaEventRecord(e1, s);
   return r;

@@ -1,8 +1,8 @@
-"""One graph over two ranks (gloo, CPU): the destination-partitioned path.
+"""One graph over two or three ranks (gloo, CPU): the destination-partitioned path.
 
 so_edge_convolution_b200.sharded splits the edges by destination owner,
 all-gathers node features, reduce-scatters grad_x and all-reduces the weight
-gradients.  These tests run that host logic with world size 2, with the
+gradients.  These tests run that host logic with world sizes 2 and 3, with the
 float64 oracle standing in for the per-device convolution, and check that
 the ranks' pieces put together equal the single-process result on the whole
 graph.
@@ -70,15 +70,16 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_rank_sharded_graph_matches_single_process():
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_graph_matches_single_process(world):
     from helpers import oracle_backward, oracle_forward
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for pr in procs:
         pr.start()
-    res = [q.get(timeout=300) for _ in range(2)]
+    res = [q.get(timeout=300) for _ in range(world)]
     for pr in procs:
         pr.join(timeout=120)
         assert pr.exitcode == 0
@@ -88,7 +89,9 @@ def test_two_rank_sharded_graph_matches_single_process():
     ref = {k: v.numpy() for k, v in oracle_backward(p).items()}
     out = np.concatenate([r[3] for r in res])
     gx = np.concatenate([r[4] for r in res])
-    assert [r[1] for r in res] == [0, res[0][2]] and res[1][2] == p.n_nodes
+    # contiguous node ranges covering every node once, in rank order
+    assert res[0][1] == 0 and res[-1][2] == p.n_nodes
+    assert all(res[k][2] == res[k + 1][1] for k in range(world - 1))
     np.testing.assert_allclose(out, ref_out, rtol=1e-10, atol=1e-10)
     np.testing.assert_allclose(gx, ref["grad_x"], rtol=1e-10, atol=1e-10)
     # every edge belongs to exactly one rank; its gradient lands in place
