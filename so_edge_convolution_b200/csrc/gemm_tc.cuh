@@ -74,6 +74,17 @@ constexpr int EPI_WARPS = SO2_EPI_WARPS;  // 4 to 16: one to four per TMEM lane 
 static_assert(EPI_WARPS % 4 == 0 && EPI_WARPS <= 16, "epilogue warps per TMEM quadrant");
 constexpr int EPI_SMEM_PER_WARP = (32 * 33 + 32 * 16 + 32) * 4;  // multiple of 16 B
 constexpr int EPI_SMEM = EPI_WARPS * EPI_SMEM_PER_WARP;
+// Plain bf16 products: each epilogue warp writes its 32 x 32 chunk of f32
+// results through a [32][33] shared-memory transpose so that every store
+// instruction covers one 128-byte row segment instead of 32 rows.
+#ifndef SO2_TSTORE
+#define SO2_TSTORE 1
+#endif
+constexpr int EPI_TST_BYTES = EPI_WARPS * 32 * 33 * 4;
+template <bool SPLIT, bool SCATTER, bool MN>
+constexpr bool gemm_tstore() {
+  return SO2_TSTORE && !SPLIT && !SCATTER && !MN;
+}
 
 // Row j of an m-group (|m| = g) of an lmax-L layout -> (l, m); rows of group
 // g >= 1 are (l, +g) for l = g..L then (l, -g).
@@ -209,8 +220,9 @@ __device__ __forceinline__ void epi_scatter_chunk(const GemmScatter &S, int M, i
 // stage with hi/lo planes is 64 KB per CTA at BK = 64.
 // With PAIR, two CTAs (a cluster) share each 256 x 256 tile: each holds 128
 // rows of A and of the output, and half (128 rows) of B.
-template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool PAIR = false>
+template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool PAIR = false, bool TST = false>
 struct GemmCfg {
+  static constexpr bool TSTORE = TST;
   static constexpr int NB = PAIR ? GEMM_BN / 2 : GEMM_BN;  // B rows held by this CTA
   static constexpr int TBM = PAIR ? 2 * GEMM_BM : GEMM_BM;  // output rows per tile
   static constexpr int A_BYTES = GEMM_BM * BK * 2;
@@ -218,7 +230,8 @@ struct GemmCfg {
   static constexpr int PLANES = SPLIT ? 2 : 1;
   static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES) * PLANES;
   static constexpr int SMEM =
-      STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + (SCATTER ? EPI_SMEM : 0);
+      STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
+      (SCATTER ? EPI_SMEM : (TST ? EPI_TST_BYTES : 0));
   static constexpr int TMEM_COLS = 2 * GEMM_BN;
   static_assert(SMEM <= 232448, "shared memory per CTA");
 };
@@ -251,7 +264,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
               const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
               const __grid_constant__ GemmParams p) {
-  using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER, PAIR>;
+  using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER, PAIR, gemm_tstore<SPLIT, SCATTER, MN>()>;
   constexpr int NB = Cfg::NB, TBM = Cfg::TBM;
   static_assert(!MN || BK % 16 == 0, "MN-major K block");
   extern __shared__ uint8_t smem_raw[];
@@ -445,7 +458,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint32_t r[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * GEMM_BN + cc * 32, r);
         // store first (when asked), so that r is dead before the reduction
-        if (p.store && row < G.M) {
+        if (Cfg::TSTORE && p.store) {
+          float *Tt = epi_smem + (warp - 2) * (32 * 33);
+          __syncwarp();  // the previous chunk's reads of Tt are done
+#pragma unroll
+          for (int k = 0; k < 32; ++k) Tt[lane * 33 + k] = __uint_as_float(r[k]);
+          __syncwarp();
+          const int nrow = G.M - row_base;  // rows of this chunk inside the product
+          if (col0 + lane < G.N) {
+            float *cp = Cg + static_cast<long long>(row_base) * G.ldc + col0 + lane;
+#pragma unroll 4
+            for (int e = 0; e < 32; ++e) {
+              if (e >= nrow) break;
+              float v = Tt[e * 33 + lane];
+              float *d = cp + static_cast<long long>(e) * G.ldc;
+              if (atomic_c) {
+                atomicAdd(d, v);
+              } else {
+                if (p.beta) v += *d;
+                *d = v;
+              }
+            }
+          }
+        } else if (p.store && row < G.M) {
           float *crow = Cg + static_cast<long long>(row) * G.ldc + col0;
           const bool vec = (col0 + 32 <= G.N) && ((reinterpret_cast<uintptr_t>(crow) & 15) == 0);
           if (atomic_c && vec) {

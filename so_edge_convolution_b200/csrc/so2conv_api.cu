@@ -24,6 +24,14 @@ using namespace so2;
 #ifndef SO2_SPLIT_BK
 #define SO2_SPLIT_BK 64
 #endif
+// plain bf16 products: the transposing store epilogue takes ~50 KB of shared memory
+#if SO2_TSTORE
+#define SO2_BF16_PLAIN_PAIR_STAGES 5
+#define SO2_BF16_PLAIN_STAGES 3
+#else
+#define SO2_BF16_PLAIN_PAIR_STAGES 6
+#define SO2_BF16_PLAIN_STAGES 4
+#endif
 #if SO2_SPLIT_BK == 64
 #define SO2_SPLIT_PLAIN_PAIR_STAGES 3
 #define SO2_SPLIT_MN_PAIR_STAGES 3
@@ -381,7 +389,7 @@ struct GemmLauncher {
 template <int BK, int STAGES, bool SPLIT, bool SCATTER, bool MN, bool PAIR = false>
 cudaError_t launch_gemm_t(const CUtensorMap &a_hi, const CUtensorMap &a_lo, const CUtensorMap &b_hi,
                           const CUtensorMap &b_lo, const GemmParams &p, cudaStream_t s) {
-  using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER, PAIR>;
+  using Cfg = GemmCfg<BK, STAGES, SPLIT, SCATTER, PAIR, gemm_tstore<SPLIT, SCATTER, MN>()>;
   auto kernel = k_gemm_tc<BK, STAGES, SPLIT, SCATTER, MN, PAIR>;
   // per device: the shared-memory attribute and the persistent grid size
   // (CTAs, or clusters for pairs)
@@ -475,10 +483,10 @@ cudaError_t launch_gemm(int kind, bool split, const CUtensorMap &a_hi, const CUt
               : launch_gemm_t<64, 4, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
   else if (pair)
     r = split ? launch_gemm_t<SO2_SPLIT_BK, SO2_SPLIT_PLAIN_PAIR_STAGES, true, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s)
-              : launch_gemm_t<64, 6, false, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
+              : launch_gemm_t<64, SO2_BF16_PLAIN_PAIR_STAGES, false, false, false, true>(a_hi, a_lo, b_hi, b_lo, p, s);
   else
     r = split ? launch_gemm_t<SO2_SPLIT_BK, SO2_SPLIT_PLAIN_STAGES, true, false, false>(a_hi, a_lo, b_hi, b_lo, p, s)
-              : launch_gemm_t<64, 4, false, false, false>(a_hi, a_lo, b_hi, b_lo, p, s);
+              : launch_gemm_t<64, SO2_BF16_PLAIN_STAGES, false, false, false>(a_hi, a_lo, b_hi, b_lo, p, s);
   if (e1) cudaEventRecord(e1, s);
   return r;
 }
