@@ -105,7 +105,8 @@ def test_hand_derived_cases(case):
     p = with_channels(base, 16)
     out = _gpu_forward(p).cpu().double()
     expect = torch.tensor(case["out"], dtype=torch.float64)
-    assert (out[..., 0] - expect).abs().max() < 1e-5
+    # f32 gate (exp) and products: ~1e-7 relative
+    assert (out[..., 0] - expect).abs().max() <= 1e-6 * max(1.0, expect.abs().max().item())
     assert out[..., 1:].abs().max() == 0
 
 

@@ -41,7 +41,10 @@ def test_hand_derived_cases(case):
     ei = I64(case["edge_index"])
     out = O.forward(x, ei[0], ei[1], T(case["edge_vec"]), T(case["w"]),
                     T(case["w_rad"]), T(case["b_rad"]), desc)
-    assert torch.allclose(out[..., 0], T(case["out"]), atol=1e-13, rtol=0)
+    expect = T(case["out"])
+    # the oracle's D comes from a least-squares fit (rounding ~1e-15 relative)
+    tol = 1e-13 * max(1.0, expect.abs().max().item())
+    assert (out[..., 0] - expect).abs().max().item() <= tol
 
 
 @pytest.mark.parametrize("L,M,ci,co", [(2, 2, 2, 3), (3, 1, 2, 2), (2, 0, 1, 2)])
@@ -195,3 +198,29 @@ def test_zero_length_edge_is_rejected():
     p.edge_vec[1] = 0.0
     with pytest.raises(ValueError):
         _run(p)
+
+
+def _wrong_width(d, desc):
+    mu = torch.linspace(0.0, desc.cutoff, desc.n_rbf, dtype=d.dtype)
+    sigma = desc.cutoff / desc.n_rbf
+    return torch.exp(-((d[:, None] - mu[None, :]) ** 2) / (2.0 * sigma * sigma))
+
+
+def _wrong_centres(d, desc):
+    sigma = desc.cutoff / (desc.n_rbf - 1)
+    mu = torch.arange(desc.n_rbf, dtype=d.dtype) * (desc.cutoff / desc.n_rbf)
+    return torch.exp(-((d[:, None] - mu[None, :]) ** 2) / (2.0 * sigma * sigma))
+
+
+@pytest.mark.parametrize("planted", [_wrong_width, _wrong_centres], ids=["width", "centres"])
+def test_radial_case_catches_a_planted_basis_mistake(planted, monkeypatch):
+    """The radial-gate hand case fails if the oracle's Gaussian basis used
+    another width or other centres (the mistake is planted in the oracle)."""
+    import oracle.so2conv as S
+    case = [c for c in _hand_cases() if c["name"] == "radial_gate_on_centres"][0]
+    monkeypatch.setattr(S, "rbf", planted)
+    desc = O.Desc(case["lmax"], case["mmax"], case["c"], case["c"], case["n_rbf"], case["cutoff"])
+    ei = I64(case["edge_index"])
+    out = O.forward(T(case["x"])[..., None], ei[0], ei[1], T(case["edge_vec"]), T(case["w"]),
+                    T(case["w_rad"]), T(case["b_rad"]), desc)
+    assert (out[..., 0] - T(case["out"])).abs().max().item() > 1e-3
