@@ -102,7 +102,14 @@ size_t so2conv_workspace_size(const so2conv_desc *desc, int64_t n_nodes,
 /* Number of packed weights (elements of w). */
 int64_t so2conv_num_weights(const so2conv_desc *desc);
 
-/* Forward: out = sum over edges of D^T (g * M_W(trunc(D x[src]))). */
+/* Forward: out = sum over edges of D^T (g * M_W(trunc(D x[src]))).
+ * Defined by "TrimSO(2): Fast and Memory-Efficient Training of Equivariant
+ * Interatomic Potentials", Abstract: rotation on gather, the dense per-m
+ * mixing, recombination and inverse rotation on reduction, in that order.
+ * Inputs as in the layout list above; `out` [N, S, c_out] f32 is
+ * overwritten (nodes without incoming edges get 0).  Returns SO2_OK or an
+ * argument / workspace status at once; device-detected problems go to
+ * so2conv_check. */
 so2_status so2conv_forward(const so2conv_desc *desc, int64_t n_nodes,
                            int64_t n_edges, const void *x,
                            const int64_t *edge_index, const float *edge_vec,
@@ -110,7 +117,13 @@ so2_status so2conv_forward(const so2conv_desc *desc, int64_t n_nodes,
                            size_t ws_bytes, so2_stream_t stream);
 
 /* Backward of <grad_out, out>: gradients w.r.t. x, w, w_rad, b_rad and the
- * edge vectors.  Any output pointer may be NULL (skipped). */
+ * edge vectors.  Any output pointer may be NULL (skipped).  Defined as the
+ * exact first derivative of the forward map ("TrimSO(2): Fast and
+ * Memory-Efficient Training of Equivariant Interatomic Potentials",
+ * Abstract: the operator supports the differentiation that training needs).
+ * grad_out [N, S, c_out] f32; grad_x [N, S, c_in], grad_w packed like w,
+ * grad_w_rad [n_rbf, c_out], grad_b_rad [c_out], grad_edge_vec [E, 3], all f32
+ * and overwritten.  Errors as for so2conv_forward. */
 so2_status so2conv_backward(const so2conv_desc *desc, int64_t n_nodes,
                             int64_t n_edges, const void *x,
                             const int64_t *edge_index, const float *edge_vec,
@@ -123,8 +136,14 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t n_nodes,
  *   Q = <gg_x, grad_x> + <gg_edge_vec, grad_edge_vec>
  * (grad_* from so2conv_backward with the same inputs) w.r.t. x, w, w_rad,
  * b_rad and grad_out.  gg_x / gg_edge_vec may be NULL (treated as zero).
+ * Defined as the exact second derivative that force training takes
+ * ("TrimSO(2): ...", Abstract: higher-order differentiation;
+ * "Breaking the Training Barrier of Billion-Parameter Universal Machine
+ * Learning Interatomic Potentials", Abstract: training needs second-order
+ * derivatives).  gg_x [N, S, c_in], gg_edge_vec [E, 3]; outputs f32 with the
+ * layouts of x, w, w_rad, b_rad, grad_out, overwritten; NULL skips one.
  * d_edge_vec (second order in the edge vectors) is not provided: it must be
- * NULL, otherwise SO2_ERR_UNSUPPORTED. */
+ * NULL, otherwise SO2_ERR_UNSUPPORTED.  Errors as for so2conv_forward. */
 so2_status so2conv_double_backward(
     const so2conv_desc *desc, int64_t n_nodes, int64_t n_edges, const void *x,
     const int64_t *edge_index, const float *edge_vec, so2conv_params params,
@@ -166,20 +185,34 @@ so2_status so2conv_edge_frames(int32_t lmax, int64_t n_edges,
  * Same arguments and results as so2conv_forward, without ws / ws_bytes.
  * Problems whose forward workspace (so2conv_workspace_size with
  * SO2_WS_FORWARD) exceeds the array are rejected with SO2_ERR_WORKSPACE
- * before anything is launched.  The first call on each device looks up the
- * array's device address with that device current; make that first call
- * before any stream capture.  All calls share the one array, which keeps the
- * last call's contents (each call re-initialises what it reads), so calls
- * that can overlap on the GPU -- different streams, or different host
- * threads -- race and must be serialised by the caller.  Device-side input
- * problems (bad index, zero-length edge) are recorded in the shared array,
- * where so2conv_check cannot see them: validate inputs first, or use
- * so2conv_forward. */
+ * before anything is launched.  The workspace grows with both sizes: about
+ * 4 E + 12 N bytes for the sort plus the per-chunk edge intermediates, so the
+ * limit is near 3,800 edges at lmax 4, C 128, f32, and even the smallest
+ * shapes stop near 20 M edges.
+ *
+ * Set-up: the array's device address belongs to the CUDA context that loaded
+ * the library's module.  The first call in each context looks it up
+ * (cudaGetSymbolAddress) and caches it under the driver's process-unique id
+ * of that context, so a context created later, for example after
+ * cudaDeviceReset, gets its own lookup.  Make that first call in each context
+ * before any stream capture.
+ *
+ * All calls in a context share the one array, which keeps the last call's
+ * contents (each call re-initialises what it reads), so calls that can
+ * overlap on the GPU -- different streams, or different host threads -- race
+ * and must be serialised by the caller.  Device-side input problems (bad
+ * index, zero-length edge) are recorded at the head of the shared array:
+ * read them with so2conv_noalloc_check. */
 so2_status so2conv_forward_noalloc(const so2conv_desc *desc, int64_t n_nodes,
                                    int64_t n_edges, const void *x,
                                    const int64_t *edge_index,
                                    const float *edge_vec, so2conv_params params,
                                    float *out, so2_stream_t stream);
+
+/* so2conv_check for the array behind so2conv_forward_noalloc in the current
+ * context: synchronises `stream`, reads and clears the device status word of
+ * the most recent no-alloc forward and returns it. */
+so2_status so2conv_noalloc_check(so2_stream_t stream);
 
 /* Self-test of failure detection without a fault: enqueues one kernel whose
  * thread waits, with the bounded wait every tensor-core kernel uses, on an

@@ -73,6 +73,8 @@ def load():
     lib.so2conv_edge_frames.restype = ctypes.c_int
     lib.so2conv_forward_noalloc.argtypes = [pd, i64, i64, vp, vp, vp, Params, vp, vp]
     lib.so2conv_forward_noalloc.restype = ctypes.c_int
+    lib.so2conv_noalloc_check.argtypes = [vp]
+    lib.so2conv_noalloc_check.restype = ctypes.c_int
     lib.so2conv_launch_count.argtypes = []
     lib.so2conv_launch_count.restype = ctypes.c_longlong
     lib.so2conv_wait_selftest.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64,
@@ -330,3 +332,9 @@ def forward_noalloc(desc, x, edge_index, edge_vec, w, w_rad, b_rad, out=None):
                                        _ptr(out), _stream(x.device))
     _check_call(code, "so2conv_forward_noalloc")
     return out
+
+
+def noalloc_check(device):
+    """Synchronise and return the device status of the last no-alloc forward
+    in the current context (0 = ok)."""
+    return int(load().so2conv_noalloc_check(_stream(device)))

@@ -14,10 +14,13 @@
 //
 // Structure: one CTA per SM loops over 128 x 256 output tiles.  Warp 0 issues
 // the TMA loads into a STAGES-deep shared-memory ring, warp 1 issues the MMAs
-// (one thread) into one of two TMEM accumulators (2 x 256 columns), warps 2..9
-// (two per TMEM lane quadrant) drain the other accumulator -- to global memory
-// and/or through the fused reduction epilogue -- so a tile's epilogue overlaps
-// the next tile's main loop.  Every wait is bounded (see mbar_wait).
+// (one thread) into one of two TMEM accumulators (2 x 256 columns), warps
+// 2..(1 + SO2_EPI_WARPS) (one to four per TMEM lane quadrant) drain the other
+// accumulator -- to global memory and/or through the fused reduction epilogue
+// -- so a tile's epilogue overlaps the next tile's main loop.  Every wait is
+// bounded (see mbar_wait); after a wait gives up, the producer and the MMA
+// thread wait (bounded) for their copies and products still in flight before
+// the CTA frees its tensor memory and exits.
 #pragma once
 
 #include "common.cuh"
@@ -274,7 +277,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t *empty = full + STAGES;
   uint64_t *tfull = empty + STAGES;  // [2]
   uint64_t *tempty = tfull + 2;      // [2]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  uint64_t *drain = tempty + 2;      // products in flight at an abort
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *epi_smem = reinterpret_cast<float *>(smem + STAGES * Cfg::STAGE_BYTES + 256);
 
@@ -297,6 +301,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], (PAIR ? 2 : 1) * EPI_WARPS);  // one arrive per epilogue warp
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -367,6 +372,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
       }
     }
+    // After an abort the MMA thread may not consume the last stages: wait
+    // (bounded) until their copies have landed before shared memory is
+    // released.  The pair's full[] barriers live in the even CTA and count
+    // both CTAs' bytes.
+    if (*abort_flag && rank == 0) {
+      for (int i = it > STAGES ? it - STAGES : 0; i < it; ++i)
+        mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.status, nullptr, 200000000ull);
+    }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ---------------- MMA issuer (the even CTA of a pair) ----------------
     constexpr uint32_t idesc = idesc_bf16_f32(TBM, GEMM_BN, MN);
@@ -428,6 +441,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         else
           umma_commit(&tfull[acc]);
       }
+    }
+    // After an abort, products already issued may still be writing tensor
+    // memory: wait (bounded) for all of them before it is freed.
+    if (*abort_flag) {
+      if (PAIR)
+        umma_commit_pair(drain);
+      else
+        umma_commit(drain);
+      mbar_wait(drain, 0, p.status, nullptr, 200000000ull);
     }
   } else if (warp >= 2) {
     // ---------------- epilogue: TMEM -> registers -> C and/or node sums ----------------

@@ -935,8 +935,65 @@ __global__ void k_wait_selftest(DevStatus *st, uint64_t limit_ns) {
 
 // Library-owned scratch for so2conv_forward_noalloc (see its declaration).
 static __device__ __align__(256) unsigned char g_noalloc_ws[SO2_NOALLOC_WORKSPACE_BYTES];
-constexpr int NOALLOC_MAX_DEVICES = 64;
-void *g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {nullptr};
+
+// The array's device address differs per CUDA context (each context loads its
+// own copy of this module), so it is cached per context, keyed by the
+// driver's process-unique context id (a context created after
+// cudaDeviceReset gets a new id, so a stale address is never reused).  The
+// driver calls go through the runtime's entry-point query, so the library
+// does not link libcuda.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+struct NoallocSlot {
+  unsigned long long ctx_id;
+  void *ptr;
+};
+constexpr int NOALLOC_MAX_CONTEXTS = 64;
+NoallocSlot g_noalloc_slots[NOALLOC_MAX_CONTEXTS];
+int g_noalloc_used = 0;
+std::mutex g_noalloc_mu;
+
+bool current_context_id(unsigned long long &id) {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_cur || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS) return false;
+  if (!ctx) {  // no context current yet: make the device's primary context current
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return false;
+    if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  }
+  return get_id(ctx, &id) == CUDA_SUCCESS;
+}
+
+// Device address of g_noalloc_ws in the current context: looked up with
+// cudaGetSymbolAddress (the host-side name of the array is not a device
+// address) the first time a context asks, then cached.
+void *noalloc_base() {
+  unsigned long long id = 0;
+  if (!current_context_id(id)) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  for (int i = 0; i < g_noalloc_used; ++i)
+    if (g_noalloc_slots[i].ctx_id == id) return g_noalloc_slots[i].ptr;
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || !p) return nullptr;
+  const int i = g_noalloc_used < NOALLOC_MAX_CONTEXTS ? g_noalloc_used++ : NOALLOC_MAX_CONTEXTS - 1;
+  g_noalloc_slots[i] = NoallocSlot{id, p};
+  return p;
+}
 
 }  // namespace
 
@@ -1253,18 +1310,16 @@ so2_status so2conv_forward_noalloc(const so2conv_desc *desc, int64_t N, int64_t 
   if (N < 0 || E < 0) return SO2_ERR_INVALID_ARG;
   const size_t need = make_plan(desc, N, E, SO2_WS_FORWARD).total;
   if (need > SO2_NOALLOC_WORKSPACE_BYTES) return SO2_ERR_WORKSPACE;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES)
-    return SO2_ERR_CUDA;
-  if (!g_noalloc_ptr[dev]) {
-    // the host-side name of the array is not a device address: ask the
-    // runtime for this device's copy (once per device, this device current)
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || !p) return SO2_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  return so2conv_forward(desc, N, E, x, edge_index, edge_vec, prm, out, g_noalloc_ptr[dev],
+  void *base = noalloc_base();
+  if (!base) return SO2_ERR_CUDA;
+  return so2conv_forward(desc, N, E, x, edge_index, edge_vec, prm, out, base,
                          SO2_NOALLOC_WORKSPACE_BYTES, stream);
+}
+
+so2_status so2conv_noalloc_check(so2_stream_t stream) {
+  void *base = noalloc_base();
+  if (!base) return SO2_ERR_CUDA;
+  return so2conv_check(base, stream);
 }
 
 so2_status so2conv_check(void *ws, so2_stream_t stream) {

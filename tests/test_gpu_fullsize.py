@@ -12,7 +12,16 @@ bench.py times.  The float64 oracle cannot run them whole, so:
   mixing weights and jointly in (W_rad, b):
       <grad_x, x> = <grad_w, w> = <grad_w_rad, W_rad> + <grad_b, b> = <grad_out, out>
   and, for the double backward with an edge-vector cotangent,
-      <d_w, w> = <gg_r, grad_edge_vec>.
+      <d_w, w> = <gg_r, grad_edge_vec>;
+* the weight gradients element by element.  They are sums over all edges, so
+  for the eSEN-like graph the oracle runs over chunks of 4,096 edges and the
+  chunks' gradients are added.  For every workload a second backward takes a
+  grad_out that is zero except on a few sampled destination nodes: the GPU
+  still runs the whole graph in the same launch configuration (chunks and
+  K-split counts depend only on the sizes), while only the sampled nodes'
+  incoming edges contribute, so the oracle on those edges gives the exact
+  gradients.  The force test does the same with an edge-vector cotangent that
+  is zero except on sampled edges.
 """
 
 import numpy as np
@@ -59,7 +68,7 @@ def _dot(a, b):
     return float((a.double() * b.double()).sum())
 
 
-def _check_workload(name, n_nodes_sample=6, n_edges_sample=64):
+def _check_workload(name, n_nodes_sample=6, n_edges_sample=64, n_wnodes=60):
     p = synth.make_problem(name, seed=0)
     d = _dev(p)
     desc = _bdesc(p)
@@ -94,19 +103,50 @@ def _check_workload(name, n_nodes_sample=6, n_edges_sample=64):
     assert abs(_dot(g["grad_w"], wr) - L) < itol * abs(L) + 1e-6
     rad = _dot(g["grad_w_rad"], d["w_rad"]) + _dot(g["grad_b_rad"], d["b_rad"])
     assert abs(rad - L) < itol * abs(L) + 1e-6
+    # weight gradients element by element: grad_out kept on sampled
+    # destinations only, so that the oracle needs only their incoming edges
+    wnodes = rng.choice(p.n_nodes, n_wnodes, replace=False)
+    Gm = np.zeros_like(p.grad_out)
+    Gm[wnodes] = p.grad_out[wnodes]
+    gm = B.backward(desc, d["x"], d["edge_index"], d["edge_vec"], d["w"], d["w_rad"],
+                    d["b_rad"], torch.from_numpy(Gm).float().to(DEV),
+                    need=["grad_w", "grad_w_rad", "grad_b_rad"])
+    torch.cuda.synchronize()
+    assert B.check(DEV) == 0
+    sel = np.nonzero(np.isin(dst, wnodes))[0]
+    wref = O.backward(*_oracle_args(p, sel), torch.from_numpy(Gm))
+    for k in ("grad_w", "grad_w_rad", "grad_b_rad"):
+        assert rel_err(gm[k].cpu(), wref[k]) < tol, k
     return p, d, desc, g
 
 
+def _oracle_weight_grads_chunked(p, chunk=4096):
+    """grad_w, grad_w_rad, grad_b_rad of the whole graph: the oracle's
+    backward over consecutive edge chunks, added up (each is a sum over
+    edges)."""
+    G = torch.from_numpy(p.grad_out)
+    acc = None
+    for e0 in range(0, p.n_edges, chunk):
+        sel = np.arange(e0, min(e0 + chunk, p.n_edges))
+        g = O.backward(*_oracle_args(p, sel), G)
+        part = {k: g[k] for k in ("grad_w", "grad_w_rad", "grad_b_rad")}
+        acc = part if acc is None else {k: acc[k] + part[k] for k in acc}
+    return acc
+
+
 def test_esen_full_size():
-    _check_workload("esen")
+    p, d, desc, g = _check_workload("esen")
+    ref = _oracle_weight_grads_chunked(p)
+    for k in ("grad_w", "grad_w_rad", "grad_b_rad"):
+        assert rel_err(g[k].cpu(), ref[k]) < 1e-4, k
 
 
 def test_uma_full_size():
-    _check_workload("uma", n_nodes_sample=3, n_edges_sample=32)
+    _check_workload("uma", n_nodes_sample=3, n_edges_sample=32, n_wnodes=20)
 
 
 def test_large_full_size():
-    _check_workload("large", n_nodes_sample=3, n_edges_sample=32)
+    _check_workload("large", n_nodes_sample=3, n_edges_sample=32, n_wnodes=40)
 
 
 def test_force_double_backward_full_size():
@@ -123,6 +163,21 @@ def test_force_double_backward_full_size():
     # <d_w, w> = <gg_r, grad_edge_vec>: both sides linear in w
     q = _dot(gg_r, g.cpu())
     assert abs(_dot(dd["d_w"], d["w"]) - q) < 1e-3 * abs(q) + 1e-6
+    # d_w, d_w_rad, d_b_rad element by element: a cotangent that is zero
+    # except on 1,024 sampled edges (Q is a sum of per-edge terms, so only
+    # those edges contribute), the GPU on the whole graph
+    es = np.sort(np.random.default_rng(9).choice(p.n_edges, 1024, replace=False))
+    ggm = torch.zeros_like(gg_r)
+    ggm[es] = gg_r[es]
+    dm = B.double_backward(desc, d["x"], d["edge_index"], d["edge_vec"], d["w"], d["w_rad"],
+                           d["b_rad"], d["grad_out"], gg_edge_vec=ggm.to(DEV),
+                           need=["d_w", "d_w_rad", "d_b_rad"])
+    torch.cuda.synchronize()
+    assert B.check(DEV) == 0
+    mref = O.double_backward(*_oracle_args(p, es), torch.from_numpy(p.grad_out),
+                             gg_edge_vec=gg_r.double()[es])
+    for k in ("d_w", "d_w_rad", "d_b_rad"):
+        assert rel_err(dm[k].cpu(), mref[k]) < 1e-4, k
     # sampled rows of d_grad_out and d_x against the oracle on the local edges
     rng = np.random.default_rng(8)
     nodes = rng.choice(p.n_nodes, 3, replace=False)

@@ -5,9 +5,10 @@ stream capture they do not own, in a plugin whose host owns all device
 memory, in a loop that must stay off the allocator).  This entry point runs
 the forward on a fixed scratch array inside the library instead of a caller
 workspace.  The test calls it through the C ABI twice in a row, on different
-inputs, and checks each result against so2conv_forward; it also checks that a
-problem too large for the array is refused before any launch.  It lives in its
-own file so that pytest collects it last.
+inputs, and checks each result against so2conv_forward and against the
+float64 oracle, with the array's own status word read after each call; it
+also checks that a problem too large for the array is refused before any
+launch.  It lives in its own file so that pytest collects it last.
 """
 
 import ctypes
@@ -18,6 +19,8 @@ import torch
 
 from so_edge_convolution_b200 import binding as B
 from so_edge_convolution_b200 import build, synth
+
+from helpers import oracle_forward, rel_err
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -38,11 +41,13 @@ def test_forward_noalloc_matches_forward_on_two_calls():
         desc = B.make_desc(p.lmax, p.mmax, p.c_in, p.c_out, p.n_rbf, p.rbf_cutoff)
         args = _tensors(p)
         ref = B.forward(desc, *args)
-        got = B.forward_noalloc(desc, *args)
         torch.cuda.synchronize()
         assert B.check(DEV) == 0
+        got = B.forward_noalloc(desc, *args)
+        assert B.noalloc_check(DEV) == 0
         err = ((got - ref).abs().max() / ref.abs().max()).item()
         assert err < 1e-4, (seed, err)
+        assert rel_err(got, oracle_forward(p)) < 1e-4, seed
 
 
 def test_forward_noalloc_refuses_a_problem_too_large():
