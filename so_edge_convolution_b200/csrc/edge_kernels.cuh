@@ -187,13 +187,20 @@ constexpr int GEO = 16;
 // blocks into this warp's shared tile sD[k][33] (entry-major, so each
 // thread's writes and the copy-out below are free of bank conflicts), then
 // copied out edge by edge with coalesced stores.  Block = one warp.
+//
+// With DT, the kept rows D^l[m][:] (|m| <= mmax) are also written row-major
+// by layout row: row t of all the chunk's edges is one contiguous run of
+// M x (2l+1) floats at DT + kept_d_prefix(t) * dt_chunk, which is the layout
+// the product's reduction epilogue stages 32 edges from with coalesced loads.
 template <int L>
 __global__ void __launch_bounds__(32) k_edge_prep(int64_t e0, int M, const int *__restrict__ perm,
                                                   const int64_t *__restrict__ ei, int64_t E,
                                                   int64_t N, int key_row,
                                                   const float *__restrict__ edge_vec,
                                                   EdgeRec *__restrict__ rec, float *__restrict__ geo,
-                                                  float *__restrict__ D, DevStatus *st) {
+                                                  float *__restrict__ D, DevStatus *st,
+                                                  int mmax = 0, float *__restrict__ DT = nullptr,
+                                                  int dt_chunk = 0) {
   constexpr int dsz = dsize(L);
   extern __shared__ float sD[];  // [dsz][33]
   const int lane = threadIdx.x;
@@ -228,6 +235,22 @@ __global__ void __launch_bounds__(32) k_edge_prep(int64_t e0, int M, const int *
   for (int j = 0; j < nj; ++j) {
     float *dst = D + (int64_t)(i0 + j) * dsz;
     for (int k = lane; k < dsz; k += 32) dst[k] = sD[k * 33 + j];
+  }
+  if (DT) {
+    for (int g = 0; g <= mmax; ++g) {
+      const int rows = g == 0 ? L + 1 : 2 * (L + 1 - g);
+      for (int j = 0; j < rows; ++j) {
+        const int l = g == 0 ? j : g + (j < L + 1 - g ? j : j - (L + 1 - g));
+        const int m = g == 0 ? 0 : (j < L + 1 - g ? g : -g);
+        const int w = 2 * l + 1;
+        const int src = dblock_off(l) + (m + l) * w;  // entry (m, 0) of block l
+        float *dst = DT + (int64_t)kept_d_prefix(L, g, j) * dt_chunk + (int64_t)i0 * w;
+        for (int idx = lane; idx < nj * w; idx += 32) {
+          const int el = idx / w, k = idx - el * w;
+          dst[idx] = sD[(src + k) * 33 + el];
+        }
+      }
+    }
   }
 }
 

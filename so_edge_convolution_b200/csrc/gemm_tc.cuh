@@ -24,6 +24,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "layout.cuh"
 
 #ifndef SO2_EPI_WARPS
 #define SO2_EPI_WARPS 12
@@ -55,9 +56,9 @@ struct GemmGroup {
 struct GemmScatter {
   const int4 *rec;     // per edge: (eid, src, dst, key)
   const float *gate;   // [rows][C] or null
-  const float *D;      // [rows][dsz] full Wigner-D blocks
+  const float *DT;     // kept D rows, row-major by layout row (see k_edge_prep)
   float *out;          // [N][S][C]
-  int C, L, dsz;
+  int C, L, dt_chunk;
 };
 
 struct GemmParams {
@@ -125,17 +126,18 @@ __device__ __forceinline__ EpiScratch epi_scratch(float *base) {
 }
 
 // Stage D^l[m][:] (W = 2l + 1 floats, row stride 16) of the warp's 32 edges
-// (rows row_base..) into Dw; zero past the end of the chunk.
+// (rows row_base..) into Dw; zero past the end of the chunk.  src is the
+// first edge's row in the kept-row copy, where the 32 edges' rows are
+// contiguous, so the loads are coalesced.
 template <int W>
-__device__ __forceinline__ void epi_stage_d(const GemmScatter &S, int M, int row_base, int doff,
+__device__ __forceinline__ void epi_stage_d(const float *__restrict__ src, int nrow,
                                             const EpiScratch &x) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int it = 0; it < W; ++it) {
     const int idx = lane + 32 * it;
     const int el = idx / W, k = idx - el * W;
-    const int ee = row_base + el;
-    x.Dw[el * 16 + k] = (ee < M) ? S.D[(int64_t)ee * S.dsz + doff + k] : 0.f;
+    x.Dw[el * 16 + k] = (el < nrow) ? __ldg(src + idx) : 0.f;
   }
 }
 
@@ -143,15 +145,16 @@ __device__ __forceinline__ void epi_stage_d(const GemmScatter &S, int M, int row
 // its 32 edges: adds sum_e D_e^l[m][m'] g_e[c] v_e[c] onto
 // out[key_e][(l, m')][c], one coalesced atomic per (node run, m', c).
 // r holds one edge's 32 values per lane (lane = edge); keys must be staged;
-// with `stage` the edges' D rows are staged into Dw first.  Each lane scales
-// its edge's values by the gate (8 vector loads of its gate row) on the way
-// into shared memory, read back with lane = channel; the warp's 32 edges split into
-// runs of equal node (a ballot finds the run starts), each summed in
-// registers and flushed with W coalesced atomics.
+// with a non-null dsrc (the first edge's kept D row) the edges' D rows are
+// staged into Dw first.  Each lane scales its edge's values by the gate (8
+// vector loads of its gate row) on the way into shared memory, read back
+// with lane = channel; the warp's 32 edges split into runs of equal node (a
+// ballot finds the run starts), each summed in registers and flushed with W
+// coalesced atomics.
 template <int W>
 __device__ __forceinline__ void epi_scatter_w(const GemmScatter &S, int M, int row_base, int l,
-                                              int m, int c0, const uint32_t (&r)[32],
-                                              bool stage, const EpiScratch &x) {
+                                              int c0, const uint32_t (&r)[32],
+                                              const float *dsrc, const EpiScratch &x) {
   const int lane = threadIdx.x & 31;
   const int my_key = x.keys[lane];
   __syncwarp();  // the previous chunk's reads of T and Dw are done
@@ -170,7 +173,7 @@ __device__ __forceinline__ void epi_scatter_w(const GemmScatter &S, int M, int r
 #pragma unroll
     for (int k = 0; k < 32; ++k) x.T[lane * 33 + k] = __uint_as_float(r[k]);
   }
-  if (stage) epi_stage_d<W>(S, M, row_base, l * (4 * l * l - 1) / 3 + (m + l) * W, x);
+  if (dsrc) epi_stage_d<W>(dsrc, M - row_base, x);
   __syncwarp();
   // lane = channel from here on
   const int c = c0 + lane;
@@ -206,16 +209,16 @@ __device__ __forceinline__ void epi_scatter_w(const GemmScatter &S, int M, int r
 }
 
 __device__ __forceinline__ void epi_scatter_chunk(const GemmScatter &S, int M, int row_base, int l,
-                                                  int m, int c0, const uint32_t (&r)[32],
-                                                  bool stage, const EpiScratch &x) {
+                                                  int c0, const uint32_t (&r)[32],
+                                                  const float *dsrc, const EpiScratch &x) {
   switch (2 * l + 1) {
-    case 1: epi_scatter_w<1>(S, M, row_base, l, m, c0, r, stage, x); break;
-    case 3: epi_scatter_w<3>(S, M, row_base, l, m, c0, r, stage, x); break;
-    case 5: epi_scatter_w<5>(S, M, row_base, l, m, c0, r, stage, x); break;
-    case 7: epi_scatter_w<7>(S, M, row_base, l, m, c0, r, stage, x); break;
-    case 9: epi_scatter_w<9>(S, M, row_base, l, m, c0, r, stage, x); break;
-    case 11: epi_scatter_w<11>(S, M, row_base, l, m, c0, r, stage, x); break;
-    default: epi_scatter_w<13>(S, M, row_base, l, m, c0, r, stage, x); break;
+    case 1: epi_scatter_w<1>(S, M, row_base, l, c0, r, dsrc, x); break;
+    case 3: epi_scatter_w<3>(S, M, row_base, l, c0, r, dsrc, x); break;
+    case 5: epi_scatter_w<5>(S, M, row_base, l, c0, r, dsrc, x); break;
+    case 7: epi_scatter_w<7>(S, M, row_base, l, c0, r, dsrc, x); break;
+    case 9: epi_scatter_w<9>(S, M, row_base, l, c0, r, dsrc, x); break;
+    case 11: epi_scatter_w<11>(S, M, row_base, l, c0, r, dsrc, x); break;
+    default: epi_scatter_w<13>(S, M, row_base, l, c0, r, dsrc, x); break;
   }
 }
 
@@ -539,7 +542,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const int j = col0 / p.sc.C, c0 = col0 % p.sc.C;
           int l, m;
           gemm_row_lm(p.sc.L, G.mgroup, j, l, m);
-          epi_scatter_chunk(p.sc, G.M, row_base, l, m, c0, r, j != staged, xs);
+          const float *dsrc =
+              j != staged ? p.sc.DT + (int64_t)kept_d_prefix(p.sc.L, G.mgroup, j) * p.sc.dt_chunk +
+                                (int64_t)row_base * (2 * l + 1)
+                          : nullptr;
+          epi_scatter_chunk(p.sc, G.M, row_base, l, c0, r, dsrc, xs);
           staged = j;
         }
       }

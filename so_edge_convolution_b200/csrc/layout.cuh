@@ -104,4 +104,30 @@ __host__ __device__ inline void lm_group_row(const Layout &y, int l, int m, int 
   j = (m > 0) ? (l - g) : (half + l - g);
 }
 
+// Kept Wigner-D rows.  Row (g, j) of the grouped edge-frame layout, i.e.
+// (l, m) with |m| <= mmax, needs the row D^l[m][:] (2l + 1 entries).  The
+// kept rows of one edge, concatenated in grouped row order, take
+// kept_d_size(L, mmax) floats; kept_d_prefix gives where row (g, j) starts.
+// Group 0 holds rows l = 0..L (sum of widths (L+1)^2), group g >= 1 rows
+// (l, +g) then (l, -g) for l = g..L (each half (L+1)^2 - g^2).
+__host__ __device__ inline int kept_d_prefix(int L, int g, int j) {
+  const int S = (L + 1) * (L + 1);
+  int base = 0;
+  for (int q = 0; q < g; ++q) base += (q == 0) ? S : 2 * (S - q * q);
+  if (g == 0) return base + j * j;
+  const int half = L + 1 - g;
+  if (j < half) {
+    const int l = g + j;
+    return base + l * l - g * g;
+  }
+  const int l = g + (j - half);
+  return base + (S - g * g) + (l * l - g * g);
+}
+__host__ __device__ inline int kept_d_size(int L, int mmax) {
+  const int S = (L + 1) * (L + 1);
+  int t = S;
+  for (int g = 1; g <= mmax; ++g) t += 2 * (S - g * g);
+  return t;
+}
+
 }  // namespace so2

@@ -46,6 +46,15 @@ using namespace so2;
 #define SO2_SPLIT_PLAIN_STAGES 4
 #endif
 
+// Whether the reduction onto nodes runs in the product's epilogue (see
+// fusable()): f32 yes, bf16 no.
+#ifndef SO2_FUSE_BF16
+#define SO2_FUSE_BF16 0
+#endif
+#ifndef SO2_FUSE_F32
+#define SO2_FUSE_F32 1
+#endif
+
 namespace {
 
 // Edges per chunk of per-edge intermediates (the workspace grows with it);
@@ -135,6 +144,7 @@ struct Plan {
   size_t total = 0;
   // byte offsets
   int na = 1, ngv = 1;  // row-stacked operand sets (double backward uses 3 and 2)
+  size_t DT = 0;  // kept D rows by layout row, for the fused reduction epilogue (f32 path)
   size_t status, counts, cursor, offsets, perm, rec, geo, D, gate, wst_hi, wst_lo, wtr_hi, wtr_lo,
       a_hi, a_lo, V, gv_hi, gv_lo, Ga, Gg, h, dws, radp, omega,
       dgate, tA, tB;
@@ -186,6 +196,7 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
   p.geo = take(c, sizeof(float) * GEO * p.chunk);
   p.D = take(c, sizeof(float) * (size_t)y.dsz * p.chunk);
   p.gate = take(c, sizeof(float) * (size_t)y.co * p.chunk);
+  if ((p.split ? SO2_FUSE_F32 : SO2_FUSE_BF16) && !dbl) p.DT = take(c, sizeof(float) * (size_t)kept_d_size(y.L, y.mmax) * p.chunk);
   p.wst_hi = take(c, 2ull * y.WR * y.WK);
   p.wst_lo = take(c, 2ull * y.WR * y.WK * lo);
   p.wtr_hi = take(c, 2ull * y.WTR * y.WTK);
@@ -609,7 +620,8 @@ so2_status chunk_prep(Ctx &c, int64_t e0, int M, const int64_t *ei, const float 
   SO2_DISPATCH_L(P.y.L, ok = allow_smem(k_edge_prep<L>, smem);
                  if (ok) k_edge_prep<L><<<(M + 31) / 32, 32, smem, c.s>>>(
                      e0, M, at<int>(c.ws, P.perm), ei, P.E, P.N, key_row, ev,
-                     at<EdgeRec>(c.ws, P.rec), at<float>(c.ws, P.geo), at<float>(c.ws, P.D), c.st));
+                     at<EdgeRec>(c.ws, P.rec), at<float>(c.ws, P.geo), at<float>(c.ws, P.D), c.st,
+                     P.y.mmax, P.DT ? at<float>(c.ws, P.DT) : nullptr, P.chunk));
   if (!ok) return SO2_ERR_CUDA;
   CKL();
   k_edge_gate<<<(M + GATE_EDGES - 1) / GATE_EDGES, 128, GATE_EDGES * P.y.nr * sizeof(float),
@@ -795,12 +807,6 @@ so2_status gemm_v(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store 
 // loop is three times shorter, so there the epilogue would set the pace:
 // bf16 products store their rows and k_reduce_nodes reduces them
 // (measured 2-4 % faster per step); the split f32 path keeps the fusion.
-#ifndef SO2_FUSE_BF16
-#define SO2_FUSE_BF16 0
-#endif
-#ifndef SO2_FUSE_F32
-#define SO2_FUSE_F32 1
-#endif
 bool fusable(int C, bool split) {
   return C % 32 == 0 && (split ? SO2_FUSE_F32 : SO2_FUSE_BF16);
 }
@@ -809,11 +815,11 @@ GemmScatter make_scatter(Ctx &c, const float *gate, float *out, int C) {
   GemmScatter sc;
   sc.rec = at<int4>(c.ws, c.P.rec);
   sc.gate = gate;
-  sc.D = at<float>(c.ws, c.P.D);
+  sc.DT = at<float>(c.ws, c.P.DT);
   sc.out = out;
   sc.C = C;
   sc.L = c.P.y.L;
-  sc.dsz = c.P.y.dsz;
+  sc.dt_chunk = c.P.chunk;
   return sc;
 }
 
@@ -1037,9 +1043,10 @@ so2_status so2conv_forward(const so2conv_desc *desc, int64_t N, int64_t E, const
   if ((r = pack_weights(c, prm.w, false)) != SO2_OK) return r;
   for (int64_t e0 = 0; e0 < E; e0 += P.chunk) {
     const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
+    const bool fuse = fusable(y.co, P.split);
     if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 1, prm)) != SO2_OK) return r;
     if ((r = rotate_x(c, M, x, P.xbf16)) != SO2_OK) return r;
-    if (fusable(y.co, P.split)) {
+    if (fuse) {
       // product, gate, inverse rotation and reduction in one kernel
       const GemmScatter sc = make_scatter(c, at<float>(ws, P.gate), out, y.co);
       if ((r = gemm_v(c, M, &sc, false)) != SO2_OK) return r;
