@@ -349,6 +349,25 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
   const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
   return make_float4(a.x, a.y, b.x, b.y);
 }
+// Four elements as loaded (raw), converted to f32 only where they are used,
+// so that a load issued ahead of its use does not wait for the data.
+template <typename T> struct Raw4;
+template <> struct Raw4<float> { float4 v; };
+template <> struct Raw4<__nv_bfloat16> { uint2 v; };
+__device__ __forceinline__ Raw4<float> ld_raw4(const float *p) {
+  return Raw4<float>{__ldg(reinterpret_cast<const float4 *>(p))};
+}
+__device__ __forceinline__ Raw4<__nv_bfloat16> ld_raw4(const __nv_bfloat16 *p) {
+  return Raw4<__nv_bfloat16>{__ldg(reinterpret_cast<const uint2 *>(p))};
+}
+__device__ __forceinline__ float4 cvt4(const Raw4<float> &r) { return r.v; }
+__device__ __forceinline__ float4 cvt4(const Raw4<__nv_bfloat16> &r) {
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.v.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.v.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+template <typename T> __device__ __forceinline__ Raw4<T> zero_raw4() { return Raw4<T>{}; }
+
 __device__ __forceinline__ void store_split4(__nv_bfloat16 *hi, __nv_bfloat16 *lo, float4 v) {
   __nv_bfloat16 h[4], l[4];
   split_bf16(v.x, h[0], l[0]);
@@ -538,8 +557,9 @@ __global__ void __launch_bounds__(256, LC == 6 ? SO2_ROT_MINB_L6 : (LC >= 0 ? SO
   }
 }
 
-// Up to three per-edge row sets F_u (grouped layout, row stride ld[u]) and
-// their per-channel coefficients: the reduced rows are
+// Up to three per-edge row sets F_u (grouped layout, row stride ld[u]; f32,
+// or bf16 where the kernel's TF says so) and their per-channel coefficients:
+// the reduced rows are
 //   Z = sum_u A_u F_u - Omega (sum_{u<2} B_u F_u)      (|m| up to mmax + 1)
 struct ScatterTerms {
   const float *F[3];
@@ -565,10 +585,10 @@ struct ScatterTerms {
 // of one edge, rows padded to a multiple of 4 floats (at most 13 x 16).
 constexpr int RN_DBUF = 13 * 16;
 
-template <int MM, int l>
+template <int MM, int l, typename TF>
 __device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int C,
                                              const int *col_off, const float *__restrict__ D,
-                                             const float *__restrict__ F, int ld,
+                                             const TF *__restrict__ F, int ld,
                                              const float *__restrict__ coef, float *o, int c,
                                              bool act, float *dsm) {
   constexpr int w = 2 * l + 1;
@@ -591,7 +611,8 @@ __device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int 
   }
   // one edge's inputs: its kept D entries (one per lane), coefficient, rows
   float dreg[nu];
-  float4 kc, fz[nm];
+  float4 kc;
+  Raw4<TF> fz[nm];
   auto load_edge = [&](int i) {
     const float *Dl = D + (int64_t)i * y.dsz + dblock_off(l) + (l - mm) * w;
 #pragma unroll
@@ -600,8 +621,7 @@ __device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int 
     if (coef && act) kc = __ldg(reinterpret_cast<const float4 *>(coef + (int64_t)i * C + c));
 #pragma unroll
     for (int m = 0; m < nm; ++m)
-      fz[m] = act ? __ldg(reinterpret_cast<const float4 *>(F + (int64_t)i * ld + cols[m]))
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      fz[m] = act ? ld_raw4(F + (int64_t)i * ld + cols[m]) : zero_raw4<TF>();
   };
   if (b < e) load_edge(b);
   for (int i = b; i < e; ++i) {
@@ -614,8 +634,10 @@ __device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int 
     }
     float4 z[nm];
 #pragma unroll
-    for (int m = 0; m < nm; ++m)
-      z[m] = make_float4(kc.x * fz[m].x, kc.y * fz[m].y, kc.z * fz[m].z, kc.w * fz[m].w);
+    for (int m = 0; m < nm; ++m) {
+      const float4 f = cvt4(fz[m]);
+      z[m] = make_float4(kc.x * f.x, kc.y * f.y, kc.z * f.z, kc.w * f.w);
+    }
     __syncwarp();
     if (i + 1 < e) load_edge(i + 1);
 #pragma unroll
@@ -655,7 +677,7 @@ __device__ __forceinline__ void reduce_level(const Layout &y, int b, int e, int 
 //   Z = sum_u A_u F_u - Omega (sum_{u<2} B_u F_u),  rows |m| <= mmax + 1,
 //   out[n][(l, m')][c] += sum_{chunk edges i of n} sum_m D_i^l[m][m'] Z_i[(l, m)][c].
 // One warp per (node, l), four channels per lane, D rows staged per edge.
-template <int MM, int l>
+template <int MM, int l, typename TF>
 __device__ __forceinline__ void reduce_level_terms(const Layout &y, int b, int e, int C,
                                                    const int *col_off, const float *__restrict__ D,
                                                    const ScatterTerms &t,
@@ -699,7 +721,8 @@ __device__ __forceinline__ void reduce_level_terms(const Layout &y, int b, int e
           (u < 2 && act) ? coef4(t.B[u < 2 ? u : 0], i, C, c) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int m = 0; m < 2 * mm + 1; ++m) {
-        const float4 f = act ? load4(t.F[u] + (int64_t)i * t.ld[u] + cols[m])
+        const float4 f = act ? load4(reinterpret_cast<const TF *>(t.F[u]) +
+                                     (int64_t)i * t.ld[u] + cols[m])
                              : make_float4(0.f, 0.f, 0.f, 0.f);
         z[m - mm + mz].x += ka.x * f.x;
         z[m - mm + mz].y += ka.y * f.y;
@@ -769,7 +792,7 @@ __device__ __forceinline__ void reduce_level_terms(const Layout &y, int b, int e
   }
 }
 
-template <int MM>
+template <int MM, typename TF = float>
 __global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes_terms(
     Layout y, int64_t e0, int M, const EdgeRec *__restrict__ rec, const int *__restrict__ offsets,
     const float *__restrict__ D, ScatterTerms t, int side, const float *__restrict__ omega,
@@ -796,24 +819,24 @@ __global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes_terms(
       const int c = c0 + 4 * lane;
       const bool act = c < C;
       switch (l) {
-        case 0: reduce_level_terms<MM, 0>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
-        case 1: reduce_level_terms<MM, 1>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
-        case 2: reduce_level_terms<MM, 2>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
-        case 3: reduce_level_terms<MM, 3>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
-        case 4: reduce_level_terms<MM, 4>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
-        case 5: reduce_level_terms<MM, 5>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
-        default: reduce_level_terms<MM, 6>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 0: reduce_level_terms<MM, 0, TF>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 1: reduce_level_terms<MM, 1, TF>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 2: reduce_level_terms<MM, 2, TF>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 3: reduce_level_terms<MM, 3, TF>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 4: reduce_level_terms<MM, 4, TF>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        case 5: reduce_level_terms<MM, 5, TF>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
+        default: reduce_level_terms<MM, 6, TF>(y, b, e, C, col_off, D, t, omega, wide, o, c, act, dsm); break;
       }
     }
   }
 }
 
-template <int MM>
+template <int MM, typename TF = float>
 __global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes(Layout y, int64_t e0, int M,
                                                       const EdgeRec *__restrict__ rec,
                                                       const int *__restrict__ offsets,
                                                       const float *__restrict__ D,
-                                                      const float *__restrict__ F, int ld,
+                                                      const TF *__restrict__ F, int ld,
                                                       const float *__restrict__ coef, int side,
                                                       float *__restrict__ out) {
   __shared__ __align__(16) float dbuf[8][2 * RN_DBUF];
@@ -840,13 +863,13 @@ __global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes(Layout y, int
       const int c = c0 + 4 * lane;
       const bool act = c < C;  // C is a multiple of 16, so c + 3 < C too
       switch (l) {
-        case 0: reduce_level<MM, 0>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
-        case 1: reduce_level<MM, 1>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
-        case 2: reduce_level<MM, 2>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
-        case 3: reduce_level<MM, 3>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
-        case 4: reduce_level<MM, 4>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
-        case 5: reduce_level<MM, 5>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
-        default: reduce_level<MM, 6>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 0: reduce_level<MM, 0, TF>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 1: reduce_level<MM, 1, TF>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 2: reduce_level<MM, 2, TF>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 3: reduce_level<MM, 3, TF>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 4: reduce_level<MM, 4, TF>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        case 5: reduce_level<MM, 5, TF>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
+        default: reduce_level<MM, 6, TF>(y, b, e, C, col_off, D, F, ld, coef, o, c, act, dsm); break;
       }
     }
   }
@@ -861,7 +884,7 @@ __global__ void __launch_bounds__(256, SO2_RN_MINB) k_reduce_nodes(Layout y, int
 // run in stream order, so every output element is updated by one thread at
 // a time and the sum order is fixed.
 // ---------------------------------------------------------------------------
-template <int MM>
+template <int MM, typename TF = float>
 __global__ void k_scatter_nodes(Layout y, int64_t e0, int M, const EdgeRec *__restrict__ rec,
                                 const int *__restrict__ offsets, const float *__restrict__ D,
                                 ScatterTerms t, int side, const float *__restrict__ omega,
@@ -904,7 +927,8 @@ __global__ void k_scatter_nodes(Layout y, int64_t e0, int M, const EdgeRec *__re
 #pragma unroll
             for (int u = 0; u < 3; ++u) {
               if (!t.F[u]) continue;
-              const float2 f = load2(t.F[u] + (int64_t)i * t.ld[u] + col_off[g] + j * C + c);
+              const float2 f = load2(reinterpret_cast<const TF *>(t.F[u]) + (int64_t)i * t.ld[u] +
+                                     col_off[g] + j * C + c);
               z0[m + W] += ka[u].x * f.x;
               z1[m + W] += ka[u].y * f.y;
               if (u < 2) {
@@ -1047,11 +1071,11 @@ __global__ void k_unstack_grad(Layout y, BlockOffsets bo, const float *__restric
 // 2 = input side only (adds its share to h).  With gv_hi, the output side
 // also writes g * (D G[dst]) on the kept rows as the transposed product's
 // operand planes (what rotation on gather of G would write).
-template <typename TX, int MM, int LC = -1, int PART = 3>
+template <typename TX, int MM, int LC = -1, int PART = 3, typename TF = float>
 __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MINB) k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
                              const float *__restrict__ D, const float *__restrict__ gate,
                              const float *__restrict__ G, const TX *__restrict__ X,
-                             const float *__restrict__ V, const float *__restrict__ Ga,
+                             const TF *__restrict__ V, const TF *__restrict__ Ga,
                              float *__restrict__ Gg, float *__restrict__ h,
                              __nv_bfloat16 *__restrict__ gv_hi, __nv_bfloat16 *__restrict__ gv_lo) {
   constexpr int W = MM + 1;  // widest |m| needed by the generators
@@ -1065,7 +1089,7 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
     float hx = 0.f, hy = 0.f;
     // output side
     const float *Gn = G + (int64_t)r.dst * y.S * y.co;
-    const float *Vi = V + (int64_t)i * y.KG;
+    const TF *Vi = V + (int64_t)i * y.KG;
     for (int c = 4 * lane; (PART & 1) && c < y.co; c += 128) {
       const float4 gv = load4(gate + (int64_t)i * y.co + c);
       float4 gg = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1131,7 +1155,7 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
     }
     // input side
     const TX *Xn = X + (int64_t)r.src * y.S * y.ci;
-    const float *Gai = Ga + (int64_t)i * y.KA;
+    const TF *Gai = Ga + (int64_t)i * y.KA;
     for (int c = 4 * lane; (PART & 2) && c < y.ci; c += 128) {
       each_level<LC>(y.L, [&](auto lv) {
         constexpr int l = decltype(lv)::value;
@@ -1362,12 +1386,12 @@ __global__ void k_edge_omega(Layout y, float cutoff, int M, const EdgeRec *__res
 // with Gy~ = D G[dst] (rows up to mmax + 1 for Omega), V = M a, dV = M(Omega a),
 // V~ = M(D gg_x[src]) (optional).  One warp per edge, four channels per lane,
 // D staged in shared memory, degrees compile-time as in k_edge_terms.
-template <int MM, int LC = -1>
+template <int MM, int LC = -1, typename TF = float>
 __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MINB)
     k_edge_terms2(Layout y, int M, const EdgeRec *__restrict__ rec, const float *__restrict__ D,
                   const float *__restrict__ G, const float *__restrict__ omega,
-                  const float *__restrict__ V, const float *__restrict__ dV,
-                  const float *__restrict__ Vt, float *__restrict__ Aout,
+                  const TF *__restrict__ V, const TF *__restrict__ dV,
+                  const TF *__restrict__ Vt, float *__restrict__ Aout,
                   float *__restrict__ Bout) {
   constexpr int W = MM + 1;
   extern __shared__ float sDall[];  // [warps][dsz]

@@ -69,6 +69,7 @@ struct GemmParams {
   int beta;   // 0: C = AB^T, 1: C += AB^T
   int split;  // 1: hi/lo planes (3 products), 0: hi only
   int store;  // write C
+  int cbf16;  // C is bf16 (plain stores only: beta 0, no K split); f32 otherwise
   int scatter;  // fused reduction epilogue (GemmScatter)
   GemmScatter sc;
   DevStatus *status;
@@ -490,7 +491,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           for (int k = 0; k < 32; ++k) Tt[lane * 33 + k] = __uint_as_float(r[k]);
           __syncwarp();
           const int nrow = G.M - row_base;  // rows of this chunk inside the product
-          if (col0 + lane < G.N) {
+          if (p.cbf16) {
+            // bf16 rows: lanes 0-15 write column pairs of row e, 16-31 of row e + 1
+            __nv_bfloat16 *cb = reinterpret_cast<__nv_bfloat16 *>(p.C) + G.c_off;
+            const int rh = lane >> 4, cp = 2 * (lane & 15);
+            if (col0 + cp < G.N) {  // N is a multiple of 16: the pair is inside
+#pragma unroll 4
+              for (int e = 0; e < 32; e += 2) {
+                const int er = e + rh;
+                if (er >= nrow) break;
+                *reinterpret_cast<__nv_bfloat162 *>(
+                    cb + static_cast<long long>(row_base + er) * G.ldc + col0 + cp) =
+                    __floats2bfloat162_rn(Tt[er * 33 + cp], Tt[er * 33 + cp + 1]);
+              }
+            }
+          } else if (col0 + lane < G.N) {
             float *cp = Cg + static_cast<long long>(row_base) * G.ldc + col0 + lane;
 #pragma unroll 4
             for (int e = 0; e < 32; ++e) {
@@ -504,6 +519,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 *d = v;
               }
             }
+          }
+        } else if (p.store && p.cbf16 && row < G.M) {
+          __nv_bfloat16 *cb = reinterpret_cast<__nv_bfloat16 *>(p.C) + G.c_off +
+                              static_cast<long long>(row) * G.ldc + col0;
+          if (col0 + 32 <= G.N) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint4 u;
+              u.x = pack_bf16x2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+              u.y = pack_bf16x2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+              u.z = pack_bf16x2(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
+              u.w = pack_bf16x2(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
+              *reinterpret_cast<uint4 *>(cb + j) = u;
+            }
+          } else {
+            for (int j = 0; j < 32 && col0 + j < G.N; ++j)
+              cb[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
           }
         } else if (p.store && row < G.M) {
           float *crow = Cg + static_cast<long long>(row) * G.ldc + col0;

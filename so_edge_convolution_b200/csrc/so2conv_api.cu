@@ -203,11 +203,12 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
   p.wtr_lo = take(c, 2ull * y.WTR * y.WTK * lo);
   p.a_hi = take(c, 2ull * na * p.chunk * y.KA);
   p.a_lo = take(c, 2ull * na * p.chunk * y.KA * lo);
-  p.V = take(c, 4ull * na * p.chunk * y.KG);
+  const size_t pe = p.split ? 4 : 2;  // bytes per product element (see prows)
+  p.V = take(c, pe * na * p.chunk * y.KG);
   if (bwd) {
     p.gv_hi = take(c, 2ull * ngv * p.chunk * y.KG);
     p.gv_lo = take(c, 2ull * ngv * p.chunk * y.KG * lo);
-    p.Ga = take(c, 4ull * ngv * p.chunk * y.KA);
+    p.Ga = take(c, pe * ngv * p.chunk * y.KA);
     p.Gg = take(c, 4ull * p.chunk * y.co);
     p.h = take(c, 8ull * p.chunk);
     p.dws = take(c, 4ull * y.WR * y.WK);
@@ -461,9 +462,10 @@ cudaError_t launch_gemm(int kind, bool split, const CUtensorMap &a_hi, const CUt
                         const CUtensorMap &b_hi, const CUtensorMap &b_lo, GemmParams p,
                         float *C, int beta, DevStatus *st, cudaStream_t s,
                         const GemmScatter *sc = nullptr, bool store = true, bool mn = false,
-                        bool pair = false) {
+                        bool pair = false, bool cbf16 = false) {
   if (p.total_tiles == 0) return cudaSuccess;
   p.C = C;
+  p.cbf16 = cbf16 ? 1 : 0;
   p.beta = beta;
   p.split = split ? 1 : 0;
   p.status = st;
@@ -518,6 +520,15 @@ struct Ctx {
 };
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Product rows (V, Ga) are f32 on the split path and bf16 on the bf16 path
+// (their rounding, 2^-9 relative, is far inside that path's tolerance, and it
+// halves the bytes every consumer reads).  Element `elems` of the rows at
+// workspace offset `off`, type-erased; kernels read it as their TF.
+inline const float *prows(const Ctx &c, size_t off, size_t elems) {
+  return reinterpret_cast<const float *>(static_cast<const char *>(c.ws) + off +
+                                         elems * (c.P.split ? 4 : 2));
+}
 
 so2_status common_checks(const so2conv_desc *d, int64_t N, int64_t E, const void *x,
                          const int64_t *ei, const float *ev, so2conv_params prm, void *ws,
@@ -780,7 +791,7 @@ so2_status gemm_ga(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store
     L.add(rows, y.Kin[g], y.Kout_pad[g], 0, y.kout_off[g], y.wt_off[g], 0, y.kin_off[g], y.KA);
   CK(launch_gemm(1, P.split, c.m_v_hi, c.m_v_lo, pair ? c.m_wtr2_hi : c.m_wtr_hi,
                  pair ? c.m_wtr2_lo : c.m_wtr_lo, L.p, at<float>(c.ws, P.Ga), 0, c.st, c.s, sc,
-                 store, false, pair));
+                 store, false, pair, !P.split));
   return SO2_OK;
 }
 
@@ -796,7 +807,7 @@ so2_status gemm_v(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store 
     L.add(rows, y.Kout[g], y.Kin_pad[g], 0, y.kin_off[g], y.wr_off[g], 0, y.kout_off[g], y.KG);
   CK(launch_gemm(0, P.split, c.m_a_hi, c.m_a_lo, pair ? c.m_wst2_hi : c.m_wst_hi,
                  pair ? c.m_wst2_lo : c.m_wst_lo, L.p, at<float>(c.ws, P.V), 0, c.st, c.s, sc,
-                 store, false, pair));
+                 store, false, pair, !P.split));
   return SO2_OK;
 }
 
@@ -838,15 +849,26 @@ so2_status scatter(Ctx &c, int64_t e0, int M, const ScatterTerms &t, int side,
   const float *D = at<float>(c.ws, P.D);
   ProfScope ps(7, c.s);
   if (!(reinterpret_cast<uintptr_t>(out) & 15)) {  // node-centric kernel with vector RMW
-    DISPATCH_MM(y.mmax, k_reduce_nodes_terms<MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
-                            y, e0, M, rec, off, D, t, side, omega, out));
+    if (P.split) {
+      DISPATCH_MM(y.mmax, k_reduce_nodes_terms<MM, float><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                              y, e0, M, rec, off, D, t, side, omega, out));
+    } else {
+      DISPATCH_MM(y.mmax, k_reduce_nodes_terms<MM, __nv_bfloat16><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                              y, e0, M, rec, off, D, t, side, omega, out));
+    }
     CKL();
     return SO2_OK;
   }
   bool ok = true;
-  DISPATCH_MM(y.mmax, ok = allow_smem(k_scatter_nodes<MM>, smem);
-              if (ok) k_scatter_nodes<MM><<<grid_for(M, 1), threads, smem, c.s>>>(
-                  y, e0, M, rec, off, D, t, side, omega, out));
+  if (P.split) {
+    DISPATCH_MM(y.mmax, ok = allow_smem(k_scatter_nodes<MM, float>, smem);
+                if (ok) k_scatter_nodes<MM, float><<<grid_for(M, 1), threads, smem, c.s>>>(
+                    y, e0, M, rec, off, D, t, side, omega, out));
+  } else {
+    DISPATCH_MM(y.mmax, ok = allow_smem(k_scatter_nodes<MM, __nv_bfloat16>, smem);
+                if (ok) k_scatter_nodes<MM, __nv_bfloat16><<<grid_for(M, 1), threads, smem, c.s>>>(
+                    y, e0, M, rec, off, D, t, side, omega, out));
+  }
   if (!ok) return SO2_ERR_CUDA;
   CKL();
   return SO2_OK;
@@ -854,6 +876,7 @@ so2_status scatter(Ctx &c, int64_t e0, int M, const ScatterTerms &t, int side,
 
 // One-term node-centric reduction (see k_reduce_nodes): out += D^T (k * F)
 // per node; falls back to the general kernel when out is not 16-byte aligned.
+// F: product rows from prows() (element type of the path).
 so2_status reduce_nodes(Ctx &c, int64_t e0, int M, const float *F, int ld, const float *coef,
                         int side, float *out) {
   const Plan &P = c.P;
@@ -866,9 +889,16 @@ so2_status reduce_nodes(Ctx &c, int64_t e0, int M, const float *F, int ld, const
     return scatter(c, e0, M, t, side, nullptr, out);
   }
   ProfScope ps(7, c.s);
-  DISPATCH_MM(y.mmax, k_reduce_nodes<MM><<<warp_grid(M, 8), 256, 0, c.s>>>(
-                          y, e0, M, at<EdgeRec>(c.ws, P.rec), at<int>(c.ws, P.offsets),
-                          at<float>(c.ws, P.D), F, ld, coef, side, out));
+  if (P.split) {
+    DISPATCH_MM(y.mmax, k_reduce_nodes<MM, float><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                            y, e0, M, at<EdgeRec>(c.ws, P.rec), at<int>(c.ws, P.offsets),
+                            at<float>(c.ws, P.D), F, ld, coef, side, out));
+  } else {
+    DISPATCH_MM(y.mmax, k_reduce_nodes<MM, __nv_bfloat16><<<warp_grid(M, 8), 256, 0, c.s>>>(
+                            y, e0, M, at<EdgeRec>(c.ws, P.rec), at<int>(c.ws, P.offsets),
+                            at<float>(c.ws, P.D), reinterpret_cast<const __nv_bfloat16 *>(F),
+                            ld, coef, side, out));
+  }
   CKL();
   return SO2_OK;
 }
@@ -903,24 +933,26 @@ so2_status edge_terms(Ctx &c, int M, int part, const void *x, const float *grad_
   const int g = warp_grid(M, 8);
   const EdgeRec *rec = at<EdgeRec>(c.ws, P.rec);
   const float *Dp = at<float>(c.ws, P.D), *gate = at<float>(c.ws, P.gate);
-  const float *Vp = at<float>(c.ws, P.V), *Gap = at<float>(c.ws, P.Ga);
+  const float *Vp = prows(c, P.V, 0), *Gap = prows(c, P.Ga, 0);
   float *Ggp = at<float>(c.ws, P.Gg), *hp = at<float>(c.ws, P.h);
   __nv_bfloat16 *gh = write_gv ? at<__nv_bfloat16>(c.ws, P.gv_hi) : nullptr;
   __nv_bfloat16 *gl = write_gv && P.split ? at<__nv_bfloat16>(c.ws, P.gv_lo) : nullptr;
-#define SO2_ET_LAUNCH(TX)                                                                    \
+#define SO2_ET_LAUNCH(TX, TF)                                                                \
   DISPATCH_LM(y.L, y.mmax,                                                                   \
               /* all levels inlined spills at lmax 6: runtime-degree kernel there */          \
               constexpr int LE = (LC >= 0 && LC <= 4) ? LC : -1;                              \
-              if (part == 1) k_edge_terms<TX, MM, LE, 1><<<g, 256, sm, c.s>>>(                 \
-                  y, M, rec, Dp, gate, grad_out, static_cast<const TX *>(x), Vp, Gap, Ggp, hp, \
-                  gh, gl);                                                                    \
-              else k_edge_terms<TX, MM, LE, 2><<<g, 256, sm, c.s>>>(                           \
-                  y, M, rec, Dp, gate, grad_out, static_cast<const TX *>(x), Vp, Gap, Ggp, hp, \
-                  nullptr, nullptr);)
+              if (part == 1) k_edge_terms<TX, MM, LE, 1, TF><<<g, 256, sm, c.s>>>(             \
+                  y, M, rec, Dp, gate, grad_out, static_cast<const TX *>(x),                  \
+                  reinterpret_cast<const TF *>(Vp), reinterpret_cast<const TF *>(Gap), Ggp,   \
+                  hp, gh, gl);                                                                \
+              else k_edge_terms<TX, MM, LE, 2, TF><<<g, 256, sm, c.s>>>(                       \
+                  y, M, rec, Dp, gate, grad_out, static_cast<const TX *>(x),                  \
+                  reinterpret_cast<const TF *>(Vp), reinterpret_cast<const TF *>(Gap), Ggp,   \
+                  hp, nullptr, nullptr);)
   if (P.xbf16) {
-    SO2_ET_LAUNCH(__nv_bfloat16)
+    SO2_ET_LAUNCH(__nv_bfloat16, __nv_bfloat16)
   } else {
-    SO2_ET_LAUNCH(float)
+    SO2_ET_LAUNCH(float, float)
   }
 #undef SO2_ET_LAUNCH
   CKL();
@@ -1052,7 +1084,7 @@ so2_status so2conv_forward(const so2conv_desc *desc, int64_t N, int64_t E, const
       if ((r = gemm_v(c, M, &sc, false)) != SO2_OK) return r;
     } else {
       if ((r = gemm_v(c, M)) != SO2_OK) return r;
-      if ((r = reduce_nodes(c, e0, M, at<float>(ws, P.V), y.KG, at<float>(ws, P.gate), 1, out)) !=
+      if ((r = reduce_nodes(c, e0, M, prows(c, P.V, 0), y.KG, at<float>(ws, P.gate), 1, out)) !=
           SO2_OK)
         return r;
     }
@@ -1117,7 +1149,7 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
       if ((r = gemm_dw(c, M, 0, 0)) != SO2_OK) return r;
     }
     if (grad_x && !fuse_gx &&
-        (r = reduce_nodes(c, e0, M, at<float>(ws, P.Ga), y.KA, nullptr, 0, grad_x)) != SO2_OK)
+        (r = reduce_nodes(c, e0, M, prows(c, P.Ga, 0), y.KA, nullptr, 0, grad_x)) != SO2_OK)
       return r;
     if (need_v) {
       if (grad_edge_vec && (r = edge_terms(c, M, 2, x, grad_out, false)) != SO2_OK) return r;
@@ -1213,10 +1245,10 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
         return r;
       if ((r = gemm_ga(c, ch + M)) != SO2_OK) return r;  // [M^T P; M^T Gv]
       ScatterTerms t{};
-      t.F[0] = at<float>(ws, P.Ga);
+      t.F[0] = prows(c, P.Ga, 0);
       t.ld[0] = y.KA;
       t.A[0] = ONE;
-      t.F[1] = at<float>(ws, P.Ga) + (size_t)ch * y.KA;
+      t.F[1] = prows(c, P.Ga, (size_t)ch * y.KA);
       t.ld[1] = y.KA;
       t.B[1] = ONE;
       if ((r = scatter(c, e0, M, t, 0, omega, d_x)) != SO2_OK) return r;
@@ -1245,9 +1277,9 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
       }
       if (has_x && (r = rotate_x(c, M, gg_x, false, 2 * ch)) != SO2_OK) return r;
       if ((r = gemm_v(c, has_x ? 2 * ch + M : (has_r ? ch + M : M))) != SO2_OK) return r;
-      const float *V = at<float>(ws, P.V);
-      const float *dV = V + (size_t)ch * y.KG;
-      const float *Vt = V + (size_t)2 * ch * y.KG;
+      const float *V = prows(c, P.V, 0);
+      const float *dV = prows(c, P.V, (size_t)ch * y.KG);
+      const float *Vt = prows(c, P.V, (size_t)2 * ch * y.KG);
       if (d_grad_out && N > 0) {
         ScatterTerms t{};
         t.F[0] = V;
@@ -1269,10 +1301,21 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
       if (d_w_rad || d_b_rad) {
         {
           ProfScope ps(5, c.s);
-          DISPATCH_LM(y.L, y.mmax, (k_edge_terms2<MM, ((LC >= 0 && LC <= 4) ? LC : -1)><<<warp_grid(M, 8), 256, 8 * y.dsz * 4, c.s>>>(
-                                y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), grad_out,
-                                has_r ? omega : nullptr, V, has_r ? dV : nullptr,
-                                has_x ? Vt : nullptr, at<float>(ws, P.tA), at<float>(ws, P.tB))));
+#define SO2_ET2_LAUNCH(TF)                                                                     \
+  DISPATCH_LM(y.L, y.mmax,                                                                     \
+              (k_edge_terms2<MM, ((LC >= 0 && LC <= 4) ? LC : -1), TF>                          \
+               <<<warp_grid(M, 8), 256, 8 * y.dsz * 4, c.s>>>(                                   \
+                   y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), grad_out,                  \
+                   has_r ? omega : nullptr, reinterpret_cast<const TF *>(V),                    \
+                   has_r ? reinterpret_cast<const TF *>(dV) : nullptr,                          \
+                   has_x ? reinterpret_cast<const TF *>(Vt) : nullptr, at<float>(ws, P.tA),     \
+                   at<float>(ws, P.tB))))
+          if (P.split) {
+            SO2_ET2_LAUNCH(float);
+          } else {
+            SO2_ET2_LAUNCH(__nv_bfloat16);
+          }
+#undef SO2_ET2_LAUNCH
           CKL();
         }
         if ((r = rad_grads(c, M, at<float>(ws, P.tA), has_r ? at<float>(ws, P.tB) : nullptr,
