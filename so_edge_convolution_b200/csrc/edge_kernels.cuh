@@ -38,6 +38,9 @@ namespace so2 {
 #define SO2_ROT_MINB_L6 3
 #endif
 
+// Largest number of radial basis functions (the ABI allows 2..64).
+constexpr int RAD_MAX_NR = 64;
+
 // Keeps the compiler from moving loads across this point.
 __device__ __forceinline__ void load_fence() { asm volatile("" ::: "memory"); }
 
@@ -143,21 +146,40 @@ __global__ void k_place(const int64_t *__restrict__ keys, int64_t E, int64_t N,
 }
 
 // Within each key's segment, order the edge ids ascending, which makes the
-// sort stable and deterministic.  One warp per segment: segments of up to 32
-// edges are placed by rank (each lane counts the smaller ids); longer ones
-// fall back to an insertion sort by lane 0.
+// sort stable and deterministic.  One warp per segment: segments of up to
+// 128 edges are placed by rank (each lane holds up to four ids and counts,
+// for each, the smaller ids of the segment; ids are distinct, so the ranks
+// are a permutation); longer ones fall back to an insertion sort by lane 0.
 __global__ void k_sort_segments(const int *__restrict__ offsets, int64_t N, int *__restrict__ perm) {
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  constexpr int PER = 4;
   for (int64_t n = blockIdx.x * (int64_t)wpb + (threadIdx.x >> 5); n < N;
        n += (int64_t)gridDim.x * wpb) {
     const int b = offsets[n], e = offsets[n + 1], len = e - b;
     if (len <= 1) continue;
-    if (len <= 32) {
-      const int v = lane < len ? perm[b + lane] : 0x7fffffff;
-      int rank = 0;
-      for (int j = 0; j < len; ++j) rank += (__shfl_sync(0xffffffffu, v, j) < v);
+    if (len <= 32 * PER) {
+      int v[PER], rank[PER];
+#pragma unroll
+      for (int q = 0; q < PER; ++q) {
+        const int k = lane + 32 * q;
+        v[q] = k < len ? perm[b + k] : 0x7fffffff;
+        rank[q] = 0;
+      }
+      const int nq = (len + 31) / 32;  // warp-uniform
+      for (int q2 = 0; q2 < nq; ++q2) {
+        for (int j = 0; j < 32; ++j) {
+          int u = v[0];
+#pragma unroll
+          for (int q = 1; q < PER; ++q) u = (q2 == q) ? v[q] : u;
+          const int w = __shfl_sync(0xffffffffu, u, j);
+#pragma unroll
+          for (int q = 0; q < PER; ++q) rank[q] += (w < v[q]);
+        }
+      }
       __syncwarp();
-      if (lane < len) perm[b + rank] = v;
+#pragma unroll
+      for (int q = 0; q < PER; ++q)
+        if (lane + 32 * q < len) perm[b + rank[q]] = v[q];
     } else if (lane == 0) {
       for (int i = b + 1; i < e; ++i) {
         const int v = perm[i];
@@ -1067,26 +1089,47 @@ __global__ void k_unstack_grad(Layout y, BlockOffsets bo, const float *__restric
 // where v (mixing output) and Ga (gradient of the rotated input) come from
 // the two products.  h_x, h_y give the frame part of dL/dr.
 // ---------------------------------------------------------------------------
-// PART: 3 = both sides in one pass; 1 = output side only (writes Gg and h);
-// 2 = input side only (adds its share to h).  With gv_hi, the output side
-// also writes g * (D G[dst]) on the kept rows as the transposed product's
-// operand planes (what rotation on gather of G would write).
+// PART: 3 = both sides in one pass; 1 = output side only (writes Gg and the
+// record h); 2 = input side only (adds its share to h and finishes the edge's
+// gradient).  With gv_hi, the output side also writes g * (D G[dst]) on the
+// kept rows as the transposed product's operand planes (what rotation on
+// gather of G would write).
+//
+// The record h[i] = (h_x, h_y, dd, -) carries the edge's sums from the output
+// side to the input side, where
+//   dL/dr = R^T (-h_y, h_x, 0) / d + dd r_hat,
+//   dd = sum_c' Gg[c'] sum_k W_rad[k][c'] phi'_k(d)
+// (the frame part through the rotation generators, the gate part through the
+// derivative of the radial basis).  grad_r (indexed by the caller's edge id)
+// is written when the input side runs and grad_r is given.
 template <typename TX, int MM, int LC = -1, int PART = 3, typename TF = float>
 __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MINB) k_edge_terms(Layout y, int M, const EdgeRec *__restrict__ rec,
                              const float *__restrict__ D, const float *__restrict__ gate,
                              const float *__restrict__ G, const TX *__restrict__ X,
                              const TF *__restrict__ V, const TF *__restrict__ Ga,
-                             float *__restrict__ Gg, float *__restrict__ h,
-                             __nv_bfloat16 *__restrict__ gv_hi, __nv_bfloat16 *__restrict__ gv_lo) {
+                             float *__restrict__ Gg, float4 *__restrict__ h,
+                             __nv_bfloat16 *__restrict__ gv_hi, __nv_bfloat16 *__restrict__ gv_lo,
+                             const float *__restrict__ geo, const float *__restrict__ w_rad,
+                             float cutoff, float *__restrict__ grad_r) {
   constexpr int W = MM + 1;  // widest |m| needed by the generators
-  extern __shared__ float sDall[];  // [warps][dsz]
+  extern __shared__ float sDall[];  // [warps][dsz + RAD_MAX_NR]
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
-  float *sD = sDall + (threadIdx.x >> 5) * y.dsz;
+  float *sD = sDall + (threadIdx.x >> 5) * (y.dsz + RAD_MAX_NR);
+  float *sPhi = sD + y.dsz;  // phi'_k(d) of the warp's edge
+  const float sig = cutoff / static_cast<float>(y.nr - 1);
   for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
     const EdgeRec r = rec[i];
     __syncwarp();
     stage_d(D + (int64_t)i * y.dsz, y.dsz, sD);
-    float hx = 0.f, hy = 0.f;
+    float hx = 0.f, hy = 0.f, dd = 0.f;
+    if (PART & 1) {  // phi'_k(d), for the output side's gate part
+      const float d = geo[(int64_t)i * GEO];
+      for (int k = lane; k < y.nr; k += 32) {
+        const float t = (d - sig * static_cast<float>(k)) / sig;
+        sPhi[k] = (-t / sig) * __expf(-0.5f * t * t);
+      }
+      __syncwarp();
+    }
     // output side
     const float *Gn = G + (int64_t)r.dst * y.S * y.co;
     const TF *Vi = V + (int64_t)i * y.KG;
@@ -1145,6 +1188,17 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
         }
       });
       *reinterpret_cast<float4 *>(Gg + (int64_t)i * y.co + c) = gg;
+      // dd share of these four channels: Gg . (W_rad^T phi'(d))
+      float4 dg = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = 0; k < y.nr; ++k) {
+        const float dk = sPhi[k];
+        const float4 wk = __ldg(reinterpret_cast<const float4 *>(w_rad + (int64_t)k * y.co + c));
+        dg.x += wk.x * dk;
+        dg.y += wk.y * dk;
+        dg.z += wk.z * dk;
+        dg.w += wk.w * dk;
+      }
+      dd += gg.x * dg.x + gg.y * dg.y + gg.z * dg.z + gg.w * dg.w;
     }
     if ((PART & 1) && gv_hi) {
       for (int g = 0; g < y.ng; ++g)
@@ -1202,55 +1256,26 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
     for (int o = 16; o > 0; o >>= 1) {
       hx += __shfl_xor_sync(0xffffffffu, hx, o);
       hy += __shfl_xor_sync(0xffffffffu, hy, o);
+      dd += __shfl_xor_sync(0xffffffffu, dd, o);
     }
     if (lane == 0) {
-      if (PART & 1) {
-        h[2 * (int64_t)i] = hx;
-        h[2 * (int64_t)i + 1] = hy;
+      if (!(PART & 1)) {  // the output side's sums
+        const float4 ho = h[i];
+        hx += ho.x;
+        hy += ho.y;
+        dd = ho.z;
+      }
+      if ((PART & 2) && grad_r) {
+        const float *gr = geo + (int64_t)i * GEO;
+        const float d = gr[0];
+        const float inv = d > 0.f ? 1.f / d : 0.f;
+        const float *R = gr + 4;
+        for (int a = 0; a < 3; ++a)
+          grad_r[3 * (int64_t)r.eid + a] =
+              (R[0 * 3 + a] * (-hy) + R[1 * 3 + a] * hx) * inv + dd * gr[1 + a];
       } else {
-        h[2 * (int64_t)i] += hx;
-        h[2 * (int64_t)i + 1] += hy;
+        h[i] = make_float4(hx, hy, dd, 0.f);
       }
-    }
-  }
-}
-
-// grad_r[eid] = R^T (-h_y, h_x, 0) / d + (sum_c' Gg[c'] sum_k W_rad[k][c'] phi'_k(d)) r_hat.
-// One warp per edge; phi'_k(d) is computed once per edge (lanes over k).
-__global__ void k_edge_final(Layout y, float cutoff, int M, const EdgeRec *__restrict__ rec,
-                             const float *__restrict__ geo, const float *__restrict__ Gg,
-                             const float *__restrict__ h, const float *__restrict__ w_rad,
-                             float *__restrict__ grad_r) {
-  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
-  const float sig = cutoff / static_cast<float>(y.nr - 1);
-  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
-    const float *gr = geo + (int64_t)i * GEO;
-    const float d = gr[0];
-    float dphi[2];  // k = lane, lane + 32
-    for (int u = 0; u < 2; ++u) {
-      const int k = lane + 32 * u;
-      const float t = (d - sig * static_cast<float>(k)) / sig;
-      dphi[u] = (k < y.nr) ? (-t / sig) * __expf(-0.5f * t * t) : 0.f;
-    }
-    float dd = 0.f;
-    // every lane runs every shuffle: the channel loop is warp-uniform
-    for (int c0 = 0; c0 < y.co; c0 += 32) {
-      const int c = c0 + lane;
-      float dg = 0.f;
-      for (int k = 0; k < y.nr; ++k) {
-        const float dk = __shfl_sync(0xffffffffu, dphi[k >> 5], k & 31);
-        if (c < y.co) dg += w_rad[k * y.co + c] * dk;
-      }
-      if (c < y.co) dd += Gg[(int64_t)i * y.co + c] * dg;
-    }
-    for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
-    if (lane == 0) {
-      const float hx = h[2 * (int64_t)i], hy = h[2 * (int64_t)i + 1];
-      const float inv = d > 0.f ? 1.f / d : 0.f;
-      const float *R = gr + 4;
-      const int e = rec[i].eid;
-      for (int a = 0; a < 3; ++a)
-        grad_r[3 * (int64_t)e + a] = (R[0 * 3 + a] * (-hy) + R[1 * 3 + a] * hx) * inv + dd * gr[1 + a];
     }
   }
 }
@@ -1262,7 +1287,6 @@ __global__ void k_edge_final(Layout y, float cutoff, int M, const EdgeRec *__res
 // in registers and reads each product once.  Stage 2 adds the blocks in
 // order.
 constexpr int RAD_TILE = 64;
-constexpr int RAD_MAX_NR = 64;
 __global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__restrict__ geo,
                               const float *__restrict__ Ag, const float *__restrict__ Bg,
                               const float *__restrict__ omega, float *__restrict__ part) {

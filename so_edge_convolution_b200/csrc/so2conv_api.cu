@@ -210,7 +210,7 @@ Plan make_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
     p.gv_lo = take(c, 2ull * ngv * p.chunk * y.KG * lo);
     p.Ga = take(c, pe * ngv * p.chunk * y.KA);
     p.Gg = take(c, 4ull * p.chunk * y.co);
-    p.h = take(c, 8ull * p.chunk);
+    p.h = take(c, 16ull * p.chunk);
     p.dws = take(c, 4ull * y.WR * y.WK);
     p.radp = take(c, 4ull * ((p.chunk + RAD_TILE - 1) / RAD_TILE) * (y.nr + 1) * y.co);
   }
@@ -923,18 +923,21 @@ so2_status rad_grads(Ctx &c, int M, const float *Ag, const float *Bg, const floa
 
 // Per-edge gradient terms of the backward (see k_edge_terms): part 1 the
 // output side (Gg, h; with write_gv also the transposed product's operand
-// planes), part 2 the input side (adds to h).
+// planes), part 2 the input side (adds to h and writes grad_r).
 so2_status edge_terms(Ctx &c, int M, int part, const void *x, const float *grad_out,
-                      bool write_gv) {
+                      bool write_gv, const float *w_rad = nullptr, float *grad_r = nullptr) {
   const Plan &P = c.P;
   const Layout &y = P.y;
   ProfScope ps(5, c.s);
-  const int sm = 8 * y.dsz * 4;
+  const int sm = 8 * (y.dsz + RAD_MAX_NR) * 4;
   const int g = warp_grid(M, 8);
   const EdgeRec *rec = at<EdgeRec>(c.ws, P.rec);
   const float *Dp = at<float>(c.ws, P.D), *gate = at<float>(c.ws, P.gate);
   const float *Vp = prows(c, P.V, 0), *Gap = prows(c, P.Ga, 0);
-  float *Ggp = at<float>(c.ws, P.Gg), *hp = at<float>(c.ws, P.h);
+  float *Ggp = at<float>(c.ws, P.Gg);
+  float4 *hp = at<float4>(c.ws, P.h);
+  const float *geo = at<float>(c.ws, P.geo);
+  const float cut = c.d->rbf_cutoff;
   __nv_bfloat16 *gh = write_gv ? at<__nv_bfloat16>(c.ws, P.gv_hi) : nullptr;
   __nv_bfloat16 *gl = write_gv && P.split ? at<__nv_bfloat16>(c.ws, P.gv_lo) : nullptr;
 #define SO2_ET_LAUNCH(TX, TF)                                                                \
@@ -944,11 +947,11 @@ so2_status edge_terms(Ctx &c, int M, int part, const void *x, const float *grad_
               if (part == 1) k_edge_terms<TX, MM, LE, 1, TF><<<g, 256, sm, c.s>>>(             \
                   y, M, rec, Dp, gate, grad_out, static_cast<const TX *>(x),                  \
                   reinterpret_cast<const TF *>(Vp), reinterpret_cast<const TF *>(Gap), Ggp,   \
-                  hp, gh, gl);                                                                \
+                  hp, gh, gl, geo, w_rad, cut, nullptr);                                      \
               else k_edge_terms<TX, MM, LE, 2, TF><<<g, 256, sm, c.s>>>(                       \
                   y, M, rec, Dp, gate, grad_out, static_cast<const TX *>(x),                  \
                   reinterpret_cast<const TF *>(Vp), reinterpret_cast<const TF *>(Gap), Ggp,   \
-                  hp, nullptr, nullptr);)
+                  hp, nullptr, nullptr, geo, w_rad, cut, grad_r);)
   if (P.xbf16) {
     SO2_ET_LAUNCH(__nv_bfloat16, __nv_bfloat16)
   } else {
@@ -1132,7 +1135,7 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
     // terms when they run (they rotate G[dst] anyway), else by rotation on gather
     if (need_v) {
       if ((r = gemm_v(c, M)) != SO2_OK) return r;
-      if ((r = edge_terms(c, M, 1, x, grad_out, true)) != SO2_OK) return r;
+      if ((r = edge_terms(c, M, 1, x, grad_out, true, prm.w_rad)) != SO2_OK) return r;
     } else if ((r = rotate_g(c, M, grad_out, 0, arr(at<float>(ws, P.gate)))) != SO2_OK) {
       return r;
     }
@@ -1152,15 +1155,9 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
         (r = reduce_nodes(c, e0, M, prows(c, P.Ga, 0), y.KA, nullptr, 0, grad_x)) != SO2_OK)
       return r;
     if (need_v) {
-      if (grad_edge_vec && (r = edge_terms(c, M, 2, x, grad_out, false)) != SO2_OK) return r;
-      if (grad_edge_vec) {
-        ProfScope ps(5, c.s);
-        k_edge_final<<<warp_grid(M, 8), 256, 0, c.s>>>(y, desc->rbf_cutoff, M,
-                                                        at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo),
-                                                        at<float>(ws, P.Gg), at<float>(ws, P.h),
-                                                        prm.w_rad, grad_edge_vec);
-        CKL();
-      }
+      if (grad_edge_vec &&
+          (r = edge_terms(c, M, 2, x, grad_out, false, prm.w_rad, grad_edge_vec)) != SO2_OK)
+        return r;
       if ((grad_w_rad || grad_b_rad) &&
           (r = rad_grads(c, M, at<float>(ws, P.Gg), nullptr, nullptr, grad_w_rad, grad_b_rad)) !=
               SO2_OK)
