@@ -8,11 +8,17 @@ f32).  Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (torchrun, one process per GPU) every rank runs its own copy of
-the workload: independent graphs, no collective on the data path ("weak"
-scaling); the barrier and the max-over-ranks of the timed region are the only
-cross-rank steps.  ``--impl reference`` times the float64 CPU oracle on a
-bounded sample of the same workload on the host cores (rank 0 only).
+With N > 1 (torchrun, one process per GPU) the default (``--split dst``)
+runs ONE graph of N times the workload's atoms (same density, so about N
+times the edges) split over the ranks by destination node: each rank owns a
+contiguous node range and the edges into it; node features are all-gathered
+before the convolution, grad_x is reduce-scattered to its owners and the
+weight gradients are all-reduced (NCCL).  Per-GPU work stays that of the
+one-GPU workload ("weak" scaling).  ``--split replicas`` runs an independent
+copy of the workload per rank instead (no collective on the data path).
+The barrier and the max-over-ranks of the timed region bracket every step.
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the
+same workload on the host cores (rank 0 only).
 """
 
 import argparse
@@ -94,23 +100,28 @@ def kernel_traffic(config):
     return rec
 
 
-def compulsory_bytes(config, t, p):
+def compulsory_bytes(config, p, n_nodes, n_edges):
     """Bytes of every input and output tensor of the step's library calls,
-    each touched once per call (the HBM floor of the step)."""
-    nb = lambda x: x.numel() * x.element_size()  # noqa: E731
-    node_out = p.n_nodes * (p.lmax + 1) ** 2 * p.c_out * 4
-    node_in = p.n_nodes * (p.lmax + 1) ** 2 * p.c_in * 4
-    nw = t["w"].numel() * 4  # gradients are f32
-    shared = sum(nb(t[k]) for k in ("x", "edge_index", "edge_vec", "w", "w_rad", "b_rad"))
+    each touched once per call (the HBM floor of the step), for calls over
+    n_nodes node rows and n_edges edges."""
+    S = (p.lmax + 1) ** 2
+    xe = 2 if p.x_bf16 else 4
+    we = 2 if p.w_bf16 else 4
+    nw = sum(r * k for r, k in synth.weight_block_shapes(p.lmax, p.mmax, p.c_in, p.c_out))
+    x = n_nodes * S * p.c_in * xe
+    node_out = n_nodes * S * p.c_out * 4
+    node_in = n_nodes * S * p.c_in * 4
+    G = node_out
+    ev = n_edges * 3 * 4
     rad = (p.n_rbf + 1) * p.c_out * 4
-    ev = nb(t["edge_vec"])
+    shared = x + n_edges * 2 * 8 + ev + nw * we + rad
     fwd = shared + node_out
     if config == "md":
-        return fwd + shared + nb(t["grad_out"]) + ev
-    bwd = shared + nb(t["grad_out"]) + node_in + nw + rad + ev
+        return fwd + shared + G + ev
+    bwd = shared + G + node_in + nw * 4 + rad + ev
     if config == "force":
-        bwd_r = shared + nb(t["grad_out"]) + ev
-        dbl = shared + nb(t["grad_out"]) + ev + nw + rad
+        bwd_r = shared + G + ev
+        dbl = shared + G + ev + nw * 4 + rad
         return fwd + bwd_r + dbl
     return fwd + bwd
 
@@ -276,6 +287,47 @@ def run_reference(args, world, rank):
 
 
 # ---------------------------------------------------------------------------
+# One graph split by destination over the ranks
+# ---------------------------------------------------------------------------
+def dst_problem(prob, world, n_atoms=None, **overrides):
+    """The job's graph: the workload's generator with world x its atoms (the
+    periodic box grows with the atom count, so the density and the edges per
+    atom stay those of the one-GPU workload).  n_atoms (per rank) and the
+    other overrides shrink it for tests."""
+    base = synth.CONFIGS[prob]["n_atoms"] if n_atoms is None else n_atoms
+    return synth.make_problem(prob, seed=0, n_atoms=base * world, **overrides)
+
+
+def dst_inputs(p, sg, xdt, wdt):
+    """This rank's host inputs: its node rows of x and grad_out, its edges."""
+    T = torch.from_numpy
+    return {
+        "x": sg.local_rows(T(p.x).to(xdt)),
+        "edge_index": sg.edge_index.clone(),
+        "edge_vec": sg.edge_vec.to(torch.float32).clone(),
+        "w": T(p.w).to(wdt),
+        "w_rad": T(p.w_rad.astype(np.float32)),
+        "b_rad": T(p.b_rad.astype(np.float32)),
+        "grad_out": sg.local_rows(T(p.grad_out.astype(np.float32))),
+    }
+
+
+def make_dst_step(sg, desc, op=None):
+    """forward + backward of the rank's share (sharded.forward / backward)
+    on the inputs in `t` (as dst_inputs lays them out)."""
+    import copy
+    from so_edge_convolution_b200 import sharded as S
+
+    def step(t, o=None):
+        v = copy.copy(sg)
+        v.edge_index, v.edge_vec = t["edge_index"], t["edge_vec"]
+        out = S.forward(v, desc, t["x"], t["w"], t["w_rad"], t["b_rad"], op=op)
+        g = S.backward(v, desc, t["x"], t["w"], t["w_rad"], t["b_rad"], t["grad_out"], op=op)
+        return out, g
+    return step
+
+
+# ---------------------------------------------------------------------------
 # The CUDA path
 # ---------------------------------------------------------------------------
 def run_ours(args, world, rank, local):
@@ -285,8 +337,13 @@ def run_ours(args, world, rank, local):
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
     prob, workload, n_products, n_executed = CONFIGS[args.config]
-    p = synth.make_problem(prob, seed=rank)
-    E = p.n_edges
+    split = args.split if args.split != "auto" else ("dst" if world > 1 else "replicas")
+    if split == "dst" and world == 1:
+        split = "replicas"  # one rank owns the whole graph
+    if split == "dst" and args.config in ("force", "md"):
+        raise SystemExit("--split dst runs the forward + backward workloads")
+    p = dst_problem(prob, world) if split == "dst" else synth.make_problem(prob, seed=rank)
+    E = p.n_edges  # edges this rank's library calls process (set below for dst)
     bf16 = p.x_bf16
     xdt = torch.bfloat16 if bf16 else torch.float32
     wdt = torch.bfloat16 if bf16 else torch.float32
@@ -302,6 +359,14 @@ def run_ours(args, world, rank, local):
         "grad_out": torch.from_numpy(p.grad_out.astype(np.float32)).pin_memory(),
         "f_ref": torch.from_numpy(p.f_ref.astype(np.float32)).pin_memory(),
     }
+    sg = None
+    if split == "dst":
+        from so_edge_convolution_b200 import sharded as S
+        sg = S.ShardedGraph(torch.from_numpy(p.edge_index), torch.from_numpy(p.edge_vec),
+                            p.n_nodes, rank, world)
+        host = {k: v.pin_memory() for k, v in dst_inputs(p, sg, xdt, wdt).items()}
+        E = int(sg.edge_ids.numel())
+    E_job = p.n_edges if split == "dst" else world * E
     d = {k: v.to(dev) for k, v in host.items()}
     ws = B.Workspace(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -349,6 +414,9 @@ def run_ours(args, world, rank, local):
         return out, {"grad_edge_vec": gr, "forces": F}
 
     step = {"force": step_force, "md": step_md}.get(args.config, step_fwd_bwd)
+    if split == "dst":
+        step = make_dst_step(sg, desc)
+        ws = None  # the sharded calls use the binding's own per-device workspace
 
     for _ in range(max(args.warmup, 3)):
         step(d)
@@ -382,7 +450,7 @@ def run_ours(args, world, rank, local):
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * E * args.steps / (total_ms * 1e-3)
+    value = E_job * args.steps / (total_ms * 1e-3)
 
     # ---- roofline (SURVEY-style accounting: algorithmic mixing FLOPs only) ----
     # The bound is the tensor-core one (compulsory bytes are ~30x below it).
@@ -400,7 +468,7 @@ def run_ours(args, world, rank, local):
     peak_tf = pk["bf16_tflops"] * tf32_ratio
     peak_tf_sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * tf32_ratio
     step_tflops = alg_flops / (total_ms * 1e-3) / 1e12
-    cbytes = compulsory_bytes(args.config, d, p)
+    cbytes = compulsory_bytes(args.config, p, sg.n_pad if sg is not None else p.n_nodes, E)
     t_roof_ms = max(n_products * fpe * E / (peak_tf * 1e12),
                     cbytes / (pk["hbm_gbs"] * 1e9)) * 1e3
     traffic = kernel_traffic(args.config)
@@ -493,7 +561,7 @@ def run_ours(args, world, rank, local):
     e2e_e.record(comp)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e2e_s.elapsed_time(e2e_e), world, dev) / n_e2e
-    e2e = {"value": world * E / (e2e_ms * 1e-3), "unit": "edges/s",
+    e2e = {"value": E_job / (e2e_ms * 1e-3), "unit": "edges/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
            "copies": "pinned host buffers, every step, on copy streams overlapping the "
                      "neighbouring steps' kernels"}
@@ -512,9 +580,13 @@ def run_ours(args, world, rank, local):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16" if bf16 else "f32", "data": "synthetic",
-                "config": {"workload": workload, "edges": E, "nodes": p.n_nodes,
+                "config": {"workload": workload if split != "dst" else
+                           workload + f"; one graph of {world} x the atoms split by destination",
+                           "edges": E_job, "edges_per_rank": E, "nodes": p.n_nodes,
                            "l2": "flushed between timed steps (256 MB write)",
-                           "parallelism": f"replicas x{world}" if world > 1 else "single"},
+                           "parallelism": (f"dst-split x{world} (all-gather x, reduce-scatter "
+                                           "grad_x, all-reduce grad_W; NCCL)" if split == "dst"
+                                           else f"replicas x{world}" if world > 1 else "single")},
                 "step_roofline_frac": roofline["step_roofline_frac"],
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches, "clocks": clk, "breakdown_ms_per_step": breakdown}
@@ -530,6 +602,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--config", choices=sorted(CONFIGS), default="esen",
                     help="workload (the headline line is esen; the others are for study)")
+    ap.add_argument("--split", choices=["auto", "dst", "replicas"], default="auto",
+                    help="N > 1: one graph split by destination (dst, the default) or "
+                         "independent replicas")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:
