@@ -141,9 +141,12 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t n_nodes,
  * "Breaking the Training Barrier of Billion-Parameter Universal Machine
  * Learning Interatomic Potentials", Abstract: training needs second-order
  * derivatives).  gg_x [N, S, c_in], gg_edge_vec [E, 3]; outputs f32 with the
- * layouts of x, w, w_rad, b_rad, grad_out, overwritten; NULL skips one.
- * d_edge_vec (second order in the edge vectors) is not provided: it must be
- * NULL, otherwise SO2_ERR_UNSUPPORTED.  Errors as for so2conv_forward. */
+ * layouts of x, w, w_rad, b_rad, grad_out, edge_vec, overwritten; NULL skips
+ * one.
+ * d_edge_vec [E, 3] (may be NULL) is the derivative with respect to the
+ * edge vectors: the Hessian of each edge's share of <grad_out, out> applied
+ * to gg_edge_vec, plus the edge gradient of the first backward with x
+ * replaced by gg_x.  Errors as for so2conv_forward. */
 so2_status so2conv_double_backward(
     const so2conv_desc *desc, int64_t n_nodes, int64_t n_edges, const void *x,
     const int64_t *edge_index, const float *edge_vec, so2conv_params params,

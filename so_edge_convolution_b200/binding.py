@@ -226,20 +226,20 @@ def double_backward(desc, x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg
     x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg_x, gg_edge_vec = map(
         _c, (x, edge_index, edge_vec, w, w_rad, b_rad, grad_out, gg_x, gg_edge_vec))
     N, E = x.shape[0], edge_index.shape[1]
-    names = ["d_x", "d_w", "d_w_rad", "d_b_rad", "d_grad_out"]
+    names = ["d_x", "d_w", "d_w_rad", "d_b_rad", "d_grad_out", "d_edge_vec"]
     need = set(names if need is None else need)
     dev = x.device
     f32 = dict(dtype=torch.float32, device=dev)
     S = (desc.lmax + 1) ** 2
     shapes = {"d_x": (N, S, desc.c_in), "d_w": (num_weights(desc),),
               "d_w_rad": (desc.n_rbf, desc.c_out), "d_b_rad": (desc.c_out,),
-              "d_grad_out": (N, S, desc.c_out)}
+              "d_grad_out": (N, S, desc.c_out), "d_edge_vec": (E, 3)}
     outs = _outputs(names, need, shapes, out, f32)
     p, nb = _wsarg(desc, N, E, WS_DOUBLE_BACKWARD, dev, ws)
     code = lib.so2conv_double_backward(
         ctypes.byref(desc), N, E, _ptr(x), _ptr(edge_index), _ptr(edge_vec),
         Params(w.data_ptr(), w_rad.data_ptr(), b_rad.data_ptr()), _ptr(grad_out),
-        _ptr(gg_x), _ptr(gg_edge_vec), *[_ptr(outs[n]) for n in names], None, p, nb,
+        _ptr(gg_x), _ptr(gg_edge_vec), *[_ptr(outs[n]) for n in names], p, nb,
         _stream(dev))
     _check_call(code, "so2conv_double_backward")
     return {n: t for n, t in outs.items() if t is not None}

@@ -1487,6 +1487,296 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
   }
 }
 
+// ---------------------------------------------------------------------------
+// Second order in the edge vectors (d_edge_vec of the double backward).
+//
+// With u = gg_r (the cotangent on grad_edge_vec) and ~x = gg_x,
+//   d_edge_vec_e = H_e u_e + dL_e/dr_e |_{x := ~x},
+// H_e the Hessian of the edge's share L_e = <b, g * V> of <grad_out, out>
+// (b = trunc(D G[dst]), V = M trunc(D x[src])).  In the edge frame (R r_hat =
+// z_hat, U = R u) a second direction W turns the frame by
+//   omega_W = (W_y, -W_x) / d,   and jointly with u by
+//   omega_uW = -(W_z omega_u + U_z omega_W) / d,
+// so d2D[u, W] = (Omega_uW + (Omega_u Omega_W + Omega_W Omega_u) / 2) D (the
+// roll parts drop out: L_e does not depend on the roll), and the gate moves
+// by g_W = g' W_z, g_uW = g'' U_z W_z + g' (U_perp . W_perp) / d.  For the
+// edge-frame axes W = x, y, z this gives (with J_x, J_y the generators,
+// Omega_u = alpha J_x + beta J_y, (alpha, beta) = omega_u):
+//   X_x = (U_z/d^2) J_y - (alpha / 2d)(J_x J_y + J_y J_x) - (beta/d) J_y^2
+//   X_y = -(U_z/d^2) J_x + (alpha/d) J_x^2 + (beta / 2d)(J_x J_y + J_y J_x)
+//   q_z = -F_D[Omega_u]/d + <Omega_u b, g' V> + <g' b, dV> + U_z <g'', Gg>
+//   q_x = F_D[X_x] + <g (-J_y b / d), dV> + U_z <(-J_y b / d), g' V>
+//         + <M^T P, -J_y a / d> + (U_x / d) <g', Gg>
+//   q_y = F_D[X_y] + <g (J_x b / d), dV> + U_z <(J_x b / d), g' V>
+//         + <M^T P, J_x a / d> + (U_y / d) <g', Gg>
+// where F_D[X] = <X b, g V> + <Ga, X a>, a = trunc(D x), dV = M trunc(Omega_u
+// D x), Ga = M^T (g b), M^T P = M^T (g Omega_u b + g_u b) (the double
+// backward's products) and Gg[c'] = sum_rows b V.  The ~x part is the first
+// backward's edge gradient: (-h_y / d, h_x / d, <g', sum_rows b ~V>) with
+// h_k = <g ~V, J_k b> + <Ga, J_k ~a>, ~a = trunc(D ~x), ~V = M ~a.
+// H u = R^T q.  The terms split by what they read: the output side (b, V,
+// dV, ~V; destination order) and the input side (a, ~a, Ga, M^T P; source
+// order); each side adds R^T of its share onto d_edge_vec[eid].
+// ---------------------------------------------------------------------------
+
+// (J_x c)[m], (J_y c)[m] and the second-order (J_x J_x c)[m], (J_y J_y c)[m],
+// ((J_x J_y + J_y J_x) c)[m] for one degree-l coefficient vector given by
+// its accessor (zero outside |q| <= l).
+template <typename F>
+__device__ __forceinline__ void gen_xy2(int l, int m, F c, float &jx, float &jy, float &xx,
+                                        float &yy, float &sym) {
+  auto cc = [&](int q) { return (q < -l || q > l) ? 0.f : c(q); };
+  gen_xy(l, m, cc, jx, jy);
+  auto jxc = [&](int q) {
+    if (q < -l || q > l) return 0.f;
+    float a, b;
+    gen_xy(l, q, cc, a, b);
+    return a;
+  };
+  auto jyc = [&](int q) {
+    if (q < -l || q > l) return 0.f;
+    float a, b;
+    gen_xy(l, q, cc, a, b);
+    return b;
+  };
+  float yx, xy;
+  gen_xy(l, m, jxc, xx, yx);  // xx = J_x J_x c, yx = J_y J_x c
+  gen_xy(l, m, jyc, xy, yy);  // xy = J_x J_y c, yy = J_y J_y c
+  sym = xy + yx;
+}
+
+__device__ __forceinline__ float comp4(const float4 &v, int k) {
+  return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
+}
+
+// The edge-frame share q (3 floats, summed over the warp) rotated back and
+// added onto d_edge_vec[eid] (one writer per edge per launch; launches run in
+// stream order).
+__device__ __forceinline__ void hess_flush(const float *gr, int eid, float qx, float qy, float qz,
+                                           float *__restrict__ d_r) {
+  const float *R = gr + 4;
+#pragma unroll
+  for (int a = 0; a < 3; ++a)
+    d_r[3 * (int64_t)eid + a] += R[0 * 3 + a] * qx + R[1 * 3 + a] * qy + R[2 * 3 + a] * qz;
+}
+
+// Output side, destination order.  omega (w_x, w_y, U_z per edge) and dV are
+// given with an edge-vector cotangent, Vt with gg_x.
+template <int MM, int LC = -1, typename TF = float>
+__global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MINB)
+    k_edge_hess_out(Layout y, float cutoff, int M, const EdgeRec *__restrict__ rec,
+                    const float *__restrict__ D, const float *__restrict__ geo,
+                    const float *__restrict__ gate, const float *__restrict__ G,
+                    const float *__restrict__ omega, const TF *__restrict__ V,
+                    const TF *__restrict__ dV, const TF *__restrict__ Vt,
+                    const float *__restrict__ w_rad, float *__restrict__ d_r) {
+  constexpr int W2 = MM + 2;
+  extern __shared__ float sDall[];  // [warps][dsz + 2 RAD_MAX_NR]
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  float *sD = sDall + (threadIdx.x >> 5) * (y.dsz + 2 * RAD_MAX_NR);
+  float *sP1 = sD + y.dsz, *sP2 = sP1 + RAD_MAX_NR;  // phi'_k(d), phi''_k(d)
+  const float sig = cutoff / static_cast<float>(y.nr - 1);
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
+    const EdgeRec r = rec[i];
+    __syncwarp();
+    stage_d(D + (int64_t)i * y.dsz, y.dsz, sD);
+    const float *gr = geo + (int64_t)i * GEO;
+    const float d = gr[0];
+    const float inv = d > 0.f ? 1.f / d : 0.f;
+    const float al = omega ? omega[4 * (int64_t)i] : 0.f;
+    const float be = omega ? omega[4 * (int64_t)i + 1] : 0.f;
+    const float Uz = omega ? omega[4 * (int64_t)i + 2] : 0.f;
+    const float Ux = -be * d, Uy = al * d;
+    for (int k = lane; k < y.nr; k += 32) {
+      const float t = (d - sig * static_cast<float>(k)) / sig;
+      const float ph = __expf(-0.5f * t * t);
+      sP1[k] = (-t / sig) * ph;
+      sP2[k] = ((t * t - 1.f) / (sig * sig)) * ph;
+    }
+    __syncwarp();
+    const float *Gn = G + (int64_t)r.dst * y.S * y.co;
+    const int64_t ro = (int64_t)i * y.KG;
+    float qx = 0.f, qy = 0.f, qz = 0.f, hx = 0.f, hy = 0.f;
+    for (int c = 4 * lane; c < y.co; c += 128) {
+      const float4 g4 = load4(gate + (int64_t)i * y.co + c);
+      float4 gp4 = make_float4(0.f, 0.f, 0.f, 0.f), gpp4 = gp4;
+      for (int k = 0; k < y.nr; ++k) {
+        const float4 wk = __ldg(reinterpret_cast<const float4 *>(w_rad + (int64_t)k * y.co + c));
+        const float p1 = sP1[k], p2 = sP2[k];
+        gp4.x += wk.x * p1;
+        gp4.y += wk.y * p1;
+        gp4.z += wk.z * p1;
+        gp4.w += wk.w * p1;
+        gpp4.x += wk.x * p2;
+        gpp4.y += wk.y * p2;
+        gpp4.z += wk.z * p2;
+        gpp4.w += wk.w * p2;
+      }
+      float Gg[4] = {0.f, 0.f, 0.f, 0.f}, Ggt[4] = {0.f, 0.f, 0.f, 0.f};
+      each_level<LC>(y.L, [&](auto lv) {
+        constexpr int l = decltype(lv)::value;
+        constexpr int w = 2 * l + 1;
+        constexpr int mb = W2 < l ? W2 : l, mm = MM < l ? MM : l;
+        float4 b[2 * W2 + 1];
+#pragma unroll
+        for (int k = 0; k < 2 * W2 + 1; ++k) b[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *Dl = sD + dblock_off(l);
+#pragma unroll
+        for (int mp = -l; mp <= l; ++mp) {
+          const float4 gx = load4(Gn + (l * l + l + mp) * y.co + c);
+#pragma unroll
+          for (int m = -mb; m <= mb; ++m) {
+            const float dv = Dl[(m + l) * w + mp + l];
+            b[m + W2].x += dv * gx.x;
+            b[m + W2].y += dv * gx.y;
+            b[m + W2].z += dv * gx.z;
+            b[m + W2].w += dv * gx.w;
+          }
+        }
+#pragma unroll
+        for (int m = -mm; m <= mm; ++m) {
+          int g, j;
+          lm_group_row(y, l, m, g, j);
+          const int64_t col = ro + y.kout_off[g] + j * y.co + c;
+          const float4 v4 = load4(V + col);
+          const float4 dv4 = dV ? load4(dV + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 vt4 = Vt ? load4(Vt + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            auto bk = [&](int q) { return (q < -mb || q > mb) ? 0.f : comp4(b[q + W2], k); };
+            float jx, jy, xx, yy, sym;
+            gen_xy2(l, m, bk, jx, jy, xx, yy, sym);
+            const float bm = comp4(b[m + W2], k);
+            const float v = comp4(v4, k), dvv = comp4(dv4, k), vt = comp4(vt4, k);
+            const float gk = comp4(g4, k), gpk = comp4(gp4, k);
+            const float gv = gk * v, gpv = gpk * v;
+            const float ob = al * jx + be * jy;  // (Omega_u b)[m]
+            const float xxb = Uz * inv * inv * jy - 0.5f * al * inv * sym - be * inv * yy;
+            const float xyb = -Uz * inv * inv * jx + al * inv * xx + 0.5f * be * inv * sym;
+            qz += -inv * ob * gv + ob * gpv + gpk * bm * dvv;
+            qx += xxb * gv - inv * jy * (gk * dvv + Uz * gpv);
+            qy += xyb * gv + inv * jx * (gk * dvv + Uz * gpv);
+            Gg[k] += bm * v;
+            Ggt[k] += bm * vt;
+            hx += gk * vt * jx;
+            hy += gk * vt * jy;
+          }
+        }
+      });
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float gpk = comp4(gp4, k), gppk = comp4(gpp4, k);
+        qz += Uz * gppk * Gg[k] + gpk * Ggt[k];
+        qx += Ux * inv * gpk * Gg[k];
+        qy += Uy * inv * gpk * Gg[k];
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      qx += __shfl_xor_sync(0xffffffffu, qx, o);
+      qy += __shfl_xor_sync(0xffffffffu, qy, o);
+      qz += __shfl_xor_sync(0xffffffffu, qz, o);
+      hx += __shfl_xor_sync(0xffffffffu, hx, o);
+      hy += __shfl_xor_sync(0xffffffffu, hy, o);
+    }
+    if (lane == 0) hess_flush(gr, r.eid, qx - hy * inv, qy + hx * inv, qz, d_r);
+  }
+}
+
+// Input side, source order.  omega and MP (= M^T P) are given with an
+// edge-vector cotangent, GX (= gg_x) with a node cotangent; Ga = M^T (g b).
+template <typename TX, int MM, int LC = -1, typename TF = float>
+__global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MINB)
+    k_edge_hess_in(Layout y, int M, const EdgeRec *__restrict__ rec, const float *__restrict__ D,
+                   const float *__restrict__ geo, const TX *__restrict__ X,
+                   const float *__restrict__ GX, const float *__restrict__ omega,
+                   const TF *__restrict__ Ga, const TF *__restrict__ MP,
+                   float *__restrict__ d_r) {
+  constexpr int W2 = MM + 2;
+  extern __shared__ float sDall[];  // [warps][dsz]
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  float *sD = sDall + (threadIdx.x >> 5) * y.dsz;
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
+    const EdgeRec r = rec[i];
+    __syncwarp();
+    stage_d(D + (int64_t)i * y.dsz, y.dsz, sD);
+    const float *gr = geo + (int64_t)i * GEO;
+    const float d = gr[0];
+    const float inv = d > 0.f ? 1.f / d : 0.f;
+    const float al = omega ? omega[4 * (int64_t)i] : 0.f;
+    const float be = omega ? omega[4 * (int64_t)i + 1] : 0.f;
+    const float Uz = omega ? omega[4 * (int64_t)i + 2] : 0.f;
+    const TX *Xn = X + (int64_t)r.src * y.S * y.ci;
+    const float *GXn = GX ? GX + (int64_t)r.src * y.S * y.ci : nullptr;
+    const int64_t ro = (int64_t)i * y.KA;
+    float qx = 0.f, qy = 0.f, qz = 0.f, hx = 0.f, hy = 0.f;
+    for (int c = 4 * lane; c < y.ci; c += 128) {
+      each_level<LC>(y.L, [&](auto lv) {
+        constexpr int l = decltype(lv)::value;
+        constexpr int w = 2 * l + 1;
+        constexpr int mb = W2 < l ? W2 : l, mm = MM < l ? MM : l;
+        float4 a[2 * W2 + 1], at[2 * W2 + 1];
+#pragma unroll
+        for (int k = 0; k < 2 * W2 + 1; ++k) {
+          a[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          at[k] = a[k];
+        }
+        const float *Dl = sD + dblock_off(l);
+#pragma unroll
+        for (int mp = -l; mp <= l; ++mp) {
+          const float4 xv = load4(Xn + (l * l + l + mp) * y.ci + c);
+          const float4 tv = GXn ? load4(GXn + (l * l + l + mp) * y.ci + c)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int m = -mb; m <= mb; ++m) {
+            const float dv = Dl[(m + l) * w + mp + l];
+            a[m + W2].x += dv * xv.x;
+            a[m + W2].y += dv * xv.y;
+            a[m + W2].z += dv * xv.z;
+            a[m + W2].w += dv * xv.w;
+            at[m + W2].x += dv * tv.x;
+            at[m + W2].y += dv * tv.y;
+            at[m + W2].z += dv * tv.z;
+            at[m + W2].w += dv * tv.w;
+          }
+        }
+#pragma unroll
+        for (int m = -mm; m <= mm; ++m) {
+          int g, j;
+          lm_group_row(y, l, m, g, j);
+          const int64_t col = ro + y.kin_off[g] + j * y.ci + c;
+          const float4 ga4 = load4(Ga + col);
+          const float4 mp4 = MP ? load4(MP + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            auto ak = [&](int q) { return (q < -mb || q > mb) ? 0.f : comp4(a[q + W2], k); };
+            auto tk = [&](int q) { return (q < -mb || q > mb) ? 0.f : comp4(at[q + W2], k); };
+            float jx, jy, xx, yy, sym, tx, ty;
+            gen_xy2(l, m, ak, jx, jy, xx, yy, sym);
+            gen_xy(l, m, tk, tx, ty);
+            const float ga = comp4(ga4, k), mpv = comp4(mp4, k);
+            const float oa = al * jx + be * jy;  // (Omega_u a)[m]
+            const float xxa = Uz * inv * inv * jy - 0.5f * al * inv * sym - be * inv * yy;
+            const float xya = -Uz * inv * inv * jx + al * inv * xx + 0.5f * be * inv * sym;
+            qz += -inv * ga * oa;
+            qx += ga * xxa - inv * mpv * jy;
+            qy += ga * xya + inv * mpv * jx;
+            hx += ga * tx;
+            hy += ga * ty;
+          }
+        }
+      });
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      qx += __shfl_xor_sync(0xffffffffu, qx, o);
+      qy += __shfl_xor_sync(0xffffffffu, qy, o);
+      qz += __shfl_xor_sync(0xffffffffu, qz, o);
+      hx += __shfl_xor_sync(0xffffffffu, hx, o);
+      hy += __shfl_xor_sync(0xffffffffu, hy, o);
+    }
+    if (lane == 0) hess_flush(gr, r.eid, qx - hy * inv, qy + hx * inv, qz, d_r);
+  }
+}
+
 // Frames and full Wigner-D for inspection, with the same per-thread code the
 // op uses.  Block = one warp, 32 edges.
 template <int L>

@@ -780,15 +780,18 @@ so2_status gemm_dw(Ctx &c, int M, int seg_g, int seg_a) {
   return SO2_OK;
 }
 
-// Ga rows = output-side operand rows times the transposed stacked weights.
-so2_status gemm_ga(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store = true) {
+// Ga rows = output-side operand rows times the transposed stacked weights
+// (rows [row0, row0 + rows) of both).
+so2_status gemm_ga(Ctx &c, int rows, const GemmScatter *sc = nullptr, bool store = true,
+                   int row0 = 0) {
   const Plan &P = c.P;
   const Layout &y = P.y;
   const bool pair = sc ? SO2_PAIR_SCATTER : SO2_PAIR_PLAIN;
   GemmLauncher L;
   L.bm = pair ? 2 * GEMM_BM : GEMM_BM;
   for (int g = 0; g < y.ng; ++g)
-    L.add(rows, y.Kin[g], y.Kout_pad[g], 0, y.kout_off[g], y.wt_off[g], 0, y.kin_off[g], y.KA);
+    L.add(rows, y.Kin[g], y.Kout_pad[g], row0, y.kout_off[g], y.wt_off[g], 0,
+          static_cast<long long>(row0) * y.KA + y.kin_off[g], y.KA);
   CK(launch_gemm(1, P.split, c.m_v_hi, c.m_v_lo, pair ? c.m_wtr2_hi : c.m_wtr_hi,
                  pair ? c.m_wtr2_lo : c.m_wtr_lo, L.p, at<float>(c.ws, P.Ga), 0, c.st, c.s, sc,
                  store, false, pair, !P.split));
@@ -1192,7 +1195,6 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
                                    float *d_edge_vec, void *ws, size_t ws_bytes,
                                    so2_stream_t stream) {
   if (!desc) return SO2_ERR_INVALID_ARG;
-  if (d_edge_vec) return SO2_ERR_UNSUPPORTED;
   Plan P;
   so2_status r = common_checks(desc, N, E, x, edge_index, edge_vec, prm, ws, ws_bytes,
                                SO2_WS_DOUBLE_BACKWARD, P);
@@ -1212,6 +1214,7 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
   if (d_w) CK(cudaMemsetAsync(d_w, 0, sizeof(float) * nw, c.s));
   if (d_w_rad) CK(cudaMemsetAsync(d_w_rad, 0, sizeof(float) * y.nr * y.co, c.s));
   if (d_b_rad) CK(cudaMemsetAsync(d_b_rad, 0, sizeof(float) * y.co, c.s));
+  if (d_edge_vec && E > 0) CK(cudaMemsetAsync(d_edge_vec, 0, sizeof(float) * 3 * E, c.s));
   if (!aligned16(gg_x)) return SO2_ERR_INVALID_ARG;
   const bool has_r = gg_edge_vec != nullptr, has_x = gg_x != nullptr;
   if (E == 0 || (!has_r && !has_x)) return SO2_OK;
@@ -1224,36 +1227,64 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
   if (d_w) CK(cudaMemsetAsync(dws, 0, 4ull * y.WR * y.WK, c.s));
   const int ch = P.chunk;
 
-  // ---- pass A (source order): d_x ----
-  if (d_x && has_r) {
+  // ---- pass A (source order): d_x, and the input side of d_edge_vec ----
+  if ((d_x && has_r) || d_edge_vec) {
     if ((r = sort_edges(c, edge_index, 0)) != SO2_OK) return r;
     for (int64_t e0 = 0; e0 < E; e0 += ch) {
       const int M = static_cast<int>((E - e0) < ch ? (E - e0) : ch);
       if ((r = chunk_prep(c, e0, M, edge_index, edge_vec, 0, prm)) != SO2_OK) return r;
-      {
+      if (has_r) {
+        {
+          ProfScope ps(5, c.s);
+          k_edge_omega<<<warp_grid(M, 8), 256, 0, c.s>>>(
+              y, desc->rbf_cutoff, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo), gg_edge_vec,
+              prm.w_rad, at<float>(ws, P.omega), at<float>(ws, P.dgate));
+          CKL();
+        }
+        // P = dg * b + g * Omega b and Gv = g * b from one rotation b = D G[dst]
+        if ((r = rotate_g2(c, M, grad_out, 0, dgate, gate, ch, gate, ZERO, omega)) != SO2_OK)
+          return r;
+        if ((r = gemm_ga(c, ch + M)) != SO2_OK) return r;  // [M^T P; M^T Gv]
+      } else {
+        if ((r = rotate_g(c, M, grad_out, ch, gate)) != SO2_OK) return r;  // Gv = g * b
+        if ((r = gemm_ga(c, M, nullptr, true, ch)) != SO2_OK) return r;    // M^T Gv
+      }
+      if (d_x && has_r) {
+        ScatterTerms t{};
+        t.F[0] = prows(c, P.Ga, 0);
+        t.ld[0] = y.KA;
+        t.A[0] = ONE;
+        t.F[1] = prows(c, P.Ga, (size_t)ch * y.KA);
+        t.ld[1] = y.KA;
+        t.B[1] = ONE;
+        if ((r = scatter(c, e0, M, t, 0, omega, d_x)) != SO2_OK) return r;
+      }
+      if (d_edge_vec) {
         ProfScope ps(5, c.s);
-        k_edge_omega<<<warp_grid(M, 8), 256, 0, c.s>>>(
-            y, desc->rbf_cutoff, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.geo), gg_edge_vec,
-            prm.w_rad, at<float>(ws, P.omega), at<float>(ws, P.dgate));
+        const float *Gap = prows(c, P.Ga, (size_t)ch * y.KA);
+        const float *MPp = has_r ? prows(c, P.Ga, 0) : nullptr;
+        const int sm = 8 * y.dsz * 4;
+#define SO2_HIN_LAUNCH(TX, TF)                                                                 \
+  DISPATCH_LM(y.L, y.mmax, constexpr int LE = (LC >= 0 && LC <= 4) ? LC : -1;                   \
+              k_edge_hess_in<TX, MM, LE, TF><<<warp_grid(M, 8), 256, sm, c.s>>>(                \
+                  y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), at<float>(ws, P.geo),       \
+                  static_cast<const TX *>(x), gg_x, has_r ? omega : nullptr,                    \
+                  reinterpret_cast<const TF *>(Gap), reinterpret_cast<const TF *>(MPp),          \
+                  d_edge_vec);)
+        if (P.xbf16) {
+          SO2_HIN_LAUNCH(__nv_bfloat16, __nv_bfloat16)
+        } else {
+          SO2_HIN_LAUNCH(float, float)
+        }
+#undef SO2_HIN_LAUNCH
         CKL();
       }
-      // P = dg * b + g * Omega b and Gv = g * b from one rotation b = D G[dst]
-      if ((r = rotate_g2(c, M, grad_out, 0, dgate, gate, ch, gate, ZERO, omega)) != SO2_OK)
-        return r;
-      if ((r = gemm_ga(c, ch + M)) != SO2_OK) return r;  // [M^T P; M^T Gv]
-      ScatterTerms t{};
-      t.F[0] = prows(c, P.Ga, 0);
-      t.ld[0] = y.KA;
-      t.A[0] = ONE;
-      t.F[1] = prows(c, P.Ga, (size_t)ch * y.KA);
-      t.ld[1] = y.KA;
-      t.B[1] = ONE;
-      if ((r = scatter(c, e0, M, t, 0, omega, d_x)) != SO2_OK) return r;
     }
   }
 
-  // ---- pass B (destination order): d_grad_out, radial gate, d_W ----
-  if (d_grad_out || d_w || d_w_rad || d_b_rad) {
+  // ---- pass B (destination order): d_grad_out, radial gate, d_W, the
+  // output side of d_edge_vec ----
+  if (d_grad_out || d_w || d_w_rad || d_b_rad || d_edge_vec) {
     if ((r = sort_edges(c, edge_index, 1)) != SO2_OK) return r;
     for (int64_t e0 = 0; e0 < E; e0 += ch) {
       const int M = static_cast<int>((E - e0) < ch ? (E - e0) : ch);
@@ -1294,6 +1325,25 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
           t.A[2] = gate;
         }
         if ((r = scatter(c, e0, M, t, 1, has_r ? omega : nullptr, d_grad_out)) != SO2_OK) return r;
+      }
+      if (d_edge_vec) {
+        ProfScope ps(5, c.s);
+        const int sm = 8 * (y.dsz + 2 * RAD_MAX_NR) * 4;
+#define SO2_HOUT_LAUNCH(TF)                                                                    \
+  DISPATCH_LM(y.L, y.mmax, constexpr int LE = (LC >= 0 && LC <= 4) ? LC : -1;                   \
+              k_edge_hess_out<MM, LE, TF><<<warp_grid(M, 8), 256, sm, c.s>>>(                   \
+                  y, desc->rbf_cutoff, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),           \
+                  at<float>(ws, P.geo), at<float>(ws, P.gate), grad_out,                       \
+                  has_r ? omega : nullptr, reinterpret_cast<const TF *>(V),                    \
+                  has_r ? reinterpret_cast<const TF *>(dV) : nullptr,                          \
+                  has_x ? reinterpret_cast<const TF *>(Vt) : nullptr, prm.w_rad, d_edge_vec);)
+        if (P.split) {
+          SO2_HOUT_LAUNCH(float)
+        } else {
+          SO2_HOUT_LAUNCH(__nv_bfloat16)
+        }
+#undef SO2_HOUT_LAUNCH
+        CKL();
       }
       if (d_w_rad || d_b_rad) {
         {

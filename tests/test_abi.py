@@ -96,16 +96,6 @@ def test_argument_errors_are_reported_before_any_launch(lib):
                                None) == 1
 
 
-def test_double_backward_rejects_second_order_edge_output(lib):
-    d = B.make_desc(2, 2, 16, 16, 8, 5.0)
-    P = ctypes.c_void_p(0x1000)
-    code = lib.so2conv_double_backward(ctypes.byref(d), 4, 3, P, P, P,
-                                       B.Params(0x1000, 0x1000, 0x1000), P, None, P,
-                                       None, None, None, None, None, P,
-                                       ctypes.c_void_p(0x100000), 1 << 40, None)
-    assert code == 2
-
-
 def test_status_strings(lib):
     for code in range(8):
         s = lib.so2conv_status_string(code)

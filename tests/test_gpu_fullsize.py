@@ -21,7 +21,8 @@ bench.py times.  The float64 oracle cannot run them whole, so:
   K-split counts depend only on the sizes), while only the sampled nodes'
   incoming edges contribute, so the oracle on those edges gives the exact
   gradients.  The force test does the same with an edge-vector cotangent that
-  is zero except on sampled edges.
+  is zero except on sampled edges (which also gives d_edge_vec of those edges
+  element by element, and zero elsewhere).
 """
 
 import numpy as np
@@ -171,13 +172,18 @@ def test_force_double_backward_full_size():
     ggm[es] = gg_r[es]
     dm = B.double_backward(desc, d["x"], d["edge_index"], d["edge_vec"], d["w"], d["w_rad"],
                            d["b_rad"], d["grad_out"], gg_edge_vec=ggm.to(DEV),
-                           need=["d_w", "d_w_rad", "d_b_rad"])
+                           need=["d_w", "d_w_rad", "d_b_rad", "d_edge_vec"])
     torch.cuda.synchronize()
     assert B.check(DEV) == 0
     mref = O.double_backward(*_oracle_args(p, es), torch.from_numpy(p.grad_out),
                              gg_edge_vec=gg_r.double()[es])
     for k in ("d_w", "d_w_rad", "d_b_rad"):
         assert rel_err(dm[k].cpu(), mref[k]) < 1e-4, k
+    # second order in the edge vectors: nonzero only on the sampled edges
+    dr = dm["d_edge_vec"].cpu()
+    assert rel_err(dr[es], mref["d_edge_vec"]) < 1e-4
+    rest = np.setdiff1d(np.arange(p.n_edges), es)
+    assert dr[rest].abs().max().item() == 0.0
     # sampled rows of d_grad_out and d_x against the oracle on the local edges
     rng = np.random.default_rng(8)
     nodes = rng.choice(p.n_nodes, 3, replace=False)

@@ -277,7 +277,7 @@ def test_double_backward_parity(name, make, which):
     gg_x = rng.standard_normal(p.x.shape) if "x" in which else None
     got = _gpu_double_backward(p, gg_x, gg_r)
     ref = oracle_double_backward(p, gg_x=gg_x, gg_edge_vec=gg_r)
-    for k in ["d_x", "d_w", "d_w_rad", "d_b_rad", "d_grad_out"]:
+    for k in ["d_x", "d_w", "d_w_rad", "d_b_rad", "d_grad_out", "d_edge_vec"]:
         err = rel_err(got[k], ref[k])
         assert err < TOL[p.x_bf16], (name, which, k, err)
 
@@ -293,7 +293,7 @@ def test_force_training_step_parity():
     got = _gpu_double_backward(p, None, gg_r)
     from helpers import oracle_double_backward
     want = oracle_double_backward(p, gg_edge_vec=gg_r)
-    for k in ["d_w", "d_w_rad", "d_b_rad", "d_x"]:
+    for k in ["d_w", "d_w_rad", "d_b_rad", "d_x", "d_edge_vec"]:
         assert rel_err(got[k], want[k]) < 1e-4, k
 
 
