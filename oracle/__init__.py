@@ -28,6 +28,10 @@ page gives no formulas, so every convention below is a stated reading:
   with width cutoff / (n_rbf - 1), applied per output channel after mixing;
 * reduction: plain sum over incoming edges.
 
+The message block (two such convolutions with an edge-frame activation
+between them, the abstract's "recombination with activation") is in
+``block.py``.
+
 Parity status: every function here is pinned by tests/test_oracle_*.py against
 closed forms, textbook tables, invariants and finite differences.
 """
@@ -44,6 +48,13 @@ from .so2conv import (  # noqa: F401
     backward,
     double_backward,
     edge_frame_rows,
+)
+from .block import (  # noqa: F401
+    BLOCK_GRADS,
+    activation,
+    block_backward,
+    block_forward,
+    mix_rows,
 )
 from .sh import real_sh, legendre  # noqa: F401
 from .wigner import frame, wigner_d, wigner_d_blocks  # noqa: F401
