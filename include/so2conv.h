@@ -154,6 +154,38 @@ so2_status so2conv_double_backward(
     float *d_x, float *d_w, float *d_w_rad, float *d_b_rad, float *d_grad_out,
     float *d_edge_vec, void *ws, size_t ws_bytes, so2_stream_t stream);
 
+/* Message block: two SO(2) convolutions with the activation between them,
+ * in the edge frame ("TrimSO(2): Fast and Memory-Efficient Training of
+ * Equivariant Interatomic Potentials", Abstract: rotation on gather,
+ * recombination with activation, inverse rotation on reduction).  Per edge:
+ *   a  = trunc(D x[s]);  h = g1 * M_W1(a);  h' = h * sigmoid(h[(0,0)])
+ *   (per channel: SiLU on the (0,0) row, the other rows gated by the same
+ *   sigmoid);  y~ = g2 * M_W2(h');  out[d] += D^T y~.
+ * p1 and p2 are the two convolutions' packed weights and radial gates, laid
+ * out as for so2conv_forward.  The block keeps one channel count: desc.c_in
+ * must equal desc.c_out (SO2_ERR_UNSUPPORTED otherwise).  The workspace comes
+ * from so2conv_block_workspace_size (which = 0 forward, 1 backward); other
+ * rules (ownership, errors, alignment, so2conv_check) as for the single
+ * convolution. */
+size_t so2conv_block_workspace_size(const so2conv_desc *desc, int64_t n_nodes,
+                                    int64_t n_edges, int which);
+so2_status so2conv_block_forward(const so2conv_desc *desc, int64_t n_nodes,
+                                 int64_t n_edges, const void *x,
+                                 const int64_t *edge_index, const float *edge_vec,
+                                 so2conv_params p1, so2conv_params p2, float *out,
+                                 void *ws, size_t ws_bytes, so2_stream_t stream);
+/* Backward of <grad_out, block output>: gradients w.r.t. x, both
+ * convolutions' weights and radial gates, and the edge vectors (the exact
+ * first derivative of the block).  Any output may be NULL (skipped); all are
+ * f32 and overwritten. */
+so2_status so2conv_block_backward(
+    const so2conv_desc *desc, int64_t n_nodes, int64_t n_edges, const void *x,
+    const int64_t *edge_index, const float *edge_vec, so2conv_params p1,
+    so2conv_params p2, const float *grad_out, float *grad_x, float *grad_w1,
+    float *grad_w_rad1, float *grad_b_rad1, float *grad_w2, float *grad_w_rad2,
+    float *grad_b_rad2, float *grad_edge_vec, void *ws, size_t ws_bytes,
+    so2_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the device error word kept in the
  * workspace, and returns it (SO2_OK if none).  Each forward / backward /
  * double backward call clears the word when it starts, so the result covers

@@ -73,6 +73,13 @@ def load():
     lib.so2conv_edge_frames.restype = ctypes.c_int
     lib.so2conv_forward_noalloc.argtypes = [pd, i64, i64, vp, vp, vp, Params, vp, vp]
     lib.so2conv_forward_noalloc.restype = ctypes.c_int
+    lib.so2conv_block_workspace_size.argtypes = [pd, i64, i64, ctypes.c_int]
+    lib.so2conv_block_workspace_size.restype = sz
+    lib.so2conv_block_forward.argtypes = [pd, i64, i64, vp, vp, vp, Params, Params, vp, vp, sz, vp]
+    lib.so2conv_block_forward.restype = ctypes.c_int
+    lib.so2conv_block_backward.argtypes = [pd, i64, i64, vp, vp, vp, Params, Params, vp,
+                                           vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.so2conv_block_backward.restype = ctypes.c_int
     lib.so2conv_noalloc_check.argtypes = [vp]
     lib.so2conv_noalloc_check.restype = ctypes.c_int
     lib.so2conv_launch_count.argtypes = []
@@ -338,3 +345,70 @@ def noalloc_check(device):
     """Synchronise and return the device status of the last no-alloc forward
     in the current context (0 = ok)."""
     return int(load().so2conv_noalloc_check(_stream(device)))
+
+
+# ---------------------------------------------------------------------------
+# Message block: two convolutions with the edge-frame activation between them
+# ---------------------------------------------------------------------------
+BLOCK_GRADS = ["grad_x", "grad_w1", "grad_w_rad1", "grad_b_rad1", "grad_w2", "grad_w_rad2",
+               "grad_b_rad2", "grad_edge_vec"]
+
+
+def block_workspace_size(desc, n_nodes, n_edges, which):
+    return int(load().so2conv_block_workspace_size(ctypes.byref(desc), n_nodes, n_edges, which))
+
+
+def _block_ws(desc, n_nodes, n_edges, which, device, ws):
+    need = block_workspace_size(desc, n_nodes, n_edges, which)
+    if need == 0:
+        raise So2Error(2, "block_workspace_size")
+    return (ws or workspace(device)).get(need)
+
+
+def _params(w, w_rad, b_rad):
+    return Params(_ptr(w).value, _ptr(w_rad).value, _ptr(b_rad).value)
+
+
+def block_forward(desc, x, edge_index, edge_vec, w1, w_rad1, b_rad1, w2, w_rad2, b_rad2,
+                  out=None, ws=None):
+    """so2conv_block_forward: out [N, S, C] of the two-convolution block."""
+    lib = load()
+    x, edge_index, edge_vec, w1, w_rad1, b_rad1, w2, w_rad2, b_rad2 = map(
+        _c, (x, edge_index, edge_vec, w1, w_rad1, b_rad1, w2, w_rad2, b_rad2))
+    N, E = x.shape[0], edge_index.shape[1]
+    if out is None:
+        out = torch.empty((N, (desc.lmax + 1) ** 2, desc.c_out), dtype=torch.float32,
+                          device=x.device)
+    p, nb = _block_ws(desc, N, E, 0, x.device, ws)
+    code = lib.so2conv_block_forward(ctypes.byref(desc), N, E, _ptr(x), _ptr(edge_index),
+                                     _ptr(edge_vec), _params(w1, w_rad1, b_rad1),
+                                     _params(w2, w_rad2, b_rad2), _ptr(out), p, nb,
+                                     _stream(x.device))
+    _check_call(code, "so2conv_block_forward")
+    return out
+
+
+def block_backward(desc, x, edge_index, edge_vec, w1, w_rad1, b_rad1, w2, w_rad2, b_rad2,
+                   grad_out, need=None, ws=None, out=None):
+    """so2conv_block_backward: a dict keyed by BLOCK_GRADS (those in `need`)."""
+    lib = load()
+    x, edge_index, edge_vec, w1, w_rad1, b_rad1, w2, w_rad2, b_rad2, grad_out = map(
+        _c, (x, edge_index, edge_vec, w1, w_rad1, b_rad1, w2, w_rad2, b_rad2, grad_out))
+    N, E = x.shape[0], edge_index.shape[1]
+    need = set(BLOCK_GRADS if need is None else need)
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    S = (desc.lmax + 1) ** 2
+    nw = num_weights(desc)
+    shapes = {"grad_x": (N, S, desc.c_in), "grad_w1": (nw,), "grad_w2": (nw,),
+              "grad_w_rad1": (desc.n_rbf, desc.c_out), "grad_w_rad2": (desc.n_rbf, desc.c_out),
+              "grad_b_rad1": (desc.c_out,), "grad_b_rad2": (desc.c_out,),
+              "grad_edge_vec": (E, 3)}
+    outs = _outputs(BLOCK_GRADS, need, shapes, out, f32)
+    p, nb = _block_ws(desc, N, E, 1, dev, ws)
+    code = lib.so2conv_block_backward(ctypes.byref(desc), N, E, _ptr(x), _ptr(edge_index),
+                                      _ptr(edge_vec), _params(w1, w_rad1, b_rad1),
+                                      _params(w2, w_rad2, b_rad2), _ptr(grad_out),
+                                      *[_ptr(outs[n]) for n in BLOCK_GRADS], p, nb, _stream(dev))
+    _check_call(code, "so2conv_block_backward")
+    return {n: t for n, t in outs.items() if t is not None}

@@ -1777,6 +1777,144 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
   }
 }
 
+// ---------------------------------------------------------------------------
+// Message block: the activation between the two SO(2) convolutions
+// ("TrimSO(2): Fast and Memory-Efficient Training of Equivariant Interatomic
+// Potentials", Abstract: recombination with activation).  In the edge frame,
+// per channel c, with h = g1 * V1 (the first conv's gated product rows):
+//   h'[row][c] = h[row][c] * s_c,  s_c = sigmoid(h[(0,0)][c])
+// (SiLU on the (0,0) row; s_c does not change under a roll of the frame).
+// The rows of both convs are the kept edge-frame rows in the grouped layout
+// (the block keeps one channel count, so input and output layouts agree).
+// One warp per edge, four channels per lane.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float4 sigmoid4(float4 h) {
+  return make_float4(1.f / (1.f + __expf(-h.x)), 1.f / (1.f + __expf(-h.y)),
+                     1.f / (1.f + __expf(-h.z)), 1.f / (1.f + __expf(-h.w)));
+}
+
+// Forward: h' as the second product's operand planes (bf16 hi, and lo on the
+// split path), zero on the padding columns.
+template <typename TF>
+__global__ void __launch_bounds__(256) k_block_act(Layout y, int M, const TF *__restrict__ V1,
+                                                   const float *__restrict__ gate1,
+                                                   __nv_bfloat16 *__restrict__ hp_hi,
+                                                   __nv_bfloat16 *__restrict__ hp_lo) {
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  const int C = y.co;
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
+    const TF *v = V1 + (int64_t)i * y.KG;
+    __nv_bfloat16 *oh = hp_hi + (int64_t)i * y.KA;
+    __nv_bfloat16 *ol = hp_lo ? hp_lo + (int64_t)i * y.KA : nullptr;
+    for (int c = 4 * lane; c < C; c += 128) {
+      const float4 g = load4(gate1 + (int64_t)i * C + c);
+      const float4 v00 = load4(v + y.kout_off[0] + c);  // row (0, 0)
+      const float4 sg = sigmoid4(make_float4(g.x * v00.x, g.y * v00.y, g.z * v00.z, g.w * v00.w));
+      const float4 k = make_float4(g.x * sg.x, g.y * sg.y, g.z * sg.z, g.w * sg.w);
+      for (int gi = 0; gi < y.ng; ++gi)
+        for (int j = 0; j < y.rows[gi]; ++j) {
+          const int col = y.kout_off[gi] + j * C + c;
+          const float4 vr = load4(v + col);
+          store_split4(oh + col, ol ? ol + col : nullptr,
+                       make_float4(k.x * vr.x, k.y * vr.y, k.z * vr.z, k.w * vr.w));
+        }
+    }
+    for (int gi = 0; gi < y.ng; ++gi)
+      for (int kk = y.rows[gi] * C + 4 * lane; kk < y.Kin_pad[gi]; kk += 128)
+        store_split4(oh + y.kin_off[gi] + kk, ol ? ol + y.kin_off[gi] + kk : nullptr,
+                     make_float4(0.f, 0.f, 0.f, 0.f));
+  }
+}
+
+// Backward through the activation.  With Gh = dL/dh' (= M2^T (g2 D G[dst]),
+// the second conv's transposed product rows):
+//   dh[row] = s Gh[row] + [row == (0,0)] s (1 - s) sum_rows h Gh,
+// and through h = g1 V1: the first conv's output-side operand gv1 = g1 dh
+// (planes, zero padding), Gg1[c] = sum_rows dh V1 (its gate's gradient), and
+// the gate's share of dL/d|r|, dd1 = sum_c Gg1[c] sum_k W_rad1[k][c] phi'_k(d),
+// added onto the edge record h_rec[i].z.
+template <typename TF>
+__global__ void __launch_bounds__(256) k_block_act_bwd(
+    Layout y, float cutoff, int M, const float *__restrict__ geo, const TF *__restrict__ V1,
+    const float *__restrict__ gate1, const TF *__restrict__ Gh, const float *__restrict__ w_rad1,
+    __nv_bfloat16 *__restrict__ gv_hi, __nv_bfloat16 *__restrict__ gv_lo,
+    float *__restrict__ Gg1, float4 *__restrict__ h_rec) {
+  __shared__ float sphi[8][RAD_MAX_NR];
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  float *sP = sphi[threadIdx.x >> 5];
+  const int C = y.co;
+  const float sig = cutoff / static_cast<float>(y.nr - 1);
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < M; i += gridDim.x * wpb) {
+    const float d = geo[(int64_t)i * GEO];
+    __syncwarp();
+    for (int k = lane; k < y.nr; k += 32) {
+      const float t = (d - sig * static_cast<float>(k)) / sig;
+      sP[k] = (-t / sig) * __expf(-0.5f * t * t);
+    }
+    __syncwarp();
+    const TF *v = V1 + (int64_t)i * y.KG;
+    const TF *gh = Gh + (int64_t)i * y.KA;
+    __nv_bfloat16 *oh = gv_hi + (int64_t)i * y.KG;
+    __nv_bfloat16 *ol = gv_lo ? gv_lo + (int64_t)i * y.KG : nullptr;
+    float dd = 0.f;
+    for (int c = 4 * lane; c < C; c += 128) {
+      const float4 g = load4(gate1 + (int64_t)i * C + c);
+      const float4 v00 = load4(v + y.kout_off[0] + c);
+      const float4 sg = sigmoid4(make_float4(g.x * v00.x, g.y * v00.y, g.z * v00.z, g.w * v00.w));
+      // sum over rows of h Gh
+      float4 hg = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int gi = 0; gi < y.ng; ++gi)
+        for (int j = 0; j < y.rows[gi]; ++j) {
+          const float4 vr = load4(v + y.kout_off[gi] + j * C + c);
+          const float4 gr = load4(gh + y.kin_off[gi] + j * C + c);
+          hg.x += g.x * vr.x * gr.x;
+          hg.y += g.y * vr.y * gr.y;
+          hg.z += g.z * vr.z * gr.z;
+          hg.w += g.w * vr.w * gr.w;
+        }
+      const float4 e00 = make_float4(sg.x * (1.f - sg.x) * hg.x, sg.y * (1.f - sg.y) * hg.y,
+                                     sg.z * (1.f - sg.z) * hg.z, sg.w * (1.f - sg.w) * hg.w);
+      float4 gg = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int gi = 0; gi < y.ng; ++gi)
+        for (int j = 0; j < y.rows[gi]; ++j) {
+          const float4 vr = load4(v + y.kout_off[gi] + j * C + c);
+          const float4 gr = load4(gh + y.kin_off[gi] + j * C + c);
+          float4 dh = make_float4(sg.x * gr.x, sg.y * gr.y, sg.z * gr.z, sg.w * gr.w);
+          if (gi == 0 && j == 0) {
+            dh.x += e00.x;
+            dh.y += e00.y;
+            dh.z += e00.z;
+            dh.w += e00.w;
+          }
+          const int col = y.kout_off[gi] + j * C + c;
+          store_split4(oh + col, ol ? ol + col : nullptr,
+                       make_float4(g.x * dh.x, g.y * dh.y, g.z * dh.z, g.w * dh.w));
+          gg.x += dh.x * vr.x;
+          gg.y += dh.y * vr.y;
+          gg.z += dh.z * vr.z;
+          gg.w += dh.w * vr.w;
+        }
+      *reinterpret_cast<float4 *>(Gg1 + (int64_t)i * C + c) = gg;
+      float4 dg = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = 0; k < y.nr; ++k) {
+        const float4 wk = __ldg(reinterpret_cast<const float4 *>(w_rad1 + (int64_t)k * C + c));
+        const float p = sP[k];
+        dg.x += wk.x * p;
+        dg.y += wk.y * p;
+        dg.z += wk.z * p;
+        dg.w += wk.w * p;
+      }
+      dd += gg.x * dg.x + gg.y * dg.y + gg.z * dg.z + gg.w * dg.w;
+    }
+    for (int gi = 0; gi < y.ng; ++gi)
+      for (int kk = y.rows[gi] * C + 4 * lane; kk < y.Kout_pad[gi]; kk += 128)
+        store_split4(oh + y.kout_off[gi] + kk, ol ? ol + y.kout_off[gi] + kk : nullptr,
+                     make_float4(0.f, 0.f, 0.f, 0.f));
+    for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
+    if (lane == 0) h_rec[i].z += dd;
+  }
+}
+
 // Frames and full Wigner-D for inspection, with the same per-thread code the
 // op uses.  Block = one warp, 32 edges.
 template <int L>

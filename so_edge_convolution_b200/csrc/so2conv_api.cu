@@ -965,6 +965,120 @@ so2_status edge_terms(Ctx &c, int M, int part, const void *x, const float *grad_
   return SO2_OK;
 }
 
+// --------------------------------------------------------------------------
+// Message block (two SO(2) convolutions with the activation between them).
+// Two contexts share one workspace: the per-edge records, frames, Wigner-D,
+// sort, edge-gradient record and output-side operand planes are common; each
+// conv has its own gate, packed weights, operand planes (conv 2's are the
+// activation h'), product rows and weight-gradient accumulator.
+// --------------------------------------------------------------------------
+struct BlockPlan {
+  Plan p1, p2;
+  size_t total = 0;
+};
+
+BlockPlan make_block_plan(const so2conv_desc *d, int64_t N, int64_t E, int which) {
+  BlockPlan b;
+  b.p1 = make_plan(d, N, E, which ? SO2_WS_BACKWARD : SO2_WS_FORWARD);
+  const Plan &p = b.p1;
+  const Layout &y = p.y;
+  size_t c = p.total;
+  Plan q = p;
+  const size_t lo = p.split ? 1 : 0, pe = p.split ? 4 : 2;
+  q.gate = take(c, 4ull * y.co * p.chunk);
+  q.wst_hi = take(c, 2ull * y.WR * y.WK);
+  q.wst_lo = take(c, 2ull * y.WR * y.WK * lo);
+  q.a_hi = take(c, 2ull * p.chunk * y.KA);
+  q.a_lo = take(c, 2ull * p.chunk * y.KA * lo);
+  if (which) {
+    q.wtr_hi = take(c, 2ull * y.WTR * y.WTK);
+    q.wtr_lo = take(c, 2ull * y.WTR * y.WTK * lo);
+    q.V = take(c, pe * p.chunk * y.KG);
+    q.Gg = take(c, 4ull * p.chunk * y.co);
+    q.dws = take(c, 4ull * y.WR * y.WK);
+  }
+  b.p2 = q;
+  b.total = (c + 1023) & ~static_cast<size_t>(1023);
+  b.p1.total = b.p2.total = b.total;
+  return b;
+}
+
+// The gate of a second conv for the chunk's edges (frames from chunk_prep).
+so2_status gate_only(Ctx &c, int M, so2conv_params prm) {
+  ProfScope ps(4, c.s);
+  k_edge_gate<<<(M + GATE_EDGES - 1) / GATE_EDGES, 128, GATE_EDGES * c.P.y.nr * sizeof(float),
+                c.s>>>(c.P.y, c.d->rbf_cutoff, M, at<float>(c.ws, c.P.geo), prm.w_rad, prm.b_rad,
+                       at<float>(c.ws, c.P.gate));
+  CKL();
+  return SO2_OK;
+}
+
+so2_status block_setup(const so2conv_desc *d, int64_t N, int64_t E, const void *x,
+                       const int64_t *ei, const float *ev, so2conv_params p1,
+                       so2conv_params p2, void *ws, size_t ws_bytes, int which,
+                       so2_stream_t stream, Ctx &c1, Ctx &c2) {
+  if (!d) return SO2_ERR_INVALID_ARG;
+  if (!desc_ok(d) || d->c_in != d->c_out) return SO2_ERR_UNSUPPORTED;
+  if (!p2.w || !p2.w_rad || !p2.b_rad) return SO2_ERR_INVALID_ARG;
+  Plan P;
+  // argument checks of the single conv (the block's workspace is larger)
+  so2_status r = common_checks(d, N, E, x, ei, ev, p1, ws, (size_t)-1,
+                               which ? SO2_WS_BACKWARD : SO2_WS_FORWARD, P);
+  if (r != SO2_OK) return r;
+  const BlockPlan bp = make_block_plan(d, N, E, which);
+  if (ws_bytes < bp.total) return SO2_ERR_WORKSPACE;
+  for (Ctx *c : {&c1, &c2}) {
+    c->d = d;
+    c->ws = ws;
+    c->s = reinterpret_cast<cudaStream_t>(stream);
+    c->st = at<DevStatus>(ws, bp.p1.status);
+  }
+  c1.P = bp.p1;
+  c2.P = bp.p2;
+  CK(cudaMemsetAsync(c1.st, 0, sizeof(DevStatus), c1.s));
+  return SO2_OK;
+}
+
+// h' = act(g1 * V1) as conv 2's operand planes.
+so2_status block_act(Ctx &c1, Ctx &c2, int M) {
+  const Plan &P = c1.P;
+  ProfScope ps(5, c1.s);
+  __nv_bfloat16 *hh = at<__nv_bfloat16>(c2.ws, c2.P.a_hi);
+  __nv_bfloat16 *hl = P.split ? at<__nv_bfloat16>(c2.ws, c2.P.a_lo) : nullptr;
+  if (P.split)
+    k_block_act<float><<<warp_grid(M, 8), 256, 0, c1.s>>>(
+        P.y, M, reinterpret_cast<const float *>(prows(c1, P.V, 0)), at<float>(c1.ws, P.gate), hh, hl);
+  else
+    k_block_act<__nv_bfloat16><<<warp_grid(M, 8), 256, 0, c1.s>>>(
+        P.y, M, reinterpret_cast<const __nv_bfloat16 *>(prows(c1, P.V, 0)),
+        at<float>(c1.ws, P.gate), hh, hl);
+  CKL();
+  return SO2_OK;
+}
+
+// Backward through the activation: conv 1's output-side planes, Gg1 and the
+// gate's share of the edge gradient (k_block_act_bwd).
+so2_status block_act_bwd(Ctx &c1, Ctx &c2, int M, const float *w_rad1) {
+  const Plan &P = c1.P;
+  ProfScope ps(5, c1.s);
+  __nv_bfloat16 *gh = at<__nv_bfloat16>(c1.ws, P.gv_hi);
+  __nv_bfloat16 *gl = P.split ? at<__nv_bfloat16>(c1.ws, P.gv_lo) : nullptr;
+#define SO2_ABW(TF)                                                                            \
+  k_block_act_bwd<TF><<<warp_grid(M, 8), 256, 0, c1.s>>>(                                      \
+      P.y, c1.d->rbf_cutoff, M, at<float>(c1.ws, P.geo),                                       \
+      reinterpret_cast<const TF *>(prows(c1, P.V, 0)), at<float>(c1.ws, P.gate),                \
+      reinterpret_cast<const TF *>(prows(c2, c2.P.Ga, 0)), w_rad1, gh, gl, at<float>(c1.ws, P.Gg), \
+      at<float4>(c1.ws, P.h))
+  if (P.split) {
+    SO2_ABW(float);
+  } else {
+    SO2_ABW(__nv_bfloat16);
+  }
+#undef SO2_ABW
+  CKL();
+  return SO2_OK;
+}
+
 // One thread waits, with the library's bounded wait, on an mbarrier phase
 // that nothing completes; the wait gives up after limit_ns and records
 // SO2_ERR_TIMEOUT (the path every tensor-core wait takes when a partner
@@ -1417,6 +1531,142 @@ so2_status so2conv_noalloc_check(so2_stream_t stream) {
   void *base = noalloc_base();
   if (!base) return SO2_ERR_CUDA;
   return so2conv_check(base, stream);
+}
+
+size_t so2conv_block_workspace_size(const so2conv_desc *desc, int64_t n_nodes, int64_t n_edges,
+                                    int which) {
+  if (!desc_ok(desc) || desc->c_in != desc->c_out || n_nodes < 0 || n_edges < 0) return 0;
+  if (which != 0 && which != 1) return 0;
+  return make_block_plan(desc, n_nodes, n_edges, which).total;
+}
+
+so2_status so2conv_block_forward(const so2conv_desc *desc, int64_t N, int64_t E, const void *x,
+                                 const int64_t *edge_index, const float *edge_vec,
+                                 so2conv_params p1, so2conv_params p2, float *out, void *ws,
+                                 size_t ws_bytes, so2_stream_t stream) {
+  Ctx c1, c2;
+  so2_status r = block_setup(desc, N, E, x, edge_index, edge_vec, p1, p2, ws, ws_bytes, 0,
+                             stream, c1, c2);
+  if (r != SO2_OK) return r;
+  if (N > 0 && !out) return SO2_ERR_INVALID_ARG;
+  const Plan &P = c1.P;
+  const Layout &y = P.y;
+  if (N > 0) CK(cudaMemsetAsync(out, 0, sizeof(float) * N * y.S * y.co, c1.s));
+  if (E == 0) return SO2_OK;
+  if ((r = build_maps(c1, false)) != SO2_OK) return r;
+  if ((r = build_maps(c2, false)) != SO2_OK) return r;
+  if ((r = sort_edges(c1, edge_index, 1)) != SO2_OK) return r;
+  if ((r = pack_weights(c1, p1.w, false)) != SO2_OK) return r;
+  if ((r = pack_weights(c2, p2.w, false)) != SO2_OK) return r;
+  for (int64_t e0 = 0; e0 < E; e0 += P.chunk) {
+    const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
+    if ((r = chunk_prep(c1, e0, M, edge_index, edge_vec, 1, p1)) != SO2_OK) return r;
+    if ((r = gate_only(c2, M, p2)) != SO2_OK) return r;
+    if ((r = rotate_x(c1, M, x, P.xbf16)) != SO2_OK) return r;
+    if ((r = gemm_v(c1, M)) != SO2_OK) return r;  // V1
+    if ((r = block_act(c1, c2, M)) != SO2_OK) return r;
+    if (fusable(y.co, P.split)) {
+      const GemmScatter sc = make_scatter(c2, at<float>(ws, c2.P.gate), out, y.co);
+      if ((r = gemm_v(c2, M, &sc, false)) != SO2_OK) return r;
+    } else {
+      if ((r = gemm_v(c2, M)) != SO2_OK) return r;
+      if ((r = reduce_nodes(c2, e0, M, prows(c2, c2.P.V, 0), y.KG, at<float>(ws, c2.P.gate), 1,
+                            out)) != SO2_OK)
+        return r;
+    }
+  }
+  return SO2_OK;
+}
+
+so2_status so2conv_block_backward(const so2conv_desc *desc, int64_t N, int64_t E, const void *x,
+                                  const int64_t *edge_index, const float *edge_vec,
+                                  so2conv_params p1, so2conv_params p2, const float *grad_out,
+                                  float *grad_x, float *grad_w1, float *grad_w_rad1,
+                                  float *grad_b_rad1, float *grad_w2, float *grad_w_rad2,
+                                  float *grad_b_rad2, float *grad_edge_vec, void *ws,
+                                  size_t ws_bytes, so2_stream_t stream) {
+  Ctx c1, c2;
+  so2_status r = block_setup(desc, N, E, x, edge_index, edge_vec, p1, p2, ws, ws_bytes, 1,
+                             stream, c1, c2);
+  if (r != SO2_OK) return r;
+  if ((N > 0 && !grad_out) || !aligned16(grad_out)) return SO2_ERR_INVALID_ARG;
+  const Plan &P = c1.P;
+  const Layout &y = P.y;
+  cudaStream_t s = c1.s;
+  const int64_t nw = num_weights(y);
+  if (grad_x && N > 0) CK(cudaMemsetAsync(grad_x, 0, sizeof(float) * N * y.S * y.ci, s));
+  for (float *g : {grad_w1, grad_w2})
+    if (g) CK(cudaMemsetAsync(g, 0, sizeof(float) * nw, s));
+  for (float *g : {grad_w_rad1, grad_w_rad2})
+    if (g) CK(cudaMemsetAsync(g, 0, sizeof(float) * y.nr * y.co, s));
+  for (float *g : {grad_b_rad1, grad_b_rad2})
+    if (g) CK(cudaMemsetAsync(g, 0, sizeof(float) * y.co, s));
+  if (E == 0) return SO2_OK;
+  if ((r = build_maps(c1, true)) != SO2_OK) return r;
+  if ((r = build_maps(c2, true)) != SO2_OK) return r;
+  if ((r = sort_edges(c1, edge_index, 0)) != SO2_OK) return r;
+  if ((r = pack_weights(c1, p1.w, true)) != SO2_OK) return r;
+  if ((r = pack_weights(c2, p2.w, true)) != SO2_OK) return r;
+  if (grad_w1) CK(cudaMemsetAsync(at<float>(ws, c1.P.dws), 0, 4ull * y.WR * y.WK, s));
+  if (grad_w2) CK(cudaMemsetAsync(at<float>(ws, c2.P.dws), 0, 4ull * y.WR * y.WK, s));
+  const bool need_ga1 = grad_x || grad_edge_vec;
+  const bool fuse_gx = grad_x && fusable(y.ci, P.split);
+  for (int64_t e0 = 0; e0 < E; e0 += P.chunk) {
+    const int M = static_cast<int>((E - e0) < P.chunk ? (E - e0) : P.chunk);
+    if ((r = chunk_prep(c1, e0, M, edge_index, edge_vec, 0, p1)) != SO2_OK) return r;
+    if ((r = gate_only(c2, M, p2)) != SO2_OK) return r;
+    if ((r = rotate_x(c1, M, x, P.xbf16)) != SO2_OK) return r;
+    if ((r = gemm_v(c1, M)) != SO2_OK) return r;  // V1
+    if ((r = block_act(c1, c2, M)) != SO2_OK) return r;
+    if ((r = gemm_v(c2, M)) != SO2_OK) return r;  // V2
+    // conv 2's output side: Gg2, the edge record (frame terms of the output
+    // rotation and the gate-2 part), gv2 = g2 * (D G[dst]) planes
+    if ((r = edge_terms(c2, M, 1, x, grad_out, true, p2.w_rad)) != SO2_OK) return r;
+    if ((r = gemm_ga(c2, M)) != SO2_OK) return r;  // dL/dh' = M2^T gv2
+    if (grad_w2) {
+      if ((r = zero_tail(c2, M, false, 0)) != SO2_OK) return r;
+      if ((r = zero_tail(c2, M, true, 0)) != SO2_OK) return r;
+      if ((r = gemm_dw(c2, M, 0, 0)) != SO2_OK) return r;  // gv2 (x) h'
+    }
+    if ((r = block_act_bwd(c1, c2, M, p1.w_rad)) != SO2_OK) return r;  // gv1, Gg1, dd1
+    if (need_ga1) {
+      const GemmScatter sc = make_scatter(c1, nullptr, grad_x, y.ci);
+      if ((r = gemm_ga(c1, M, fuse_gx ? &sc : nullptr, grad_edge_vec != nullptr || !fuse_gx)) !=
+          SO2_OK)
+        return r;
+    }
+    if (grad_w1) {
+      if ((r = zero_tail(c1, M, false, 0)) != SO2_OK) return r;
+      if ((r = zero_tail(c1, M, true, 0)) != SO2_OK) return r;
+      if ((r = gemm_dw(c1, M, 0, 0)) != SO2_OK) return r;  // gv1 (x) a
+    }
+    if (grad_x && !fuse_gx &&
+        (r = reduce_nodes(c1, e0, M, prows(c1, P.Ga, 0), y.KA, nullptr, 0, grad_x)) != SO2_OK)
+      return r;
+    if (grad_edge_vec &&
+        (r = edge_terms(c1, M, 2, x, grad_out, false, p1.w_rad, grad_edge_vec)) != SO2_OK)
+      return r;
+    if ((grad_w_rad2 || grad_b_rad2) &&
+        (r = rad_grads(c2, M, at<float>(ws, c2.P.Gg), nullptr, nullptr, grad_w_rad2,
+                       grad_b_rad2)) != SO2_OK)
+      return r;
+    if ((grad_w_rad1 || grad_b_rad1) &&
+        (r = rad_grads(c1, M, at<float>(ws, c1.P.Gg), nullptr, nullptr, grad_w_rad1,
+                       grad_b_rad1)) != SO2_OK)
+      return r;
+  }
+  ProfScope ps(7, s);
+  if (grad_w1) {
+    k_unstack_grad<<<dim3(64, y.ng), 256, 0, s>>>(y, block_offsets(y), at<float>(ws, c1.P.dws),
+                                                   grad_w1);
+    CKL();
+  }
+  if (grad_w2) {
+    k_unstack_grad<<<dim3(64, y.ng), 256, 0, s>>>(y, block_offsets(y), at<float>(ws, c2.P.dws),
+                                                   grad_w2);
+    CKL();
+  }
+  return SO2_OK;
 }
 
 so2_status so2conv_check(void *ws, so2_stream_t stream) {
