@@ -57,6 +57,9 @@ CONFIGS = {
             "C=128, bf16 features and weights, f32 accumulation, forward+backward", 3, 4),
     "large": ("large", "Large periodic: N=20000 atoms, 50 nearest within 6 A (E=1000000), "
               "lmax=4, mmax=2, C=128, bf16 features, f32 accumulation, forward+backward", 3, 4),
+    "block": ("esen", "message block on the eSEN-like graph: two SO(2) convolutions with the "
+              "edge-frame activation between them (E=60000, lmax=4, mmax=2, C=128, f32), "
+              "forward+backward", 6, 8),
 }
 WORKLOAD = CONFIGS["esen"][1]
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
@@ -118,6 +121,9 @@ def compulsory_bytes(config, p, n_nodes, n_edges):
     fwd = shared + node_out
     if config == "md":
         return fwd + shared + G + ev
+    if config == "block":  # a second weight set and gate, read and differentiated
+        extra = nw * we + rad
+        return fwd + extra + shared + extra + G + node_in + 2 * (nw * 4 + rad) + ev
     bwd = shared + G + node_in + nw * 4 + rad + ev
     if config == "force":
         bwd_r = shared + G + ev
@@ -340,7 +346,7 @@ def run_ours(args, world, rank, local):
     split = args.split if args.split != "auto" else ("dst" if world > 1 else "replicas")
     if split == "dst" and world == 1:
         split = "replicas"  # one rank owns the whole graph
-    if split == "dst" and args.config in ("force", "md"):
+    if split == "dst" and args.config in ("force", "md", "block"):
         raise SystemExit("--split dst runs the forward + backward workloads")
     p = dst_problem(prob, world) if split == "dst" else synth.make_problem(prob, seed=rank)
     E = p.n_edges  # edges this rank's library calls process (set below for dst)
@@ -349,6 +355,11 @@ def run_ours(args, world, rank, local):
     wdt = torch.bfloat16 if bf16 else torch.float32
     desc = B.make_desc(p.lmax, p.mmax, p.c_in, p.c_out, p.n_rbf, p.rbf_cutoff,
                        B.SO2_BF16 if bf16 else B.SO2_F32)
+    if args.config == "block":  # the second convolution's weights and gate
+        rng2 = np.random.default_rng(1000 + rank)
+        w2 = rng2.standard_normal(p.w.shape) * p.w.std()
+        w_rad2 = rng2.standard_normal(p.w_rad.shape) / np.sqrt(p.n_rbf)
+        b_rad2 = rng2.standard_normal(p.b_rad.shape) / np.sqrt(p.n_rbf)
     host = {
         "x": torch.from_numpy(p.x).to(xdt).pin_memory(),
         "edge_index": torch.from_numpy(p.edge_index).pin_memory(),
@@ -359,6 +370,10 @@ def run_ours(args, world, rank, local):
         "grad_out": torch.from_numpy(p.grad_out.astype(np.float32)).pin_memory(),
         "f_ref": torch.from_numpy(p.f_ref.astype(np.float32)).pin_memory(),
     }
+    if args.config == "block":
+        host.update(w2=torch.from_numpy(w2).to(wdt).pin_memory(),
+                    w_rad2=torch.from_numpy(w_rad2.astype(np.float32)).pin_memory(),
+                    b_rad2=torch.from_numpy(b_rad2.astype(np.float32)).pin_memory())
     sg = None
     if split == "dst":
         from so_edge_convolution_b200 import sharded as S
@@ -413,7 +428,15 @@ def run_ours(args, world, rank, local):
         F.index_add_(0, src, -gr).index_add_(0, dst, gr)
         return out, {"grad_edge_vec": gr, "forces": F}
 
-    step = {"force": step_force, "md": step_md}.get(args.config, step_fwd_bwd)
+    def step_block(t, o=None):
+        a = (t["x"], t["edge_index"], t["edge_vec"], t["w"], t["w_rad"], t["b_rad"], t["w2"],
+             t["w_rad2"], t["b_rad2"])
+        out = B.block_forward(desc, *a, ws=ws, out=o["out"] if o else None)
+        g = B.block_backward(desc, *a, t["grad_out"], ws=ws, out=o["g"] if o else None)
+        return out, g
+
+    step = {"force": step_force, "md": step_md, "block": step_block}.get(args.config,
+                                                                       step_fwd_bwd)
     if split == "dst":
         step = make_dst_step(sg, desc)
         ws = None  # the sharded calls use the binding's own per-device workspace
