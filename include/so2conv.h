@@ -135,7 +135,8 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t n_nodes,
 /* Double backward: derivatives of
  *   Q = <gg_x, grad_x> + <gg_edge_vec, grad_edge_vec>
  * (grad_* from so2conv_backward with the same inputs) w.r.t. x, w, w_rad,
- * b_rad and grad_out.  gg_x / gg_edge_vec may be NULL (treated as zero).
+ * b_rad, grad_out and the edge vectors.  gg_x / gg_edge_vec may be NULL
+ * (treated as zero).
  * Defined as the exact second derivative that force training takes
  * ("TrimSO(2): ...", Abstract: higher-order differentiation;
  * "Breaking the Training Barrier of Billion-Parameter Universal Machine
