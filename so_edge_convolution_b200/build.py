@@ -16,14 +16,16 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libso2conv.so")
-SOURCES = ["so2conv_api.cu"]
+# translation units, compiled in parallel and linked into one shared object
+SOURCES = ["so2conv_api.cu", "so2conv_dbl_terms.cu"]
+OBJDIR = os.path.join(HERE, "_build")
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
-    "-Xcompiler", "-fPIC", "-shared",
+    "-Xcompiler", "-fPIC",
     "--expt-relaxed-constexpr",
-    "-cudart", "static",
 ]
+LINK_FLAGS = ["-shared", "-cudart", "static"]
 
 
 def _nvcc():
@@ -48,16 +50,34 @@ def up_to_date():
 def build(force=False, verbose=False, extra=()):
     if not force and up_to_date():
         return LIB
-    cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"),
-           *[os.path.join(CSRC, s) for s in SOURCES], "-o", LIB]
+    os.makedirs(OBJDIR, exist_ok=True)
+    objs, procs = [], []
+    for src in SOURCES:
+        obj = os.path.join(OBJDIR, os.path.splitext(src)[0] + ".o")
+        cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-c",
+               os.path.join(CSRC, src), "-o", obj]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        objs.append(obj)
+        procs.append(subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT,
+                                      text=True))
+    failed = False
+    for src, pr in zip(SOURCES, procs):
+        out = pr.communicate()[0]
+        if pr.returncode != 0:
+            failed = True
+            sys.stderr.write(f"--- {src}\n" + out)
+        elif verbose and out:
+            sys.stderr.write(out)
+    if failed:
+        raise RuntimeError("nvcc failed building libso2conv.so")
+    cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", *LINK_FLAGS, *objs, "-o", LIB]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libso2conv.so")
-    if verbose and (res.stdout or res.stderr):
-        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed linking libso2conv.so")
     return LIB
 
 

@@ -90,13 +90,16 @@ __device__ __forceinline__ void each_level(int L, F &&f) {
 }
 static_assert(LMAX_SUPPORTED == 6, "each_level instantiates degrees 0..6");
 
+// The library is built from more than one translation unit that include this
+// header: its kernels that are not templates have internal linkage (static).
+
 // ---------------------------------------------------------------------------
 // Graph preparation: stable counting sort of edges by one endpoint.
 // ---------------------------------------------------------------------------
 
 // counts[key]++ for every edge; keys outside [0, N) raise SO2_ERR_INDEX and
 // are counted as node 0 so that every later access stays in bounds.
-__global__ void k_count_keys(const int64_t *__restrict__ keys, int64_t E, int64_t N,
+static __global__ void k_count_keys(const int64_t *__restrict__ keys, int64_t E, int64_t N,
                              int *__restrict__ counts, DevStatus *st) {
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < E;
        e += (int64_t)gridDim.x * blockDim.x) {
@@ -110,7 +113,7 @@ __global__ void k_count_keys(const int64_t *__restrict__ keys, int64_t E, int64_
 }
 
 // Exclusive scan of counts[0..N) into offsets[0..N] with one block.
-__global__ void k_scan_offsets(const int *__restrict__ counts, int64_t N, int *__restrict__ offsets) {
+static __global__ void k_scan_offsets(const int *__restrict__ counts, int64_t N, int *__restrict__ offsets) {
   __shared__ int partial[1024];
   const int t = threadIdx.x;
   const int64_t per = (N + blockDim.x - 1) / blockDim.x;
@@ -133,7 +136,7 @@ __global__ void k_scan_offsets(const int *__restrict__ counts, int64_t N, int *_
   if (t == blockDim.x - 1) offsets[N] = partial[t];
 }
 
-__global__ void k_place(const int64_t *__restrict__ keys, int64_t E, int64_t N,
+static __global__ void k_place(const int64_t *__restrict__ keys, int64_t E, int64_t N,
                         const int *__restrict__ offsets, int *__restrict__ cursor,
                         int *__restrict__ perm) {
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < E;
@@ -150,7 +153,7 @@ __global__ void k_place(const int64_t *__restrict__ keys, int64_t E, int64_t N,
 // 128 edges are placed by rank (each lane holds up to four ids and counts,
 // for each, the smaller ids of the segment; ids are distinct, so the ranks
 // are a permutation); longer ones fall back to an insertion sort by lane 0.
-__global__ void k_sort_segments(const int *__restrict__ offsets, int64_t N, int *__restrict__ perm) {
+static __global__ void k_sort_segments(const int *__restrict__ offsets, int64_t N, int *__restrict__ perm) {
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
   constexpr int PER = 4;
   for (int64_t n = blockIdx.x * (int64_t)wpb + (threadIdx.x >> 5); n < N;
@@ -289,7 +292,7 @@ __device__ __forceinline__ float rbf_val(float d, int k, const Layout &y, float 
 // registers, reading each w_rad[k][c'] once and four basis values per
 // shared-memory load.
 constexpr int GATE_EDGES = 32;
-__global__ void k_edge_gate(Layout y, float cutoff, int M, const float *__restrict__ geo,
+static __global__ void k_edge_gate(Layout y, float cutoff, int M, const float *__restrict__ geo,
                             const float *__restrict__ w_rad, const float *__restrict__ b_rad,
                             float *__restrict__ gate) {
   extern __shared__ float4 phi4[];  // [nr][GATE_EDGES / 4]
@@ -1056,7 +1059,7 @@ __global__ void k_pack_weights(Layout y, BlockOffsets bo, const TW *__restrict__
 
 // d(stacked) -> packed gradient blocks: W0 directly; for g >= 1
 // grad W1 = A + D, grad W2 = C - B where d(stacked) = [[A, B], [C, D]].
-__global__ void k_unstack_grad(Layout y, BlockOffsets bo, const float *__restrict__ dws,
+static __global__ void k_unstack_grad(Layout y, BlockOffsets bo, const float *__restrict__ dws,
                                float *__restrict__ grad_w) {
   const int g = blockIdx.y;
   if (g >= y.ng) return;
@@ -1287,7 +1290,7 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
 // in registers and reads each product once.  Stage 2 adds the blocks in
 // order.
 constexpr int RAD_TILE = 64;
-__global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__restrict__ geo,
+static __global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__restrict__ geo,
                               const float *__restrict__ Ag, const float *__restrict__ Bg,
                               const float *__restrict__ omega, float *__restrict__ part) {
   extern __shared__ float phi[];  // [2][RAD_TILE][nr]
@@ -1334,7 +1337,7 @@ __global__ void k_rad_partial(Layout y, float cutoff, int M, const float *__rest
 // Stage 2: block = 32 consecutive (k, c') entries x 8 warps; each warp sums a
 // strided share of the blocks' partials, then the 8 shares are added in a
 // fixed order.
-__global__ void k_rad_reduce(Layout y, int nblk, const float *__restrict__ part,
+static __global__ void k_rad_reduce(Layout y, int nblk, const float *__restrict__ part,
                              float *__restrict__ grad_w_rad, float *__restrict__ grad_b) {
   __shared__ float red[8][32];
   const int P = (y.nr + 1) * y.co;
@@ -1364,7 +1367,7 @@ __global__ void k_rad_reduce(Layout y, int nblk, const float *__restrict__ part,
 // dd = r_hat . gg_r and dg[c'] = dd * sum_k W_rad[k][c'] phi'_k(d).
 // omega[i] = (w_x, w_y, dd, 0).  One warp per edge.
 // ---------------------------------------------------------------------------
-__global__ void k_edge_omega(Layout y, float cutoff, int M, const EdgeRec *__restrict__ rec,
+static __global__ void k_edge_omega(Layout y, float cutoff, int M, const EdgeRec *__restrict__ rec,
                              const float *__restrict__ geo, const float *__restrict__ gg_r,
                              const float *__restrict__ w_rad, float *__restrict__ omega,
                              float *__restrict__ dgate) {
@@ -1519,34 +1522,51 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
 // order); each side adds R^T of its share onto d_edge_vec[eid].
 // ---------------------------------------------------------------------------
 
-// (J_x c)[m], (J_y c)[m] and the second-order (J_x J_x c)[m], (J_y J_y c)[m],
-// ((J_x J_y + J_y J_x) c)[m] for one degree-l coefficient vector given by
-// its accessor (zero outside |q| <= l).
-template <typename F>
-__device__ __forceinline__ void gen_xy2(int l, int m, F c, float &jx, float &jy, float &xx,
-                                        float &yy, float &sym) {
-  auto cc = [&](int q) { return (q < -l || q > l) ? 0.f : c(q); };
-  gen_xy(l, m, cc, jx, jy);
-  auto jxc = [&](int q) {
-    if (q < -l || q > l) return 0.f;
-    float a, b;
-    gen_xy(l, q, cc, a, b);
-    return a;
-  };
-  auto jyc = [&](int q) {
-    if (q < -l || q > l) return 0.f;
-    float a, b;
-    gen_xy(l, q, cc, a, b);
-    return b;
-  };
-  float yx, xy;
-  gen_xy(l, m, jxc, xx, yx);  // xx = J_x J_x c, yx = J_y J_x c
-  gen_xy(l, m, jyc, xy, yy);  // xy = J_x J_y c, yy = J_y J_y c
-  sym = xy + yx;
+// First- and second-order generator rows of one degree-l coefficient vector
+// (zero outside |q| <= l): for |m| <= MM, jx = (J_x c)[m], jy = (J_y c)[m],
+// xx = (J_x J_x c)[m], yy = (J_y J_y c)[m], sym = ((J_x J_y + J_y J_x) c)[m].
+// c holds rows |q| <= MM + 2 (index q + MM + 2); the first-order rows at
+// |q| <= MM + 1 are formed once and the second generator is applied to them.
+template <int MM>
+struct GenRows {
+  float jx[2 * MM + 1], jy[2 * MM + 1], xx[2 * MM + 1], yy[2 * MM + 1], sym[2 * MM + 1];
+};
+template <int MM>
+__device__ __forceinline__ void gen_rows2(int l, const float (&c)[2 * MM + 5], GenRows<MM> &o) {
+  constexpr int W1 = MM + 1, W2 = MM + 2;
+  auto cc = [&](int q) { return (q < -l || q > l || q < -W2 || q > W2) ? 0.f : c[q + W2]; };
+  float fx[2 * W1 + 1], fy[2 * W1 + 1];
+#pragma unroll
+  for (int q = -W1; q <= W1; ++q) {
+    fx[q + W1] = 0.f;
+    fy[q + W1] = 0.f;
+    if (q >= -l && q <= l) gen_xy(l, q, cc, fx[q + W1], fy[q + W1]);
+  }
+  auto ax = [&](int q) { return (q < -l || q > l || q < -W1 || q > W1) ? 0.f : fx[q + W1]; };
+  auto ay = [&](int q) { return (q < -l || q > l || q < -W1 || q > W1) ? 0.f : fy[q + W1]; };
+#pragma unroll
+  for (int m = -MM; m <= MM; ++m) {
+    o.jx[m + MM] = fx[m + W1];
+    o.jy[m + MM] = fy[m + W1];
+    float yx = 0.f, xy = 0.f;
+    o.xx[m + MM] = 0.f;
+    o.yy[m + MM] = 0.f;
+    if (m >= -l && m <= l) {
+      gen_xy(l, m, ax, o.xx[m + MM], yx);  // J_x J_x c, J_y J_x c
+      gen_xy(l, m, ay, xy, o.yy[m + MM]);  // J_x J_y c, J_y J_y c
+    }
+    o.sym[m + MM] = xy + yx;
+  }
 }
 
 __device__ __forceinline__ float comp4(const float4 &v, int k) {
   return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
+}
+__device__ __forceinline__ void acc4(float4 &v, int k, float a) {
+  if (k == 0) v.x += a;
+  else if (k == 1) v.y += a;
+  else if (k == 2) v.z += a;
+  else v.w += a;
 }
 
 // The edge-frame share q (3 floats, summed over the warp) rotated back and
@@ -1612,7 +1632,7 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
         gpp4.z += wk.z * p2;
         gpp4.w += wk.w * p2;
       }
-      float Gg[4] = {0.f, 0.f, 0.f, 0.f}, Ggt[4] = {0.f, 0.f, 0.f, 0.f};
+      float4 Gg = make_float4(0.f, 0.f, 0.f, 0.f), Ggt = Gg;
       each_level<LC>(y.L, [&](auto lv) {
         constexpr int l = decltype(lv)::value;
         constexpr int w = 2 * l + 1;
@@ -1633,22 +1653,25 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
             b[m + W2].w += dv * gx.w;
           }
         }
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+          float bk[2 * W2 + 1];
 #pragma unroll
-        for (int m = -mm; m <= mm; ++m) {
-          int g, j;
-          lm_group_row(y, l, m, g, j);
-          const int64_t col = ro + y.kout_off[g] + j * y.co + c;
-          const float4 v4 = load4(V + col);
-          const float4 dv4 = dV ? load4(dV + col) : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4 vt4 = Vt ? load4(Vt + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int q = 0; q < 2 * W2 + 1; ++q) bk[q] = comp4(b[q], k);
+          GenRows<MM> gr2;
+          gen_rows2<MM>(l, bk, gr2);
+          const float gk = comp4(g4, k), gpk = comp4(gp4, k);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            auto bk = [&](int q) { return (q < -mb || q > mb) ? 0.f : comp4(b[q + W2], k); };
-            float jx, jy, xx, yy, sym;
-            gen_xy2(l, m, bk, jx, jy, xx, yy, sym);
-            const float bm = comp4(b[m + W2], k);
-            const float v = comp4(v4, k), dvv = comp4(dv4, k), vt = comp4(vt4, k);
-            const float gk = comp4(g4, k), gpk = comp4(gp4, k);
+          for (int m = -mm; m <= mm; ++m) {
+            int g, j;
+            lm_group_row(y, l, m, g, j);
+            const int64_t col = ro + y.kout_off[g] + j * y.co + c;
+            const float v = comp4(load4(V + col), k);
+            const float dvv = dV ? comp4(load4(dV + col), k) : 0.f;
+            const float vt = Vt ? comp4(load4(Vt + col), k) : 0.f;
+            const float jx = gr2.jx[m + MM], jy = gr2.jy[m + MM];
+            const float xx = gr2.xx[m + MM], yy = gr2.yy[m + MM], sym = gr2.sym[m + MM];
+            const float bm = bk[m + W2];
             const float gv = gk * v, gpv = gpk * v;
             const float ob = al * jx + be * jy;  // (Omega_u b)[m]
             const float xxb = Uz * inv * inv * jy - 0.5f * al * inv * sym - be * inv * yy;
@@ -1656,8 +1679,8 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
             qz += -inv * ob * gv + ob * gpv + gpk * bm * dvv;
             qx += xxb * gv - inv * jy * (gk * dvv + Uz * gpv);
             qy += xyb * gv + inv * jx * (gk * dvv + Uz * gpv);
-            Gg[k] += bm * v;
-            Ggt[k] += bm * vt;
+            acc4(Gg, k, bm * v);
+            acc4(Ggt, k, bm * vt);
             hx += gk * vt * jx;
             hy += gk * vt * jy;
           }
@@ -1665,10 +1688,10 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
       });
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float gpk = comp4(gp4, k), gppk = comp4(gpp4, k);
-        qz += Uz * gppk * Gg[k] + gpk * Ggt[k];
-        qx += Ux * inv * gpk * Gg[k];
-        qy += Uy * inv * gpk * Gg[k];
+        const float gpk = comp4(gp4, k), gppk = comp4(gpp4, k), ggk = comp4(Gg, k);
+        qz += Uz * gppk * ggk + gpk * comp4(Ggt, k);
+        qx += Ux * inv * gpk * ggk;
+        qy += Uy * inv * gpk * ggk;
       }
     }
     for (int o = 16; o > 0; o >>= 1) {
@@ -1739,21 +1762,28 @@ __global__ void __launch_bounds__(256, LC >= 0 ? SO2_ET_MINB_LC : SO2_GATHER_MIN
             at[m + W2].w += dv * tv.w;
           }
         }
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+          float ak[2 * W2 + 1], tk[2 * W2 + 1];
 #pragma unroll
-        for (int m = -mm; m <= mm; ++m) {
-          int g, j;
-          lm_group_row(y, l, m, g, j);
-          const int64_t col = ro + y.kin_off[g] + j * y.ci + c;
-          const float4 ga4 = load4(Ga + col);
-          const float4 mp4 = MP ? load4(MP + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int q = 0; q < 2 * W2 + 1; ++q) {
+            ak[q] = comp4(a[q], k);
+            tk[q] = comp4(at[q], k);
+          }
+          GenRows<MM> ga2;
+          gen_rows2<MM>(l, ak, ga2);
+          auto tq = [&](int q) { return (q < -mb || q > mb) ? 0.f : tk[q + W2]; };
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            auto ak = [&](int q) { return (q < -mb || q > mb) ? 0.f : comp4(a[q + W2], k); };
-            auto tk = [&](int q) { return (q < -mb || q > mb) ? 0.f : comp4(at[q + W2], k); };
-            float jx, jy, xx, yy, sym, tx, ty;
-            gen_xy2(l, m, ak, jx, jy, xx, yy, sym);
-            gen_xy(l, m, tk, tx, ty);
-            const float ga = comp4(ga4, k), mpv = comp4(mp4, k);
+          for (int m = -mm; m <= mm; ++m) {
+            int g, j;
+            lm_group_row(y, l, m, g, j);
+            const int64_t col = ro + y.kin_off[g] + j * y.ci + c;
+            const float ga = comp4(load4(Ga + col), k);
+            const float mpv = MP ? comp4(load4(MP + col), k) : 0.f;
+            float tx, ty;
+            gen_xy(l, m, tq, tx, ty);
+            const float jx = ga2.jx[m + MM], jy = ga2.jy[m + MM];
+            const float xx = ga2.xx[m + MM], yy = ga2.yy[m + MM], sym = ga2.sym[m + MM];
             const float oa = al * jx + be * jy;  // (Omega_u a)[m]
             const float xxa = Uz * inv * inv * jy - 0.5f * al * inv * sym - be * inv * yy;
             const float xya = -Uz * inv * inv * jx + al * inv * xx + 0.5f * be * inv * sym;

@@ -7,6 +7,8 @@
 #include <mutex>
 #include <vector>
 
+#include "dbl_terms.h"
+#include "dispatch.cuh"
 #include "edge_kernels.cuh"
 #include "gemm_tc.cuh"
 
@@ -309,34 +311,6 @@ int grid_for(int64_t n, int block) {
   if (g > 148 * 16) g = 148 * 16;
   return static_cast<int>(g);
 }
-
-// Common shapes get kernels with lmax fixed at compile time (LC), the rest
-// the generic ones (LC = -1).
-#define DISPATCH_LM(L_, mm, ...)                                        \
-  if ((L_) == 4 && (mm) == 2) {                                         \
-    constexpr int MM = 2, LC = 4;                                       \
-    __VA_ARGS__;                                                        \
-  } else if ((L_) == 6 && (mm) == 2) {                                  \
-    constexpr int MM = 2, LC = 6;                                       \
-    __VA_ARGS__;                                                        \
-  } else if ((L_) == 2 && (mm) == 2) {                                  \
-    constexpr int MM = 2, LC = 2;                                       \
-    __VA_ARGS__;                                                        \
-  } else {                                                              \
-    constexpr int LC = -1;                                              \
-    DISPATCH_MM(mm, __VA_ARGS__);                                       \
-  }
-
-#define DISPATCH_MM(mm, ...)                  \
-  switch (mm) {                               \
-    case 0: { constexpr int MM = 0; __VA_ARGS__; } break; \
-    case 1: { constexpr int MM = 1; __VA_ARGS__; } break; \
-    case 2: { constexpr int MM = 2; __VA_ARGS__; } break; \
-    case 3: { constexpr int MM = 3; __VA_ARGS__; } break; \
-    case 4: { constexpr int MM = 4; __VA_ARGS__; } break; \
-    case 5: { constexpr int MM = 5; __VA_ARGS__; } break; \
-    default: { constexpr int MM = 6; __VA_ARGS__; } break; \
-  }
 
 // Raise the dynamic shared memory limit of a kernel (once per kernel).
 template <typename K>
@@ -1377,20 +1351,9 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
         ProfScope ps(5, c.s);
         const float *Gap = prows(c, P.Ga, (size_t)ch * y.KA);
         const float *MPp = has_r ? prows(c, P.Ga, 0) : nullptr;
-        const int sm = 8 * y.dsz * 4;
-#define SO2_HIN_LAUNCH(TX, TF)                                                                 \
-  DISPATCH_LM(y.L, y.mmax, constexpr int LE = (LC >= 0 && LC <= 4) ? LC : -1;                   \
-              k_edge_hess_in<TX, MM, LE, TF><<<warp_grid(M, 8), 256, sm, c.s>>>(                \
-                  y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), at<float>(ws, P.geo),       \
-                  static_cast<const TX *>(x), gg_x, has_r ? omega : nullptr,                    \
-                  reinterpret_cast<const TF *>(Gap), reinterpret_cast<const TF *>(MPp),          \
-                  d_edge_vec);)
-        if (P.xbf16) {
-          SO2_HIN_LAUNCH(__nv_bfloat16, __nv_bfloat16)
-        } else {
-          SO2_HIN_LAUNCH(float, float)
-        }
-#undef SO2_HIN_LAUNCH
+        CK(launch_hess_in(y, warp_grid(M, 8), M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
+                          at<float>(ws, P.geo), x, P.xbf16, gg_x, has_r ? omega : nullptr, Gap,
+                          MPp, !P.split, d_edge_vec, c.s));
         CKL();
       }
     }
@@ -1442,41 +1405,19 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
       }
       if (d_edge_vec) {
         ProfScope ps(5, c.s);
-        const int sm = 8 * (y.dsz + 2 * RAD_MAX_NR) * 4;
-#define SO2_HOUT_LAUNCH(TF)                                                                    \
-  DISPATCH_LM(y.L, y.mmax, constexpr int LE = (LC >= 0 && LC <= 4) ? LC : -1;                   \
-              k_edge_hess_out<MM, LE, TF><<<warp_grid(M, 8), 256, sm, c.s>>>(                   \
-                  y, desc->rbf_cutoff, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),           \
-                  at<float>(ws, P.geo), at<float>(ws, P.gate), grad_out,                       \
-                  has_r ? omega : nullptr, reinterpret_cast<const TF *>(V),                    \
-                  has_r ? reinterpret_cast<const TF *>(dV) : nullptr,                          \
-                  has_x ? reinterpret_cast<const TF *>(Vt) : nullptr, prm.w_rad, d_edge_vec);)
-        if (P.split) {
-          SO2_HOUT_LAUNCH(float)
-        } else {
-          SO2_HOUT_LAUNCH(__nv_bfloat16)
-        }
-#undef SO2_HOUT_LAUNCH
+        CK(launch_hess_out(y, desc->rbf_cutoff, warp_grid(M, 8), M, at<EdgeRec>(ws, P.rec),
+                           at<float>(ws, P.D), at<float>(ws, P.geo), at<float>(ws, P.gate),
+                           grad_out, has_r ? omega : nullptr, V, has_r ? dV : nullptr,
+                           has_x ? Vt : nullptr, !P.split, prm.w_rad, d_edge_vec, c.s));
         CKL();
       }
       if (d_w_rad || d_b_rad) {
         {
           ProfScope ps(5, c.s);
-#define SO2_ET2_LAUNCH(TF)                                                                     \
-  DISPATCH_LM(y.L, y.mmax,                                                                     \
-              (k_edge_terms2<MM, ((LC >= 0 && LC <= 4) ? LC : -1), TF>                          \
-               <<<warp_grid(M, 8), 256, 8 * y.dsz * 4, c.s>>>(                                   \
-                   y, M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D), grad_out,                  \
-                   has_r ? omega : nullptr, reinterpret_cast<const TF *>(V),                    \
-                   has_r ? reinterpret_cast<const TF *>(dV) : nullptr,                          \
-                   has_x ? reinterpret_cast<const TF *>(Vt) : nullptr, at<float>(ws, P.tA),     \
-                   at<float>(ws, P.tB))))
-          if (P.split) {
-            SO2_ET2_LAUNCH(float);
-          } else {
-            SO2_ET2_LAUNCH(__nv_bfloat16);
-          }
-#undef SO2_ET2_LAUNCH
+          CK(launch_edge_terms2(y, warp_grid(M, 8), M, at<EdgeRec>(ws, P.rec), at<float>(ws, P.D),
+                              grad_out, has_r ? omega : nullptr, V, has_r ? dV : nullptr,
+                              has_x ? Vt : nullptr, !P.split, at<float>(ws, P.tA),
+                              at<float>(ws, P.tB), c.s));
           CKL();
         }
         if ((r = rad_grads(c, M, at<float>(ws, P.tA), has_r ? at<float>(ws, P.tB) : nullptr,
