@@ -441,12 +441,31 @@ def run_ours(args, world, rank, local):
         step = make_dst_step(sg, desc)
         ws = None  # the sharded calls use the binding's own per-device workspace
 
+    torch.cuda.synchronize()
+    resident = torch.cuda.memory_allocated(dev)  # inputs, flush buffer (before any step)
+    torch.cuda.reset_peak_memory_stats(dev)
     for _ in range(max(args.warmup, 3)):
         step(d)
     torch.cuda.synchronize()
     st = B.check(dev, ws)
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
+    # device memory: the library's workspace per call (sized by the ABI) and the
+    # peak torch allocation of a step above what was resident before it (the
+    # workspace, the outputs and, for --split dst, the gathered node arrays)
+    if args.config == "block":
+        ws_sizes = {"block_forward": B.block_workspace_size(desc, int(d["x"].shape[0]), E, 0),
+                    "block_backward": B.block_workspace_size(desc, int(d["x"].shape[0]), E, 1)}
+    else:
+        n_call = sg.n_pad if sg is not None else p.n_nodes
+        ws_sizes = {k: B.workspace_size(desc, n_call, E, w) for k, w in
+                    (("forward", B.WS_FORWARD), ("backward", B.WS_BACKWARD),
+                     ("double_backward", B.WS_DOUBLE_BACKWARD))}
+    memory = {"workspace_bytes": ws_sizes,
+              "peak_step_bytes_above_inputs": int(torch.cuda.max_memory_allocated(dev) - resident),
+              "chunk_edges": int(B.load().so2conv_max_chunk_edges()),
+              "note": "no tensor of E x (lmax+1)^2 x C is allocated; per-edge intermediates "
+                      "live in the workspace for one chunk of edges at a time"}
 
     # ---- device-resident timed region ----
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -612,7 +631,8 @@ def run_ours(args, world, rank, local):
                                            else f"replicas x{world}" if world > 1 else "single")},
                 "step_roofline_frac": roofline["step_roofline_frac"],
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches, "clocks": clk, "breakdown_ms_per_step": breakdown}
+                "gpu_launches": launches, "clocks": clk, "breakdown_ms_per_step": breakdown,
+                "memory": memory}
         print(json.dumps(line), flush=True)
 
 
