@@ -100,3 +100,24 @@ def test_status_strings(lib):
     for code in range(8):
         s = lib.so2conv_status_string(code)
         assert s and len(s) > 1
+
+
+def test_block_argument_errors_are_reported_before_any_launch(lib):
+    # (never dereferenced) the block's checks run before any CUDA call
+    P = ctypes.c_void_p(0x1000)
+    good = B.Params(0x1000, 0x1000, 0x1000)
+
+    def fwd(desc, p2=good, nbytes=1 << 40, x=P):
+        return lib.so2conv_block_forward(ctypes.byref(desc), 4, 3, x, P, P, good, p2,
+                                         ctypes.c_void_p(0x2000), ctypes.c_void_p(0x100000),
+                                         nbytes, None)
+    d = B.make_desc(2, 2, 16, 16, 8, 5.0)
+    assert fwd(B.make_desc(2, 2, 16, 32, 8, 5.0)) == 2        # the block keeps one C
+    assert fwd(B.make_desc(7, 2, 16, 16, 8, 5.0)) == 2        # lmax > 6
+    assert fwd(d, p2=B.Params(0, 0x1000, 0x1000)) == 1        # second conv's weights
+    assert fwd(d, x=None) == 1
+    assert fwd(d, nbytes=B.block_workspace_size(d, 4, 3, 0) - 1) == 3
+    # the block's workspace holds the single convolution's and more
+    assert B.block_workspace_size(d, 4, 3, 0) > B.workspace_size(d, 4, 3, B.WS_FORWARD)
+    assert B.block_workspace_size(d, 4, 3, 1) > B.workspace_size(d, 4, 3, B.WS_BACKWARD)
+    assert B.block_workspace_size(d, 4, 3, 2) == 0

@@ -81,3 +81,35 @@ def test_block_parity(name, kw):
 def test_block_rejects_unequal_channels():
     desc = B.make_desc(2, 2, 16, 32, 8, 5.0)
     assert B.block_workspace_size(desc, 10, 20, 0) == 0
+
+
+def test_block_lmax6_and_empty_graphs():
+    t = lambda a, d=torch.float32: torch.as_tensor(np.asarray(a)).to(d).to(DEV)  # noqa: E731
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
+    # lmax 6, mmax 3: the runtime-degree kernels and every m group
+    p, w2, wr2, b2 = _case(L=6, M=3, C=32, n=60, nb=10, seed=8)
+    desc = B.make_desc(p.lmax, p.mmax, p.c_in, p.c_out, p.n_rbf, p.rbf_cutoff)
+    args = (t(p.x), t(p.edge_index, torch.int64), t(p.edge_vec), t(p.w), t(p.w_rad),
+            t(p.b_rad), t(w2), t(wr2), t(b2))
+    out = B.block_forward(desc, *args)
+    g = B.block_backward(desc, *args, t(p.grad_out))
+    torch.cuda.synchronize()
+    assert B.check(DEV) == 0
+    oargs = (T(p.x), T(p.edge_index[0]), T(p.edge_index[1]), T(p.edge_vec), T(p.w), T(p.w_rad),
+             T(p.b_rad), T(w2), T(wr2), T(b2), desc_of(p))
+    assert rel_err(out, O.block_forward(*oargs)) < 1e-4
+    ref = O.block_backward(*oargs, T(p.grad_out))
+    for k in B.BLOCK_GRADS:
+        assert rel_err(g[k], ref[k]) < 1e-4, k
+    # no edges: zero output and zero gradients, nothing launched on the edges
+    ei0 = torch.zeros((2, 0), dtype=torch.int64, device=DEV)
+    ev0 = torch.zeros((0, 3), dtype=torch.float32, device=DEV)
+    a0 = (args[0], ei0, ev0) + args[3:]
+    out0 = B.block_forward(desc, *a0)
+    g0 = B.block_backward(desc, *a0, t(p.grad_out))
+    torch.cuda.synchronize()
+    assert B.check(DEV) == 0
+    assert out0.abs().max().item() == 0.0
+    for k in B.BLOCK_GRADS:
+        if g0[k].numel():
+            assert g0[k].abs().max().item() == 0.0, k
