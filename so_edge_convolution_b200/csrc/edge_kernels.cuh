@@ -336,13 +336,6 @@ __device__ __forceinline__ float2 load2(const float *p) { return *reinterpret_ca
 __device__ __forceinline__ float2 load2(const __nv_bfloat16 *p) {
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
 }
-__device__ __forceinline__ void store_split2(__nv_bfloat16 *hi, __nv_bfloat16 *lo, float a, float b) {
-  __nv_bfloat16 h0, l0, h1, l1;
-  split_bf16(a, h0, l0);
-  split_bf16(b, h1, l1);
-  *reinterpret_cast<__nv_bfloat162 *>(hi) = __halves2bfloat162(h0, h1);
-  if (lo) *reinterpret_cast<__nv_bfloat162 *>(lo) = __halves2bfloat162(l0, l1);
-}
 
 // Per-channel coefficient: 0 (absent), 1, or an [edge][channel] array.
 struct Coef {

@@ -1,7 +1,8 @@
 // so2conv_api.cu -- host side of libso2conv: argument checks, workspace plan,
 // tensor maps and the launch sequence of forward / backward / double
-// backward.  Every step runs in this library's own kernels; the host only
-// orchestrates on the caller's stream.
+// backward and of the message block.  Every step runs in this library's own
+// kernels (the double backward's per-edge terms in so2conv_dbl_terms.cu);
+// the host only orchestrates on the caller's stream.
 #include <cstdio>
 #include <cstring>
 #include <mutex>
