@@ -309,6 +309,7 @@ static __global__ void k_edge_gate(Layout y, float cutoff, int M, const float *_
     const float b = b_rad[c];
 #pragma unroll
     for (int i = 0; i < GATE_EDGES; ++i) acc[i] = b;
+#pragma unroll 4
     for (int k = 0; k < y.nr; ++k) {
       const float w = w_rad[k * y.co + c];
 #pragma unroll
@@ -1307,9 +1308,7 @@ static __global__ void k_rad_partial(Layout y, float cutoff, int M, const float 
       float acc[16], bias = 0.f;
 #pragma unroll
       for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-      for (int i = 0; i < n; ++i) {
-        const float a = Ag[(int64_t)(i0 + i) * y.co + c];
-        const float b = Bg ? Bg[(int64_t)(i0 + i) * y.co + c] : 0.f;
+      auto add = [&](int i, float a, float b) {
         bias += a;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -1318,7 +1317,21 @@ static __global__ void k_rad_partial(Layout y, float cutoff, int M, const float 
             if (Bg) acc[k] += dphi[i * y.nr + k0 + k] * b;
           }
         }
+      };
+      // four edges' loads in flight before their (in-order) sums
+      int i = 0;
+      for (; i + 4 <= n; i += 4) {
+        float a[4], b[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          a[u] = Ag[(int64_t)(i0 + i + u) * y.co + c];
+          b[u] = Bg ? Bg[(int64_t)(i0 + i + u) * y.co + c] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) add(i + u, a[u], b[u]);
       }
+      for (; i < n; ++i)
+        add(i, Ag[(int64_t)(i0 + i) * y.co + c], Bg ? Bg[(int64_t)(i0 + i) * y.co + c] : 0.f);
 #pragma unroll
       for (int k = 0; k < 16; ++k)
         if (k0 + k < y.nr) part[(int64_t)blockIdx.x * P + (k0 + k) * y.co + c] = acc[k];
@@ -1327,23 +1340,27 @@ static __global__ void k_rad_partial(Layout y, float cutoff, int M, const float 
   }
 }
 
-// Stage 2: block = 32 consecutive (k, c') entries x 8 warps; each warp sums a
-// strided share of the blocks' partials, then the 8 shares are added in a
-// fixed order.
-static __global__ void k_rad_reduce(Layout y, int nblk, const float *__restrict__ part,
-                             float *__restrict__ grad_w_rad, float *__restrict__ grad_b) {
-  __shared__ float red[8][32];
+// Stage 2: block = 32 consecutive (k, c') entries x RAD_RED_WARPS warps; each
+// warp sums a strided share of the blocks' partials (four loads in flight),
+// then the shares are added in a fixed order.
+constexpr int RAD_RED_WARPS = 32;
+static __global__ void __launch_bounds__(32 * RAD_RED_WARPS)
+    k_rad_reduce(Layout y, int nblk, const float *__restrict__ part,
+                 float *__restrict__ grad_w_rad, float *__restrict__ grad_b) {
+  __shared__ float red[RAD_RED_WARPS][32];
   const int P = (y.nr + 1) * y.co;
   const int pidx = blockIdx.x * 32 + (threadIdx.x & 31);
   const int w = threadIdx.x >> 5;
   float s = 0.f;
-  if (pidx < P)
-    for (int b = w; b < nblk; b += 8) s += part[(int64_t)b * P + pidx];
+  if (pidx < P) {
+#pragma unroll 4
+    for (int b = w; b < nblk; b += RAD_RED_WARPS) s += part[(int64_t)b * P + pidx];
+  }
   red[w][threadIdx.x & 31] = s;
   __syncthreads();
   if (w == 0 && pidx < P) {
     float t = 0.f;
-    for (int u = 0; u < 8; ++u) t += red[u][threadIdx.x];
+    for (int u = 0; u < RAD_RED_WARPS; ++u) t += red[u][threadIdx.x];
     const int k = pidx / y.co, c = pidx % y.co;
     if (k < y.nr) {
       if (grad_w_rad) grad_w_rad[k * y.co + c] += t;

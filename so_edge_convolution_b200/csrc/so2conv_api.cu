@@ -333,6 +333,11 @@ bool allow_smem(K kernel, int bytes) {
 #define SO2_PAIR_MN 1
 #endif
 
+// Blocks per weight group of the packing and unstacking kernels: enough that
+// each thread handles a few elements (their loops are load-latency bound).
+constexpr int PACK_BLOCKS = 1024;
+constexpr int UNSTACK_BLOCKS = 512;
+
 int warp_grid(int M, int warps_per_block) {
   int g = (M + warps_per_block - 1) / warps_per_block;
   if (g < 1) g = 1;
@@ -583,7 +588,7 @@ so2_status pack_weights(Ctx &c, const void *w, bool transposes) {
     CK(cudaMemsetAsync(th, 0, 2ull * y.WTR * y.WTK, c.s));
     if (tl) CK(cudaMemsetAsync(tl, 0, 2ull * y.WTR * y.WTK, c.s));
   }
-  dim3 grid(256, y.ng);
+  dim3 grid(PACK_BLOCKS, y.ng);
   BlockOffsets bo = block_offsets(y);
   for (int t = 0; t < (transposes ? 2 : 1); ++t) {
     __nv_bfloat16 *h = t ? th : wh, *l = t ? tl : wl;
@@ -893,8 +898,8 @@ so2_status rad_grads(Ctx &c, int M, const float *Ag, const float *Bg, const floa
                                         omega, at<float>(c.ws, P.radp));
   CKL();
   const int Pn = (y.nr + 1) * y.co;
-  k_rad_reduce<<<(Pn + 31) / 32, 256, 0, c.s>>>(y, nblk, at<float>(c.ws, P.radp), grad_w_rad,
-                                                 grad_b);
+  k_rad_reduce<<<(Pn + 31) / 32, 32 * RAD_RED_WARPS, 0, c.s>>>(y, nblk, at<float>(c.ws, P.radp),
+                                                                grad_w_rad, grad_b);
   CKL();
   return SO2_OK;
 }
@@ -1258,7 +1263,8 @@ so2_status so2conv_backward(const so2conv_desc *desc, int64_t N, int64_t E, cons
   }
   if (grad_w) {
     ProfScope ps(7, c.s);
-    k_unstack_grad<<<dim3(64, y.ng), 256, 0, c.s>>>(y, block_offsets(y), dws, grad_w);
+    k_unstack_grad<<<dim3(UNSTACK_BLOCKS, y.ng), 256, 0, c.s>>>(y, block_offsets(y), dws,
+                                                             grad_w);
     CKL();
   }
   return SO2_OK;
@@ -1449,7 +1455,7 @@ so2_status so2conv_double_backward(const so2conv_desc *desc, int64_t N, int64_t 
   }
   if (d_w) {
     ProfScope ps(7, c.s);
-    k_unstack_grad<<<dim3(64, y.ng), 256, 0, c.s>>>(y, block_offsets(y), dws, d_w);
+    k_unstack_grad<<<dim3(UNSTACK_BLOCKS, y.ng), 256, 0, c.s>>>(y, block_offsets(y), dws, d_w);
     CKL();
   }
   return SO2_OK;
@@ -1599,13 +1605,13 @@ so2_status so2conv_block_backward(const so2conv_desc *desc, int64_t N, int64_t E
   }
   ProfScope ps(7, s);
   if (grad_w1) {
-    k_unstack_grad<<<dim3(64, y.ng), 256, 0, s>>>(y, block_offsets(y), at<float>(ws, c1.P.dws),
-                                                   grad_w1);
+    k_unstack_grad<<<dim3(UNSTACK_BLOCKS, y.ng), 256, 0, s>>>(
+        y, block_offsets(y), at<float>(ws, c1.P.dws), grad_w1);
     CKL();
   }
   if (grad_w2) {
-    k_unstack_grad<<<dim3(64, y.ng), 256, 0, s>>>(y, block_offsets(y), at<float>(ws, c2.P.dws),
-                                                   grad_w2);
+    k_unstack_grad<<<dim3(UNSTACK_BLOCKS, y.ng), 256, 0, s>>>(
+        y, block_offsets(y), at<float>(ws, c2.P.dws), grad_w2);
     CKL();
   }
   return SO2_OK;
