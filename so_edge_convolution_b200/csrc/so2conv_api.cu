@@ -333,9 +333,8 @@ bool allow_smem(K kernel, int bytes) {
 #define SO2_PAIR_MN 1
 #endif
 
-// Blocks per weight group of the packing and unstacking kernels: enough that
-// each thread handles a few elements (their loops are load-latency bound).
-constexpr int PACK_BLOCKS = 1024;
+// Blocks per weight group of the gradient unstacking: enough that each
+// thread handles a few elements (its loop is load-latency bound).
 constexpr int UNSTACK_BLOCKS = 512;
 
 int warp_grid(int M, int warps_per_block) {
@@ -588,7 +587,7 @@ so2_status pack_weights(Ctx &c, const void *w, bool transposes) {
     CK(cudaMemsetAsync(th, 0, 2ull * y.WTR * y.WTK, c.s));
     if (tl) CK(cudaMemsetAsync(tl, 0, 2ull * y.WTR * y.WTK, c.s));
   }
-  dim3 grid(PACK_BLOCKS, y.ng);
+  dim3 grid(256, y.ng);
   BlockOffsets bo = block_offsets(y);
   for (int t = 0; t < (transposes ? 2 : 1); ++t) {
     __nv_bfloat16 *h = t ? th : wh, *l = t ? tl : wl;

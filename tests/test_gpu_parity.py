@@ -64,21 +64,24 @@ def _lib():
 
 
 # ---------------------------------------------------------------------------
-def test_frames_and_wigner_d():
+@pytest.mark.parametrize("lmax", [2, 4, 6])
+def test_frames_and_wigner_d(lmax):
+    # lmax <= 4 runs the register-carried recursion, lmax 6 the one that reads
+    # each previous block back from shared memory
     rng = np.random.default_rng(0)
     v = rng.standard_normal((500, 3)) * 3
     v[:6] = [[0, 0, 2], [0, 0, -2], [1, 0, 0], [0, 1e-7, -1], [1e-6, 0, 1], [0, -3, 0]]
     ev = torch.tensor(v, dtype=torch.float32, device=DEV)
-    R, D = B.edge_frames(6, ev)
+    R, D = B.edge_frames(lmax, ev)
     R64 = R.double().cpu()
     rh = torch.tensor(v / np.linalg.norm(v, axis=1, keepdims=True))
     z = torch.einsum("eij,ej->ei", R64, rh)
     assert (z - torch.tensor([0, 0, 1.0], dtype=torch.float64)).abs().max() < 2e-6
     eye = torch.eye(3, dtype=torch.float64)
     assert (R64 @ R64.transpose(1, 2) - eye).abs().max() < 2e-6
-    ref = O.wigner_d_blocks(R64, 6)
+    ref = O.wigner_d_blocks(R64, lmax)
     off = 0
-    for l in range(7):
+    for l in range(lmax + 1):
         n = (2 * l + 1) ** 2
         got = D[:, off:off + n].double().cpu().view(-1, 2 * l + 1, 2 * l + 1)
         assert (got - ref[l]).abs().max() < 5e-6, l
