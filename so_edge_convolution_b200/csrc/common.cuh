@@ -191,6 +191,18 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr)
                : "memory");
 }
+// Arrives without release semantics, for a barrier that only orders tensor
+// memory reads already completed (tcgen05.wait::ld) before the signal: the
+// arrive then does not wait for the thread's earlier global stores and
+// atomics to be performed.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t caddr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
 // 2-D tiled TMA load into this CTA's shared memory whose completion is
 // counted on an mbarrier of the CTA pair (shared::cluster address; no
 // multicast).

@@ -29,6 +29,9 @@
 #ifndef SO2_EPI_WARPS
 #define SO2_EPI_WARPS 12
 #endif
+#ifndef SO2_EPI_RELAXED_ARRIVE
+#define SO2_EPI_RELAXED_ARRIVE 1
+#endif
 
 namespace so2 {
 
@@ -582,13 +585,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           staged = j;
         }
       }
+      // The accumulator is free once this warp's tensor-memory loads are done
+      // (tcgen05.wait::ld above); its global stores and atomics need no
+      // ordering with the next tile's MMAs, so the arrive is relaxed.
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
+#if SO2_EPI_RELAXED_ARRIVE
         if (PAIR)
-          mbar_arrive_cluster(tempty_c + 8u * acc);  // the even CTA's barrier
+          mbar_arrive_cluster_relaxed(tempty_c + 8u * acc);  // the even CTA's barrier
+        else
+          mbar_arrive_relaxed(&tempty[acc]);
+#else
+        if (PAIR)
+          mbar_arrive_cluster(tempty_c + 8u * acc);
         else
           mbar_arrive(&tempty[acc]);
+#endif
       }
     }
   }
