@@ -495,7 +495,7 @@ def run_ours(args, world, rank, local):
     ms_per_step = total_ms / args.steps
     value = E_job * args.steps / (total_ms * 1e-3)
 
-    # ---- roofline (SURVEY-style accounting: algorithmic mixing FLOPs only) ----
+    # ---- roofline (algorithmic mixing FLOPs only: the recomputed product is not counted) ----
     # The bound is the tensor-core one (compulsory bytes are ~30x below it).
     # Peaks: the burst bf16 figure applies (the timed region is ~0.1 s, not a
     # seconds-long loop); the f32 path is held against the TF32-equivalent
