@@ -155,10 +155,14 @@ __device__ __forceinline__ void epi_stage_d(const float *__restrict__ src, int n
 // with lane = channel; the warp's 32 edges split into runs of equal node (a
 // ballot finds the run starts), each summed in registers and flushed with W
 // coalesced atomics.
+// With cst, the chunk's values (ungated: S.gate is null then) are also
+// stored to rows cst + el * ldc, el < the chunk's valid rows, one 128-byte
+// row segment per store instruction, from the transposed staging.
 template <int W>
 __device__ __forceinline__ void epi_scatter_w(const GemmScatter &S, int M, int row_base, int l,
                                               int c0, const uint32_t (&r)[32],
-                                              const float *dsrc, const EpiScratch &x) {
+                                              const float *dsrc, const EpiScratch &x,
+                                              float *cst, int ldc, bool cst_lane) {
   const int lane = threadIdx.x & 31;
   const int my_key = x.keys[lane];
   __syncwarp();  // the previous chunk's reads of T and Dw are done
@@ -184,6 +188,10 @@ __device__ __forceinline__ void epi_scatter_w(const GemmScatter &S, int M, int r
   const int S_ = (S.L + 1) * (S.L + 1);
   const int prev_key = lane ? x.keys[lane - 1] : -2;
   const int nvalid = __popc(__ballot_sync(0xffffffffu, my_key >= 0));  // a prefix of the warp
+  if (cst && cst_lane) {
+#pragma unroll 4
+    for (int el = 0; el < nvalid; ++el) cst[(int64_t)el * ldc + lane] = x.T[el * 33 + lane];
+  }
   unsigned starts = __ballot_sync(0xffffffffu, my_key != prev_key && my_key >= 0);
   while (starts) {
     const int s0 = __ffs(starts) - 1;
@@ -214,15 +222,16 @@ __device__ __forceinline__ void epi_scatter_w(const GemmScatter &S, int M, int r
 
 __device__ __forceinline__ void epi_scatter_chunk(const GemmScatter &S, int M, int row_base, int l,
                                                   int c0, const uint32_t (&r)[32],
-                                                  const float *dsrc, const EpiScratch &x) {
+                                                  const float *dsrc, const EpiScratch &x,
+                                                  float *cst, int ldc, bool cst_lane) {
   switch (2 * l + 1) {
-    case 1: epi_scatter_w<1>(S, M, row_base, l, c0, r, dsrc, x); break;
-    case 3: epi_scatter_w<3>(S, M, row_base, l, c0, r, dsrc, x); break;
-    case 5: epi_scatter_w<5>(S, M, row_base, l, c0, r, dsrc, x); break;
-    case 7: epi_scatter_w<7>(S, M, row_base, l, c0, r, dsrc, x); break;
-    case 9: epi_scatter_w<9>(S, M, row_base, l, c0, r, dsrc, x); break;
-    case 11: epi_scatter_w<11>(S, M, row_base, l, c0, r, dsrc, x); break;
-    default: epi_scatter_w<13>(S, M, row_base, l, c0, r, dsrc, x); break;
+    case 1: epi_scatter_w<1>(S, M, row_base, l, c0, r, dsrc, x, cst, ldc, cst_lane); break;
+    case 3: epi_scatter_w<3>(S, M, row_base, l, c0, r, dsrc, x, cst, ldc, cst_lane); break;
+    case 5: epi_scatter_w<5>(S, M, row_base, l, c0, r, dsrc, x, cst, ldc, cst_lane); break;
+    case 7: epi_scatter_w<7>(S, M, row_base, l, c0, r, dsrc, x, cst, ldc, cst_lane); break;
+    case 9: epi_scatter_w<9>(S, M, row_base, l, c0, r, dsrc, x, cst, ldc, cst_lane); break;
+    case 11: epi_scatter_w<11>(S, M, row_base, l, c0, r, dsrc, x, cst, ldc, cst_lane); break;
+    default: epi_scatter_w<13>(S, M, row_base, l, c0, r, dsrc, x, cst, ldc, cst_lane); break;
   }
 }
 
@@ -481,6 +490,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int row = row_base + lane;
       float *Cg = p.C + G.c_off;
       int staged = -1;  // edge-frame row whose D rows are in Dw
+      // an ungated fused reduction that also stores the product (plain f32,
+      // no accumulation into C) stores it from the reduction's transposed
+      // staging, with coalesced row segments
+      const bool store_staged = SCATTER && p.scatter && p.store && !p.sc.gate && !p.cbf16 &&
+                                !p.beta && !atomic_c;
       for (int cc = half; cc < GEMM_BN / 32; cc += EPI_WARPS / 4) {
         const int col0 = n0 + cc * 32;
         if (col0 >= G.N) break;  // warp-uniform
@@ -540,7 +554,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int j = 0; j < 32 && col0 + j < G.N; ++j)
               cb[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
           }
-        } else if (p.store && row < G.M) {
+        } else if (p.store && row < G.M && !store_staged) {
           float *crow = Cg + static_cast<long long>(row) * G.ldc + col0;
           const bool vec = (col0 + 32 <= G.N) && ((reinterpret_cast<uintptr_t>(crow) & 15) == 0);
           if (atomic_c && vec) {
@@ -581,7 +595,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               j != staged ? p.sc.DT + (int64_t)kept_d_prefix(p.sc.L, G.mgroup, j) * p.sc.dt_chunk +
                                 (int64_t)row_base * (2 * l + 1)
                           : nullptr;
-          epi_scatter_chunk(p.sc, G.M, row_base, l, c0, r, dsrc, xs);
+          epi_scatter_chunk(p.sc, G.M, row_base, l, c0, r, dsrc, xs,
+                            store_staged ? Cg + static_cast<long long>(row_base) * G.ldc + col0
+                                         : nullptr,
+                            G.ldc, col0 + lane < G.N);
           staged = j;
         }
       }
