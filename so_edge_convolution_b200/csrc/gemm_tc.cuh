@@ -150,11 +150,11 @@ __device__ __forceinline__ void epi_stage_d(const float *__restrict__ src, int n
 // out[key_e][(l, m')][c], one coalesced atomic per (node run, m', c).
 // r holds one edge's 32 values per lane (lane = edge); keys must be staged;
 // with a non-null dsrc (the first edge's kept D row) the edges' D rows are
-// staged into Dw first.  Each lane scales its edge's values by the gate (8
-// vector loads of its gate row) on the way into shared memory, read back
-// with lane = channel; the warp's 32 edges split into runs of equal node (a
-// ballot finds the run starts), each summed in registers and flushed with W
-// coalesced atomics.
+// staged into Dw first.  Each lane writes its edge's values into shared
+// memory; read back with lane = channel, each lane scales its column by the
+// gate (one 128-byte gate row segment per load); the warp's 32 edges split
+// into runs of equal node (a ballot finds the run starts), each summed in
+// registers and flushed with W coalesced atomics.
 // With cst, the chunk's values (ungated: S.gate is null then) are also
 // stored to rows cst + el * ldc, el < the chunk's valid rows, one 128-byte
 // row segment per store instruction, from the transposed staging.
@@ -166,21 +166,8 @@ __device__ __forceinline__ void epi_scatter_w(const GemmScatter &S, int M, int r
   const int lane = threadIdx.x & 31;
   const int my_key = x.keys[lane];
   __syncwarp();  // the previous chunk's reads of T and Dw are done
-  if (S.gate && my_key >= 0) {
-    const float4 *gp =
-        reinterpret_cast<const float4 *>(S.gate + (int64_t)(row_base + lane) * S.C + c0);
 #pragma unroll
-    for (int k4 = 0; k4 < 8; ++k4) {
-      const float4 g = __ldg(gp + k4);
-      x.T[lane * 33 + 4 * k4 + 0] = __uint_as_float(r[4 * k4 + 0]) * g.x;
-      x.T[lane * 33 + 4 * k4 + 1] = __uint_as_float(r[4 * k4 + 1]) * g.y;
-      x.T[lane * 33 + 4 * k4 + 2] = __uint_as_float(r[4 * k4 + 2]) * g.z;
-      x.T[lane * 33 + 4 * k4 + 3] = __uint_as_float(r[4 * k4 + 3]) * g.w;
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < 32; ++k) x.T[lane * 33 + k] = __uint_as_float(r[k]);
-  }
+  for (int k = 0; k < 32; ++k) x.T[lane * 33 + k] = __uint_as_float(r[k]);
   if (dsrc) epi_stage_d<W>(dsrc, M - row_base, x);
   __syncwarp();
   // lane = channel from here on
@@ -188,6 +175,13 @@ __device__ __forceinline__ void epi_scatter_w(const GemmScatter &S, int M, int r
   const int S_ = (S.L + 1) * (S.L + 1);
   const int prev_key = lane ? x.keys[lane - 1] : -2;
   const int nvalid = __popc(__ballot_sync(0xffffffffu, my_key >= 0));  // a prefix of the warp
+  if (S.gate) {
+    // each lane scales its own channel column: one 128-byte gate row segment
+    // per load instruction
+    const float *gp = S.gate + (int64_t)row_base * S.C + c;
+#pragma unroll 8
+    for (int el = 0; el < nvalid; ++el) x.T[el * 33 + lane] *= __ldg(gp + (int64_t)el * S.C);
+  }
   if (cst && cst_lane) {
 #pragma unroll 4
     for (int el = 0; el < nvalid; ++el) cst[(int64_t)el * ldc + lane] = x.T[el * 33 + lane];
